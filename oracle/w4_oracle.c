@@ -1,0 +1,188 @@
+/*
+ * w4_oracle.c -- plain, slow, obviously-correct CPU reference for weight-only
+ * per-group INT4 (W4A16) quantize / pack / dequantize / matmul.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the test-suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code with the CUDA library.
+ *
+ * Sources (cited by page and section):
+ *   [Accel 2.1]  discosf.com "LLM inference acceleration" article, section 2.1
+ *                "what quantization actually does": an affine map of a float
+ *                range onto integers through a scale and a zero point, with
+ *                per-group granularity (e.g. 128 elements per group).
+ *   [Accel 2.2]  same article, section 2.2: INT4 cuts a 70B model from about
+ *                140 GB (FP16) to about 35 GB.
+ *   [Accel 2.3]  same article, section 2.3: scale and zero_point are loaded
+ *                together with the weights ("dequantize mapping").
+ *   [Ch22 22.3]  aiwing.uk chapter 22 "Advanced inference optimisation",
+ *                section 22.3 "Model quantization": bytes-per-parameter table
+ *                (INT4 = 0.5 B), weight-only quantization (dequantize back to
+ *                FP16 then matmul), and the AWQ equation W^ = quant(W/s) * s.
+ *
+ * Readings taken where the pages are silent (each one is exercised by a test):
+ *   - codes are asymmetric uint4 in [0,15]; one fp16 scale and one fp16 zero
+ *     point per group of G = 128 consecutive input channels (k) of a row n;
+ *   - every step runs in IEEE fp32 with round-to-nearest-even; rint() is
+ *     round-half-to-even; scale = fp16((max - min) / 15), and z and q are
+ *     computed with that fp16-rounded scale widened back to fp32, so the
+ *     stored (scale, zero) describe exactly the grid that was used;
+ *   - z = clamp(rint(-min / scale), 0, 15); q = clamp(rint(w / scale) + z, 0, 15)
+ *     (rint first, then add z);
+ *   - degenerate group: if the fp16 scale is 0 (max == min, or fp16
+ *     underflow) the scale is taken as 1.0;
+ *   - packing: two codes per byte, low nibble = even k, high nibble = odd k;
+ *   - dequant: w^ = ((float)q - z) * scale * s[k], fp32, left to right;
+ *   - matmul: y[m][n] = sum_k x[m][k] * w^[n][k], accumulated in fp64 in
+ *     increasing k; bound[m][n] = sum_k |x[m][k] * w^[n][k]|.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* fp32 -> IEEE binary16, round-to-nearest-even (compiler conversion). */
+static uint16_t f32_to_f16_bits(float v) {
+    _Float16 h = (_Float16)v;
+    uint16_t b;
+    memcpy(&b, &h, sizeof b);
+    return b;
+}
+
+static float f16_bits_to_f32(uint16_t b) {
+    _Float16 h;
+    memcpy(&h, &b, sizeof h);
+    return (float)h;
+}
+
+/* Exposed so the tests can pin the conversion against an independent one. */
+uint16_t w4o_f32_to_f16(float v) { return f32_to_f16_bits(v); }
+float w4o_f16_to_f32(uint16_t b) { return f16_bits_to_f32(b); }
+
+static float clamp_0_15(float v) {
+    if (v < 0.0f) return 0.0f;
+    if (v > 15.0f) return 15.0f;
+    return v;
+}
+
+/*
+ * Quantize W [N][K] (fp32, row-major) group by group [Accel 2.1], with the
+ * optional AWQ per-input-channel scale s [K] applied as W / s first
+ * [Ch22 22.3, AWQ equation].  Outputs: codes [N][K] (one code per byte),
+ * scales [N][K/G] and zeros [N][K/G] as fp16 bit patterns.
+ * Returns 0, or -1 for arguments it cannot serve.
+ */
+int w4o_quantize(const float *W, const float *awq_s, int64_t N, int64_t K,
+                 int group, uint8_t *codes, uint16_t *scales, uint16_t *zeros) {
+    if (N < 0 || K < 0 || group <= 0 || K % group != 0) return -1;
+    fesetround(FE_TONEAREST);
+    const int64_t Kg = K / group;
+    float wp[1024];
+    if (group > 1024) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < Kg; ++g) {
+            const int64_t k0 = g * group;
+            /* step 1: AWQ prescale w' = w / s[k] (IEEE division) */
+            for (int i = 0; i < group; ++i) {
+                float w = W[n * K + k0 + i];
+                wp[i] = awq_s ? w / awq_s[k0 + i] : w;
+            }
+            /* step 2: group min and max */
+            float mn = wp[0], mx = wp[0];
+            for (int i = 1; i < group; ++i) {
+                if (wp[i] < mn) mn = wp[i];
+                if (wp[i] > mx) mx = wp[i];
+            }
+            /* step 3: scale = fp16((max - min) / 15); degenerate -> 1.0 */
+            float sc32 = (mx - mn) / 15.0f;
+            uint16_t sc_bits = f32_to_f16_bits(sc32);
+            float sc = f16_bits_to_f32(sc_bits);
+            if (sc == 0.0f) {
+                sc = 1.0f;
+                sc_bits = f32_to_f16_bits(1.0f);
+            }
+            /* step 4: zero point z = clamp(rint(-min / scale), 0, 15) */
+            float z = clamp_0_15(rintf(-mn / sc));
+            scales[n * Kg + g] = sc_bits;
+            zeros[n * Kg + g] = f32_to_f16_bits(z);
+            /* step 5: codes q = clamp(rint(w' / scale) + z, 0, 15) */
+            for (int i = 0; i < group; ++i) {
+                float q = clamp_0_15(rintf(wp[i] / sc) + z);
+                codes[n * K + k0 + i] = (uint8_t)q;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Pack codes [N][K] into bytes [N][K/2]: byte j of a row holds the code of
+ * k = 2j in its low nibble and of k = 2j+1 in its high nibble (0.5 byte per
+ * parameter, [Ch22 22.3] table).  Codes above 15 are masked to 4 bits.
+ */
+int w4o_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed) {
+    if (N < 0 || K < 0 || K % 2 != 0) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 2; ++j) {
+            uint8_t lo = codes[n * K + 2 * j] & 0x0F;
+            uint8_t hi = codes[n * K + 2 * j + 1] & 0x0F;
+            packed[n * (K / 2) + j] = (uint8_t)(lo | (hi << 4));
+        }
+    return 0;
+}
+
+/* Inverse of w4o_pack. */
+int w4o_unpack(const uint8_t *packed, int64_t N, int64_t K, uint8_t *codes) {
+    if (N < 0 || K < 0 || K % 2 != 0) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 2; ++j) {
+            uint8_t b = packed[n * (K / 2) + j];
+            codes[n * K + 2 * j] = b & 0x0F;
+            codes[n * K + 2 * j + 1] = b >> 4;
+        }
+    return 0;
+}
+
+/*
+ * Dequantize: w^[n][k] = ((float)q - z) * scale * s[k] in fp32, left to
+ * right (weight-only path, [Ch22 22.3]; AWQ re-multiplies by s).
+ */
+int w4o_dequant(const uint8_t *codes, const uint16_t *scales,
+                const uint16_t *zeros, const float *awq_s, int64_t N,
+                int64_t K, int group, float *What) {
+    if (N < 0 || K < 0 || group <= 0 || K % group != 0) return -1;
+    fesetround(FE_TONEAREST);
+    const int64_t Kg = K / group;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            float sc = f16_bits_to_f32(scales[n * Kg + k / group]);
+            float z = f16_bits_to_f32(zeros[n * Kg + k / group]);
+            float t = (float)codes[n * K + k] - z;
+            float w = t * sc;
+            if (awq_s) w = w * awq_s[k];
+            What[n * K + k] = w;
+        }
+    return 0;
+}
+
+/*
+ * Y = X . W^T with X [M][K] and W^ [N][K] given as fp32 (fp16/bf16 inputs
+ * widen exactly), accumulated in fp64 in increasing k.  bound[m][n] receives
+ * sum_k |x * w^| (the scale of the tolerance).  Either output may be NULL.
+ */
+int w4o_gemm(const float *X, const float *What, int64_t M, int64_t N,
+             int64_t K, double *Y, double *bound) {
+    if (M < 0 || N < 0 || K < 0) return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, abs_acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = (double)X[m * K + k] * (double)What[n * K + k];
+                acc += p;
+                abs_acc += fabs(p);
+            }
+            if (Y) Y[m * N + n] = acc;
+            if (bound) bound[m * N + n] = abs_acc;
+        }
+    return 0;
+}
