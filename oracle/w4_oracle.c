@@ -59,8 +59,10 @@ static float f16_bits_to_f32(uint16_t b) {
 uint16_t w4o_f32_to_f16(float v) { return f32_to_f16_bits(v); }
 float w4o_f16_to_f32(uint16_t b) { return f16_bits_to_f32(b); }
 
+/* clamp to [0, 15]; codes and zero points are integers, so -0 clamps to +0
+ * (IEEE 754-2019 maximum orders -0 below +0). */
 static float clamp_0_15(float v) {
-    if (v < 0.0f) return 0.0f;
+    if (!(v > 0.0f)) return 0.0f;
     if (v > 15.0f) return 15.0f;
     return v;
 }

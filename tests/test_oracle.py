@@ -161,6 +161,8 @@ def test_degenerate_groups():
     codes, scales, zeros = oracle.quantize(W)
     assert np.all(scales.astype(np.float32) == 1.0)
     assert list(zeros[:, 0].astype(int)) == [0, 0, 2, 0]
+    # a zero point is an integer: zero is stored as +0 (bits 0x0000), never -0
+    assert np.all(zeros.view(np.uint16)[[0, 1, 3], 0] == 0)
     What = oracle.dequant(codes, scales, zeros)
     assert np.array_equal(What[0], W[0]) and np.array_equal(What[1], W[1]) and np.array_equal(What[2], W[2])
     assert np.all(codes[3] == 0)  # rint(0.5) = 0 (ties to even), z = 0
