@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 hot path on B200.
+
+Headline (``value``): decode GEMM HBM throughput at Llama-3-8B linear-layer
+shapes, M = 1 -- one step = the four fused dequantize-matmul calls
+(qkv 4096->6144, o_proj 4096->4096, gate_up 4096->28672, down 14336->4096) on
+bf16 activations with packed uint4 weights resident in HBM.  Throughput is
+algorithmic bytes (packed codes + fp16 scale/zero + X + fp32 Y) per second.
+
+Also reported on the same JSON line:
+  * roofline of the dominant kernel (gate_up), timed by CUDA events recorded
+    inside the same CUDA graph as the timed steps;
+  * e2e: the same metric through the C ABI's host-buffer entry point
+    (pinned X in, fp32 Y out, copies inside the timed region);
+  * quantize: the quantize+pack kernel on the same four layers (fp32 W in);
+  * prefill: TFLOP/s of the tensor-core path at Llama-3-70B shapes, M = 8192;
+  * cpu_baseline: the oracle (plain C, one core) on a bounded sample.
+
+Multi-GPU: each rank runs its own copy of the step (independent problems, no
+collective on the data path): weak scaling, value = all ranks' bytes / max time.
+
+``--impl reference`` times the oracle alone on the host (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_only_int4_w4_b200 import synthetic  # noqa: E402
+
+METRIC = "W4A16 GEMM: decode HBM GB/s and prefill TFLOP/s vs B200 roofline, 1 GPU"
+G = 128
+LAYERS = list(synthetic.SHAPES_8B)  # qkv, o_proj, gate_up, down
+DOMINANT = "gate_up"
+N_COPIES = 5  # weight copies rotated across steps: 5 x 116 MB > 4 x L2 (126 MB)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def gemm_bytes(M, N, K):
+    """Algorithmic bytes of one fused call: packed codes + fp16 scale & zero + X (bf16) + Y (fp32)."""
+    return N * K // 2 + 4 * N * (K // G) + 2 * M * K + 4 * M * N
+
+
+def quant_bytes(N, K):
+    """fp32 W in, packed codes + fp16 scale & zero out."""
+    return 4 * N * K + N * K // 2 + 4 * N * (K // G)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "weight_only_int4_w4_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it matches today's kernels."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t.get(kernel_key)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            uuid = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+                if not uuid.startswith("GPU-"):
+                    uuid = "GPU-" + uuid
+            except Exception:
+                pass
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if uuid:
+                cmd += ["-i", uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not getattr(self, "out", ""):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_step(rows_per_layer):
+    """One oracle decode step on a sample: for each 8B layer, dequantize `rows_per_layer`
+    rows of pre-quantized weights and do the fp64 matmul with X (M=1).  Returns bytes."""
+    import oracle  # test/bench-only: the CPU baseline leg
+    total = 0
+    for name in LAYERS:
+        K, N = synthetic.SHAPES_8B[name]
+        key = (name, rows_per_layer)
+        if key not in _ORACLE_CACHE:
+            rows = list(range(min(rows_per_layer, N)))
+            W = synthetic.weight_rows(K, N, 0.02, 0.001, ("decode_8b", name), rows=rows).numpy()
+            X = synthetic.activations(1, K, "bf16", ("decode_8b", name)).float().numpy()
+            _ORACLE_CACHE[key] = (oracle.quantize(W), X)
+        (codes, sc, zp), X = _ORACLE_CACHE[key]
+        What = oracle.dequant(codes, sc, zp)
+        oracle.gemm(X, What)
+        total += gemm_bytes(1, codes.shape[0], K)
+    return total
+
+
+_ORACLE_CACHE = {}
+
+
+def time_cpu_oracle(budget_s=12.0, rows_per_layer=512):
+    cpu_oracle_step(rows_per_layer)  # build caches
+    t0 = time.perf_counter()
+    nbytes, reps = 0, 0
+    while time.perf_counter() - t0 < budget_s:
+        nbytes += cpu_oracle_step(rows_per_layer)
+        reps += 1
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows_per_layer} output rows of each of the 4 Llama-3-8B layers (dequant + fp64 matmul, M=1), "
+                      f"{reps} repetitions in {dt:.1f} s on one host core"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    rows = 256
+    for _ in range(args.warmup):
+        cpu_oracle_step(rows)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += cpu_oracle_step(rows)
+    dt = time.perf_counter() - t0
+    v = nbytes / dt / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32xu4->f64", "data": "synthetic",
+        "config": {"workload": "decode_8b (oracle sample)", "global_batch": 1, "seq_len": 1, "parallelism": "none"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} output rows of each of the 4 Llama-3-8B layers per step (dequant + fp64 matmul, M=1)"},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU legs
+def build_decode_state(w4, dev):
+    gen = torch.Generator(device=dev)
+    layers = {}
+    for name in LAYERS:
+        K, N = synthetic.SHAPES_8B[name]
+        gen.manual_seed(synthetic.seed_of("bench", "decode_8b", name) % (2 ** 62))
+        W = torch.randn((N, K), generator=gen, device=dev, dtype=torch.float32) * 0.02
+        mask = torch.rand((N, K), generator=gen, device=dev) < 0.001
+        W = torch.where(mask, torch.randn((N, K), generator=gen, device=dev) * synthetic.OUTLIER_STD, W)
+        packed, scales, zeros = w4.w4_quantize(W)
+        del W, mask
+        X = (torch.randn((1, K), generator=gen, device=dev)).to(torch.bfloat16)
+        copies = [(packed, scales, zeros)] + [(packed.clone(), scales.clone(), zeros.clone()) for _ in range(N_COPIES - 1)]
+        Y = torch.empty((1, N), dtype=torch.float32, device=dev)
+        ws_bytes = w4.w4a16_gemm_workspace_size(1, N, K)
+        ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        layers[name] = dict(K=K, N=N, X=X, copies=copies, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    return layers
+
+
+def decode_leg(w4, layers, steps, warmup, world):
+    dev = torch.device("cuda")
+    stream = torch.cuda.Stream()
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in range(steps)]
+
+    def step(i, record=False):
+        for name in LAYERS:
+            L = layers[name]
+            packed, scales, zeros = L["copies"][i % N_COPIES]
+            if record and name == DOMINANT:
+                ev[i][0].record()
+            w4.w4a16_gemm(L["X"], packed, scales, zeros, out=L["Y"], ws=L["ws"])
+            if record and name == DOMINANT:
+                ev[i][1].record()
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            step(i, record=True)
+    # warm replay of the graph itself
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            g.replay()
+            t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = t_start.elapsed_time(t_end)
+    dom = [a.elapsed_time(b) for a, b in ev]
+    del g
+    return ms, dom, clk.summary()
+
+
+def e2e_leg(w4, layers, steps, warmup, world):
+    """Same step through the C ABI's host-buffer entry point: pinned X in, Y out, per layer."""
+    host = {}
+    for name in LAYERS:
+        L = layers[name]
+        host[name] = (L["X"].cpu().pin_memory(), torch.empty((1, L["N"]), dtype=torch.float32).pin_memory())
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        for name in LAYERS:
+            L = layers[name]
+            packed, scales, zeros = L["copies"][i % N_COPIES]
+            Xh, Yh = host[name]
+            w4.w4a16_gemm_host(Xh, L["X"], packed, scales, zeros, Yh, L["Y"], ws=L["ws"], stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    h2d = sum(2 * layers[n]["K"] for n in LAYERS)
+    d2h = sum(4 * layers[n]["N"] for n in LAYERS)
+    return a.elapsed_time(b), h2d, d2h
+
+
+def quantize_leg(w4, steps=5):
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    Ws = []
+    for name in LAYERS:
+        K, N = synthetic.SHAPES_8B[name]
+        gen.manual_seed(synthetic.seed_of("bench", "quant", name) % (2 ** 62))
+        Ws.append(torch.randn((N, K), generator=gen, device=dev) * 0.02)
+    outs = [(torch.empty((W.shape[0], W.shape[1] // 2), dtype=torch.uint8, device=dev),
+             torch.empty((W.shape[0], W.shape[1] // G), dtype=torch.float16, device=dev),
+             torch.empty((W.shape[0], W.shape[1] // G), dtype=torch.float16, device=dev)) for W in Ws]
+    import ctypes
+    lib = w4.lib
+
+    def run():
+        s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for W, (p, sc, z) in zip(Ws, outs):
+            st = lib.w4_quantize(ctypes.c_void_p(W.data_ptr()), 0, None, W.shape[0], W.shape[1], G,
+                                 ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(sc.data_ptr()),
+                                 ctypes.c_void_p(z.data_ptr()), None, s)
+            assert st == 0
+    run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    nbytes = sum(quant_bytes(W.shape[0], W.shape[1]) for W in Ws)
+    del Ws, outs
+    torch.cuda.empty_cache()
+    return ms, nbytes
+
+
+def prefill_leg(w4, M=8192, steps=3):
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    res = {}
+    total_flop, total_ms = 0.0, 0.0
+    for name, (K, N) in synthetic.SHAPES_70B.items():
+        gen.manual_seed(synthetic.seed_of("bench", "prefill", name) % (2 ** 62))
+        W = torch.randn((N, K), generator=gen, device=dev) * 0.015
+        packed, scales, zeros = w4.w4_quantize(W)
+        del W
+        X = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+        Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        ws = w4.workspace(M, N, K, dev)
+        w4.w4a16_gemm(X, packed, scales, zeros, out=Y, ws=ws)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            w4.w4a16_gemm(X, packed, scales, zeros, out=Y, ws=ws)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        flop = 2.0 * M * N * K
+        res[name] = round(flop / (ms * 1e-3) / 1e12, 1)
+        total_flop += flop
+        total_ms += ms
+        del packed, scales, zeros, X, Y
+        torch.cuda.empty_cache()
+    return res, total_flop / (total_ms * 1e-3) / 1e12, total_ms
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the quantize and prefill legs")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world, rank, local = dist_setup(args.gpus)
+    from weight_only_int4_w4_b200 import w4  # fails loudly if libw4.so is missing
+
+    hbm_peak, bf16_peak, bf16_sust, peak_src = peaks()
+    layers = build_decode_state(w4, torch.device("cuda"))
+    step_bytes = sum(gemm_bytes(1, layers[n]["N"], layers[n]["K"]) for n in LAYERS)
+
+    ms, dom, clocks = decode_leg(w4, layers, args.steps, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    value = sum_over_ranks(step_bytes * args.steps, world) / (ms * 1e-3) / 1e9
+
+    K, N = synthetic.SHAPES_8B[DOMINANT]
+    dom_bytes = gemm_bytes(1, N, K)
+    dom_ms = sum(dom) / len(dom)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = e2e_leg(w4, layers, max(20, args.steps // 4), args.warmup, world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_steps = max(20, args.steps // 4)
+    e2e_value = sum_over_ranks(step_bytes * e2e_steps, world) / (e2e_ms * 1e-3) / 1e9
+    del layers
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if not args.no_extras:
+        q_ms, q_bytes = quantize_leg(w4)
+        q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+        extras["quantize"] = {"value": round(q_gbs, 1), "unit": "GB/s", "ms_per_call_4_layers": round(q_ms, 4),
+                              "workload": "quantize+pack of the 4 Llama-3-8B layers, fp32 W",
+                              "roofline": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm_peak,
+                                           "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4)}}
+        pf, pf_all, pf_ms = prefill_leg(w4)
+        extras["prefill"] = {"value": round(pf_all, 1), "unit": "TFLOP/s", "ms_per_step": round(pf_ms, 3),
+                             "workload": "Llama-3-70B qkv/o_proj/gate_up/down, M=8192, bf16 X",
+                             "per_layer_tflops": pf,
+                             "roofline": {"bound": "tensor", "achieved": round(pf_all, 1), "peak": bf16_peak,
+                                          "unit": "TFLOP/s", "frac": round(pf_all / bf16_peak, 4)}}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_cpu_oracle()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16xu4->f32", "data": "synthetic",
+            "config": {"workload": "decode_8b: Llama-3-8B qkv/o_proj/gate_up/down, M=1, bf16 X ~N(0,1), "
+                                   "W ~N(0,0.02) with 0.1% N(0,0.4) outliers, uint4 G=128",
+                       "global_batch": world, "seq_len": 1, "parallelism": f"replicas{world}",
+                       "l2": f"{N_COPIES} rotating weight copies ({N_COPIES * step_bytes / 1e6:.0f} MB > 4x L2): "
+                             "each step reads weights not touched for 4 steps",
+                       "graph": "timed steps captured in one CUDA graph"},
+            "roofline": {"bound": "hbm", "kernel": f"gemv_mma ({DOMINANT} 4096->28672, M=1)",
+                         "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(achieved / hbm_peak, 4), "peak_source": peak_src,
+                         "bytes_per_launch": dom_bytes, "avg_launch_us": round(dom_ms * 1e3, 3),
+                         "traffic": committed_traffic("gemv_mma_gate_up_m1")},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "w4a16_gemm_host (pinned host X/Y, copies + sync inside the call)"},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * w4.h -- C ABI of libw4: weight-only, per-group INT4 (W4A16) linear layers
+ * on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources cited by page and section):
+ *   - Quantization maps a float range onto integers through a scale and a
+ *     zero point, per group of 128 elements ("LLM inference acceleration"
+ *     article, discosf.com, section 2.1).  Here: asymmetric uint4 codes in
+ *     [0,15], one fp16 scale and one fp16 zero point per group of G = 128
+ *     consecutive input channels k of an output row n.
+ *   - Weight-only quantization: the weights are dequantized back to 16-bit and
+ *     multiplied by 16-bit activations, or a mixed-precision kernel does both
+ *     at once (aiwing.uk ch. 22 "Advanced inference optimisation", section
+ *     22.3 "Model quantization").  w4a16_gemm is that fused kernel.
+ *   - AWQ: weights are divided by a per-input-channel activation magnitude s
+ *     before quantization and multiplied back after, W^ = quant(W/s) * s
+ *     (ch. 22, section 22.3, AWQ equation).
+ *   - Scale and zero point travel with the packed weights as one unit
+ *     (article section 2.3); INT4 takes 0.5 byte per parameter (ch. 22,
+ *     section 22.3 table).
+ *
+ * Exact rule (the pages leave it open; this is the library's definition):
+ *   w'    = s ? w / s[k] : w                         (fp32, IEEE division)
+ *   mn,mx = min, max of w' over the group
+ *   scale = fp16_rn((mx - mn) / 15), taken as 1.0 if that is 0
+ *   z     = clamp(rint(-mn / scale), 0, 15)          (fp32, ties to even)
+ *   q     = clamp(rint(w' / scale) + z, 0, 15)
+ *   packed byte j of a row = q[2j] | q[2j+1] << 4    (low nibble = even k)
+ *   W^[n][k] = (q - z) * scale * (s ? s[k] : 1)
+ *   Y[m][n]  = sum_k X[m][k] * W^[n][k]               (fp32 accumulation)
+ *
+ * Layouts (all row-major, all buffers owned by the caller):
+ *   W       [N][K]   fp32, fp16 or bf16          (quantize input)
+ *   awq_s   [K]      fp32, > 0, or NULL
+ *   packed  [N][K/2] uint8
+ *   scales  [N][K/G] IEEE binary16 bit patterns
+ *   zeros   [N][K/G] IEEE binary16 bit patterns (integers 0..15)
+ *   codes   [N][K]   uint8, one code per byte (optional quantize output)
+ *   X       [M][K]   fp16 or bf16
+ *   Y       [M][N]   fp32 or bf16
+ *
+ * Conventions:
+ *   - Device pointers are device memory of the current CUDA device; every
+ *     device pointer must be 16-byte aligned.  The library allocates nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronize the device, except the
+ *     host-buffer entry point, which waits for its own stream.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns W4_ERR_INVALID_ARG or W4_ERR_UNSUPPORTED and
+ *     launches nothing.  A CUDA launch error returns W4_ERR_CUDA.
+ *     w4_last_error() gives a message for the last failure on this thread.
+ *   - Non-finite weights give unspecified codes.
+ *   - Thread-safe: no global state is written on the host except the
+ *     per-thread error message and a per-device cache of driver entry points.
+ */
+#ifndef W4_H_
+#define W4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  W4_OK = 0,
+  W4_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer, short workspace */
+  W4_ERR_UNSUPPORTED = 2, /* valid but not served: group != 128, dtype combination */
+  W4_ERR_CUDA = 3         /* a CUDA call or kernel launch failed */
+} w4_status;
+
+typedef enum { W4_F32 = 0, W4_F16 = 1, W4_BF16 = 2 } w4_dtype;
+
+/* Same type as cudaStream_t, declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st *w4_stream_t;
+
+/*
+ * Quantize and pack W (the whole a1..a5 path in one kernel launch).
+ *   W        device [N][K], dtype w_dtype (F32, F16 or BF16)
+ *   awq_s    device [K] fp32 or NULL (no AWQ)
+ *   N, K     N >= 1, K >= 1, K % group == 0
+ *   group    must be 128
+ *   packed   device [N][K/2] out; scales, zeros device [N][K/128] out
+ *   codes    device [N][K] out, or NULL (unpacked codes, a test aid)
+ * Outputs match the rule above bit for bit.
+ */
+w4_status w4_quantize(const void *W, w4_dtype w_dtype, const float *awq_s,
+                      int64_t N, int64_t K, int group, uint8_t *packed,
+                      uint16_t *scales, uint16_t *zeros, uint8_t *codes,
+                      w4_stream_t stream);
+
+/*
+ * Pack one-code-per-byte codes [N][K] (device) into packed [N][K/2]
+ * (device): low nibble = even k.  Values above 15 are masked to 4 bits.
+ * K must be a positive multiple of 32.
+ */
+w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed,
+                  w4_stream_t stream);
+
+/*
+ * Fused dequantize-matmul Y = X . W^T (a6..a7).
+ *   X         device [M][K], x_dtype F16 or BF16
+ *   M, N, K   >= 1; K % group == 0
+ *   group     must be 128
+ *   packed, scales, zeros   as produced by w4_quantize
+ *   awq_s     device [K] fp32, the SAME vector given to w4_quantize, or NULL
+ *   Y         device [M][N], y_dtype F32 or BF16 (overwritten)
+ *   workspace device scratch of at least w4a16_gemm_workspace_size(M,N,K)
+ *             bytes (may be NULL when that size is 0).  It must be zero-filled
+ *             once before its first use; every call leaves it zero-filled
+ *             again.  Calls that share a workspace must not overlap in time.
+ * Accuracy: |Y - Y_exact| <= 2e-3 * sum_k |X[m][k] * W^[n][k]| per element on
+ * the library's test distributions (fp32 accumulation; the prefill path rounds
+ * W^ to 16 bits once, the decode path keeps (q - z) exact).
+ */
+w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N,
+                     int64_t K, int group, const uint8_t *packed,
+                     const uint16_t *scales, const uint16_t *zeros,
+                     const float *awq_s, void *Y, w4_dtype y_dtype,
+                     void *workspace, size_t workspace_bytes,
+                     w4_stream_t stream);
+
+/* Bytes of workspace w4a16_gemm needs for this shape (0 if none). */
+size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * End-to-end variant with HOST activations and outputs: copies X_host
+ * (pinned host memory, [M][K]) into X_dev, runs w4a16_gemm, copies Y_dev
+ * back into Y_host (pinned host memory, [M][N]) and waits for `stream`.
+ * X_dev and Y_dev are caller-owned device staging buffers of the same sizes.
+ */
+w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype,
+                          int64_t M, int64_t N, int64_t K, int group,
+                          const uint8_t *packed, const uint16_t *scales,
+                          const uint16_t *zeros, const float *awq_s,
+                          void *Y_host, void *Y_dev, w4_dtype y_dtype,
+                          void *workspace, size_t workspace_bytes,
+                          w4_stream_t stream);
+
+/*
+ * Device-side error word: kernels whose bounded waits run out set it instead
+ * of hanging.  Copies its value to *flag (0 = no error) and clears it; this
+ * call synchronizes the current device.
+ */
+w4_status w4_device_error(int *flag);
+
+/* Human-readable name of a status code (static string). */
+const char *w4_status_string(w4_status status);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *w4_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* W4_H_ */

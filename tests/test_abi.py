@@ -1,0 +1,116 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_only_int4_w4_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = build.build_library()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(w4[a-z0-9_]*)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("w4_quantize", "w4_pack", "w4a16_gemm", "w4a16_gemm_workspace_size", "w4_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def _setup(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.w4_quantize.argtypes = [P, ctypes.c_int, P, I64, I64, ctypes.c_int, P, P, P, P, P]
+    lib.w4_pack.argtypes = [P, I64, I64, P, P]
+    lib.w4a16_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, ctypes.c_int, P, P, P, P, P, ctypes.c_int, P,
+                               ctypes.c_size_t, P]
+    lib.w4a16_gemm_workspace_size.argtypes = [I64, I64, I64]
+    lib.w4a16_gemm_workspace_size.restype = ctypes.c_size_t
+    lib.w4_status_string.argtypes = [ctypes.c_int]
+    lib.w4_status_string.restype = ctypes.c_char_p
+    lib.w4_last_error.restype = ctypes.c_char_p
+
+
+A = 0x10000  # fake, 16-byte aligned "device" addresses: never dereferenced (rejected first)
+
+
+def test_status_strings(lib):
+    _setup(lib)
+    assert lib.w4_status_string(0) == b"W4_OK"
+    assert lib.w4_status_string(1) == b"W4_ERR_INVALID_ARG"
+    assert lib.w4_status_string(2) == b"W4_ERR_UNSUPPORTED"
+    assert lib.w4_status_string(3) == b"W4_ERR_CUDA"
+
+
+@pytest.mark.parametrize("N,K,group,expect", [
+    (0, 128, 128, 1),      # empty
+    (4, 0, 128, 1),
+    (4, 200, 128, 1),      # K not a multiple of the group
+    (4, 256, 64, 2),       # unsupported group size
+    (-1, 128, 128, 1),
+])
+def test_quantize_rejects_bad_shapes(lib, N, K, group, expect):
+    _setup(lib)
+    st = lib.w4_quantize(A, 0, None, N, K, group, A, A, A, None, None)
+    assert st == expect, lib.w4_last_error()
+
+
+def test_quantize_rejects_null_and_misaligned(lib):
+    _setup(lib)
+    assert lib.w4_quantize(None, 0, None, 4, 128, 128, A, A, A, None, None) == 1
+    assert lib.w4_quantize(A, 0, None, 4, 128, 128, None, A, A, None, None) == 1
+    assert lib.w4_quantize(A + 4, 0, None, 4, 128, 128, A, A, A, None, None) == 1
+    assert lib.w4_quantize(A, 0, A + 8, 4, 128, 128, A, A, A, None, None) == 1
+    assert lib.w4_quantize(A, 0, A + 8, 4, 128, 128, A, A, A, None, None) == 1
+    assert b"aligned" in lib.w4_last_error()
+    assert lib.w4_quantize(A, 7, None, 4, 128, 128, A, A, A, None, None) == 2  # unknown dtype
+
+
+def test_pack_rejects(lib):
+    _setup(lib)
+    assert lib.w4_pack(A, 4, 48, A, None) == 1   # K not a multiple of 32
+    assert lib.w4_pack(None, 4, 64, A, None) == 1
+    assert lib.w4_pack(A, 4, 64, A + 1, None) == 1
+
+
+def test_gemm_rejects(lib):
+    _setup(lib)
+    g = lambda **kw: lib.w4a16_gemm(kw.get("X", A), kw.get("xd", 2), kw.get("M", 1), kw.get("N", 16),
+                                     kw.get("K", 128), kw.get("G", 128), kw.get("P", A), A, A, None,
+                                     kw.get("Y", A), kw.get("yd", 0), None, 0, None)
+    assert g(M=0) == 1
+    assert g(K=100) == 1
+    assert g(G=32) == 2
+    assert g(xd=0) == 2          # fp32 activations are not served
+    assert g(yd=1) == 2          # fp16 output not served
+    assert g(X=None) == 1
+    assert g(Y=A + 4) == 1
+    assert g(P=A + 2) == 1
+    assert b"aligned" in lib.w4_last_error()
+
+
+def test_workspace_size_plan(lib):
+    _setup(lib)
+    # decode of a 14336-deep layer splits K across CTAs -> needs partials + counters
+    assert lib.w4a16_gemm_workspace_size(1, 4096, 14336) > 4096 * 4
+    # invalid shapes need none
+    assert lib.w4a16_gemm_workspace_size(0, 16, 128) == 0
+    assert lib.w4a16_gemm_workspace_size(1, 16, 100) == 0

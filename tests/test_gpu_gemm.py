@@ -1,0 +1,205 @@
+"""GPU parity of the fused dequantize-matmul (K1 decode path, K2 tensor-core
+path) against the oracle: |y - y_ref| <= 2e-3 * sum_k |x w^| per element.
+
+The weights given to the GPU GEMM are the ORACLE's packed codes, scales and
+zeros (uploaded), so these tests check the matmul independently of K0; the
+end-to-end tests at the bottom chain K0 -> GEMM."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_int4_w4_b200 import synthetic
+
+from ._util import check_close, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w4():
+    from weight_only_int4_w4_b200 import w4 as mod
+    return mod
+
+
+class forced_path:
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        self.old = os.environ.get("W4_FORCE_PATH")
+        if self.path:
+            os.environ["W4_FORCE_PATH"] = self.path
+        else:
+            os.environ.pop("W4_FORCE_PATH", None)
+
+    def __exit__(self, *a):
+        if self.old is None:
+            os.environ.pop("W4_FORCE_PATH", None)
+        else:
+            os.environ["W4_FORCE_PATH"] = self.old
+
+
+def _upload_oracle_weights(W_np, awq_np=None):
+    codes, scales, zeros = oracle.quantize(W_np, awq_np)
+    packed = oracle.pack(codes)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return (dev(packed), dev(scales.view(np.uint16)).view(torch.float16), dev(zeros.view(np.uint16)).view(torch.float16),
+            (codes, scales, zeros))
+
+
+def _run_case(w4, M, N, K, x_dtype="bf16", awq=False, outliers=0.0, std=0.02, path=None, rows=None,
+              out_dtype=torch.float32, tag=None):
+    tag = tag or ("case", M, N, K, x_dtype, awq, outliers)
+    W = synthetic.weight(K, N, std, outliers, tag)
+    s = synthetic.awq_scale(K, tag) if awq else None
+    X = synthetic.activations(M, K, x_dtype, tag)
+    packed, scales, zeros, (codes, sc, zp) = _upload_oracle_weights(W.numpy(), None if s is None else s.numpy())
+    with forced_path(path):
+        Y = w4.w4a16_gemm(X.cuda(), packed, scales, zeros, None if s is None else s.cuda(), out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    rows = np.arange(N) if rows is None else rows
+    What = oracle.dequant(codes[rows], sc[rows], zp[rows], None if s is None else s.numpy())
+    Yref, bound = oracle.gemm(X.float().numpy(), What)
+    Yg = Y.float().cpu().numpy()[:, rows]
+    return check_close(Yg, Yref, bound, out_bf16=out_dtype == torch.bfloat16, what=f"M={M} N={N} K={K} {path}")
+
+
+def test_tiny_workload(w4):
+    """256x256 fp32 weights, fp16 activations, M=1 (the oracle-sized case)."""
+    _run_case(w4, 1, 256, 256, x_dtype="f16", tag=("tiny", "tiny"))
+
+
+@pytest.mark.parametrize("layer", list(synthetic.SHAPES_8B))
+def test_decode_8b_full(w4, layer):
+    """M=1 bf16 decode at Llama-3-8B shapes with 0.1% outliers: every output checked."""
+    K, N = synthetic.SHAPES_8B[layer]
+    _run_case(w4, 1, N, K, outliers=0.001, tag=("decode_8b", layer))
+
+
+@pytest.mark.parametrize("M", [4, 8, 16, 32, 48, 64])
+@pytest.mark.parametrize("layer", list(synthetic.SHAPES_8B))
+def test_verify_8b_awq_sampled(w4, M, layer):
+    """Speculative-verification / small-batch M with the AWQ scale folded in."""
+    K, N = synthetic.SHAPES_8B[layer]
+    rows = sample_rows(N, 192, seed=M * 7 + K)
+    _run_case(w4, M, N, K, awq=True, rows=rows, tag=("verify_8b", layer))
+
+
+@pytest.mark.parametrize("layer", list(synthetic.SHAPES_70B))
+def test_prefill_70b_sampled(w4, layer):
+    """Prefill at Llama-3-70B shapes, M in {512, 2048, 8192}: sampled outputs of
+    full-size launches, one weight quantization per layer reused for all M."""
+    K, N = synthetic.SHAPES_70B[layer]
+    tag = ("prefill_70b", layer)
+    rows = sample_rows(N, 40, seed=K ^ N)
+    Wr = synthetic.weight_rows(K, N, 0.015, 0.0, tag, rows=rows).numpy()
+    # the GPU quantizes the full matrix itself (K0 is checked bit-exact elsewhere)
+    W = synthetic.weight(K, N, 0.015, 0.0, tag).cuda()
+    packed, scales, zeros = w4.w4_quantize(W)
+    del W
+    codes, sc, zp = oracle.quantize(Wr)
+    What = oracle.dequant(codes, sc, zp)
+    Xall = synthetic.activations(8192, K, "bf16", tag)
+    for M in (512, 2048, 8192):
+        X = Xall[:M]
+        toks = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(M).choice(M, 24, replace=False)]))
+        Y = w4.w4a16_gemm(X.cuda(), packed, scales, zeros)
+        torch.cuda.synchronize()
+        Yg = Y[torch.from_numpy(toks).cuda()][:, torch.from_numpy(rows).cuda()].float().cpu().numpy()
+        del Y
+        Yref, bound = oracle.gemm(X[torch.from_numpy(toks)].float().numpy(), What)
+        check_close(Yg, Yref, bound, what=f"{layer} M={M}")
+
+
+@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("M,N,K", [
+    (1, 16, 128), (1, 1, 128), (2, 100, 256), (3, 129, 384), (7, 300, 1024), (9, 64, 128),
+    (15, 200, 640), (17, 130, 256), (31, 77, 512), (33, 128, 1024), (63, 257, 256), (64, 320, 384),
+])
+def test_edge_shapes_both_paths(w4, M, N, K, path):
+    _run_case(w4, M, N, K, path=path, tag=("edge", M, N, K))
+
+
+@pytest.mark.parametrize("M,N,K", [(65, 300, 384), (100, 129, 1024), (129, 64, 256), (256, 513, 512),
+                                   (300, 200, 1280)])
+def test_edge_shapes_tc_only(w4, M, N, K):
+    _run_case(w4, M, N, K, tag=("edge", M, N, K))
+
+
+@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("x_dtype", ["f16", "bf16"])
+def test_awq_and_dtypes(w4, path, x_dtype):
+    _run_case(w4, 5, 384, 1024, x_dtype=x_dtype, awq=True, path=path, tag=("awq-dt", x_dtype))
+    _run_case(w4, 24, 256, 512, x_dtype=x_dtype, awq=True, path=path, tag=("awq-dt24", x_dtype))
+
+
+@pytest.mark.parametrize("path", ["gemv", "tc"])
+def test_bf16_output(w4, path):
+    _run_case(w4, 4, 512, 1024, path=path, out_dtype=torch.bfloat16, tag=("bf16out",))
+
+
+def test_long_k_split_both_paths(w4):
+    """K = 28672 (70B down_proj depth) at small M: split-K on both paths."""
+    for path in ("gemv", "tc"):
+        _run_case(w4, 2, 512, 28672, path=path, tag=("longk",))
+
+
+def test_workspace_reuse_is_stable(w4):
+    """Split-K counters are left at zero: repeated calls give identical bits."""
+    K, N = 14336, 4096
+    tag = ("reuse",)
+    W = synthetic.weight(K, N, 0.02, 0.0, tag).cuda()
+    packed, scales, zeros = w4.w4_quantize(W)
+    X = synthetic.activations(1, K, "bf16", tag).cuda()
+    for path in ("gemv", "tc"):
+        with forced_path(path):
+            outs = [w4.w4a16_gemm(X, packed, scales, zeros).clone() for _ in range(3)]
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+def test_end_to_end_quantize_then_gemm(w4):
+    """K0 on the GPU feeding the GEMM, against the oracle's whole path."""
+    M, N, K = 3, 1000, 4096
+    tag = ("e2e",)
+    W = synthetic.weight(K, N, 0.02, 0.001, tag)
+    s = synthetic.awq_scale(K, tag)
+    X = synthetic.activations(M, K, "bf16", tag)
+    packed, scales, zeros = w4.w4_quantize(W.cuda(), s.cuda())
+    Y = w4.w4a16_gemm(X.cuda(), packed, scales, zeros, s.cuda())
+    Yref, bound, _ = oracle.reference_linear(X.float().numpy(), W.numpy(), s.numpy())
+    check_close(Y.cpu().numpy(), Yref, bound, what="e2e")
+
+
+def test_host_entry_point(w4):
+    M, N, K = 2, 640, 2048
+    tag = ("host",)
+    W = synthetic.weight(K, N, 0.02, 0.0, tag)
+    X = synthetic.activations(M, K, "bf16", tag)
+    packed, scales, zeros = w4.w4_quantize(W.cuda())
+    Xh = X.pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    w4.w4a16_gemm_host(Xh, torch.empty_like(X, device="cuda"), packed, scales, zeros, Yh,
+                       torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    Yref, bound, _ = oracle.reference_linear(X.float().numpy(), W.numpy())
+    check_close(Yh.numpy(), Yref, bound, what="host")
+
+
+def test_short_workspace_rejected(w4):
+    M, N, K = 1, 4096, 14336
+    need = w4.w4a16_gemm_workspace_size(M, N, K)
+    assert need > 0
+    X = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    packed = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros((N, K // 128), dtype=torch.float16, device="cuda")
+    small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(w4.W4Error) as ei:
+        w4.w4a16_gemm(X, packed, sc, sc, ws=small)
+    assert ei.value.status == w4.W4_ERR_INVALID_ARG
+
+
+def test_no_device_error(w4):
+    assert w4.w4_device_error() == 0

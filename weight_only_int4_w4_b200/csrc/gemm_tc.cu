@@ -1,0 +1,307 @@
+// gemm_tc.cu -- K2: prefill W4A16 matmul on the 5th-generation tensor cores.
+//
+// Prefill is compute-bound (ch. 22 "Advanced inference optimisation", section
+// 22.2 table; "LLM inference acceleration" article, section 1.1), so the
+// dequantized weights go through tcgen05.mma.  The weight-only path of ch. 22
+// section 22.3 (dequantize back to 16 bits, then matmul, fused in one kernel):
+//
+//   D[n][m] = sum_k W^[n][k] * X[m][k]      (swap-AB: weights are the MMA's M side)
+//
+// One CTA computes a tile of 128 weight rows x BN tokens over a k-range:
+//   warp 0      TMA producer: X tile [BN x 64] (128-byte swizzle) and the packed
+//               weight tile [128 rows x 32 bytes] into a ring of NS stages.
+//   warps 4..7  dequantize: thread r converts row r's 64 codes of the stage
+//               into 16-bit (q - z) * scale (* s[k] for AWQ), rounded once,
+//               and stores them with tcgen05.st straight into TMEM, where they
+//               are the A operand (TMEM lane = weight row, 2 values per column).
+//   warp 1      one thread issues tcgen05.mma (A from TMEM, B = X from shared
+//               memory, fp32 accumulator in TMEM) and tcgen05.commit.
+//   warps 4..7  epilogue: tcgen05.ld of the accumulator, fp32 or bf16 stores
+//               (each warp store covers 32 consecutive output channels).
+// TMEM columns: [0, BN) accumulator, then NS stages of 32 columns of A.
+// All waits are bounded (see common.cuh).  No TMA multicast anywhere.
+#include "common.cuh"
+
+namespace w4 {
+
+struct TcParams {
+  int64_t M, N, K;
+  const uint16_t *scales;
+  const uint16_t *zeros;
+  const float *awq_s;
+  void *Y;
+  int y_bf16;
+  float *ws;           // [splits][M][N] partials (split-K only)
+  uint32_t *counters;  // [tiles] arrival counters (split-K only)
+  int splits;
+  int kb_per_split;  // k-blocks of 64 per split
+};
+
+namespace tc_impl {
+
+constexpr int kBK = 64;   // k per pipeline stage
+constexpr int kNS = 4;    // pipeline stages
+constexpr int kPStage = 128 * 32;
+
+template <int BN>
+struct TcCfg {
+  static constexpr int kXStage = BN * 128;
+  static constexpr uint32_t kTmemCols = (BN + 32 * kNS <= 256) ? 256u : 512u;
+  static constexpr int kSmem = 1024 /*align slack*/ + kNS * (kXStage + kPStage) + 256;
+};
+
+// 64 codes of one row (32 bytes) -> 32 columns of 16-bit pairs (k even in the low half).
+// Each byte is moved to bits 15..22 of a word; OR-ing 256.0f (0x43800000) then
+// gives the exact fp32 values 256 + q_lo (nibble at bits 15..18) and
+// 256 + 16 q_hi (bits 19..22), both inside the 23-bit mantissa.  One FFMA per
+// weight turns them into (q - z) * scale: the offsets -(256 + z) * scale and
+// -(16 + z) * scale are exact in fp32 (9 + 11 significant bits), so the only
+// rounding is that of the final 16-bit conversion.
+template <bool kBf16, bool kAwq>
+__device__ __forceinline__ void dequant_row64(const uint4 &w0, const uint4 &w1, float sc, float z,
+                                              const float *__restrict__ sk, uint32_t (&out)[32]) {
+  const float off_lo = -(256.0f + z) * sc;
+  const float sc16 = sc * 0.0625f;
+  const float off_hi = -(16.0f + z) * sc;
+  const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+  for (int wi = 0; wi < 8; ++wi) {
+    const uint32_t w = words[wi];
+    const uint32_t tb[4] = {w << 15, w << 7, w >> 1, w >> 9};  // byte b at bits 15..22
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float flo = __uint_as_float(lop3_and_or(tb[b], 0x00078000u, 0x43800000u));
+      const float fhi = __uint_as_float(lop3_and_or(tb[b], 0x00780000u, 0x43800000u));
+      float vlo = fmaf(flo, sc, off_lo);
+      float vhi = fmaf(fhi, sc16, off_hi);
+      const int col = wi * 4 + b;
+      if constexpr (kAwq) {
+        const float2 s2 = *reinterpret_cast<const float2 *>(sk + 2 * col);
+        vlo *= s2.x;
+        vhi *= s2.y;
+      }
+      if constexpr (kBf16) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(vlo, vhi);
+        out[col] = *reinterpret_cast<const uint32_t *>(&v);
+      } else {
+        const __half2 v = __floats2half2_rn(vlo, vhi);
+        out[col] = *reinterpret_cast<const uint32_t *>(&v);
+      }
+    }
+  }
+}
+
+// AND of a predicate over the 128 dequant/epilogue threads (named barrier 1).
+__device__ __forceinline__ bool epilogue_vote(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+template <int BN, bool kBf16, bool kAwq>
+__global__ void __launch_bounds__(256, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                   const TcParams p) {
+  using Cfg = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sX = smem;
+  uint8_t *sP = sX + kNS * Cfg::kXStage;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sP + kNS * kPStage);
+  uint64_t *empty = full + kNS;
+  uint64_t *afull = empty + kNS;
+  uint64_t *accfull = afull + kNS;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accfull + 1);
+  int *s_last = reinterpret_cast<int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t M = p.M, N = p.N, K = p.K;
+  const int64_t n0 = (int64_t)blockIdx.x * 128;
+  const int64_t m0 = (int64_t)blockIdx.y * BN;
+  const int split = blockIdx.z;
+  const int total_kb = (int)(K / kBK);
+  const int kb0 = split * p.kb_per_split;
+  const int kb1 = min(kb0 + p.kb_per_split, total_kb);
+  const int nkb = max(kb1 - kb0, 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&afull[s], 128);
+    }
+    mbar_init(accfull, 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmP);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % kNS;
+        const uint32_t ph = (uint32_t)(i / kNS) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) break;
+        mbar_arrive_expect_tx(&full[s], Cfg::kXStage + kPStage);
+        const int kb = kb0 + i;
+        tma_load_2d(sX + s * Cfg::kXStage, &tmX, &full[s], kb * kBK, (int32_t)m0);
+        tma_load_2d(sP + s * kPStage, &tmP, &full[s], kb * (kBK / 2), (int32_t)n0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(kBf16, BN);
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % kNS;
+        const uint32_t ph = (uint32_t)(i / kNS) & 1u;
+        if (!mbar_wait(&full[s], ph, kErrTimeoutMma)) break;
+        if (!mbar_wait(&afull[s], ph, kErrTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + (uint32_t)(BN + s * 32);
+        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sX + s * Cfg::kXStage));
+#pragma unroll
+        for (int j = 0; j < kBK / 16; ++j)
+          tc_mma_ts(tmem, a_tmem + 8 * j, bdesc + (uint64_t)(2 * j), idesc, (i > 0 || j > 0) ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      tc_commit(accfull);
+    }
+  } else if (warp >= 4) {
+    const int q = warp - 4;
+    const int r = q * 32 + lane;
+    const int64_t n = n0 + r;
+    const bool row_ok = n < N;
+    const int64_t Kg = K / kGroup;
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    float sc = 0.0f, z = 0.0f;
+    bool ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % kNS;
+      const uint32_t ph = (uint32_t)(i / kNS) & 1u;
+      const int kb = kb0 + i;
+      if (i == 0 || (kb & 1) == 0) {
+        const int64_t grp = kb / 2;
+        sc = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp)) : 0.0f;
+        z = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp)) : 0.0f;
+      }
+      if (!mbar_wait(&full[s], ph, kErrTimeoutDequant)) { ok = false; break; }
+      const uint4 *src = reinterpret_cast<const uint4 *>(sP + s * kPStage + r * 32);
+      const uint4 w0 = src[0], w1 = src[1];
+      uint32_t out[32];
+      dequant_row64<kBf16, kAwq>(w0, w1, sc, z, kAwq ? p.awq_s + (int64_t)kb * kBK : nullptr, out);
+      tmem_st_32x32b_x32(lane_base + (uint32_t)(BN + s * 32), out);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&afull[s]);
+    }
+
+    // ---- epilogue (the decision to run it is made uniform over the 128 threads,
+    // so the named barriers below are reached by all of them or by none)
+    bool go = ok && nkb > 0 && mbar_wait(accfull, 0, kErrTimeoutEpilogue);
+    go = epilogue_vote(go);
+    if (go) {
+      tc_fence_after();
+      const bool direct = p.splits == 1;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), v);
+        tc_wait_ld();
+        if (!row_ok) continue;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int64_t m = m0 + c * 32 + j;
+          if (m < M) {
+            const float val = __uint_as_float(v[j]);
+            if (direct) {
+              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[m * N + n] = __float2bfloat16_rn(val);
+              else static_cast<float *>(p.Y)[m * N + n] = val;
+            } else {
+              p.ws[((int64_t)split * M + m) * N + n] = val;
+            }
+          }
+        }
+      }
+      if (!direct) {
+        // last CTA of this output tile to arrive sums the split-K partials
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int64_t tile = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+        if (r == 0) {
+          const uint32_t prev = atomicAdd(&p.counters[tile], 1u);
+          *s_last = prev == (uint32_t)(p.splits - 1);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*s_last) {
+          __threadfence();
+          if (row_ok) {
+            for (int j = 0; j < BN; ++j) {
+              const int64_t m = m0 + j;
+              if (m >= M) break;
+              float acc = 0.0f;
+              for (int s = 0; s < p.splits; ++s) acc += __ldcg(p.ws + ((int64_t)s * M + m) * N + n);
+              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[m * N + n] = __float2bfloat16_rn(acc);
+              else static_cast<float *>(p.Y)[m * N + n] = acc;
+            }
+          }
+          if (r == 0) atomicExch(&p.counters[tile], 0u);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+template <int BN, bool kBf16, bool kAwq>
+cudaError_t launch_t(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, cudaStream_t stream) {
+  using Cfg = TcCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, kBf16, kAwq>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN), (unsigned)p.splits);
+  kern<<<grid, 256, Cfg::kSmem, stream>>>(tmX, tmP, p);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, bool bf16,
+                      cudaStream_t stream) {
+  const bool awq = p.awq_s != nullptr;
+  if (bf16) return awq ? launch_t<BN, true, true>(tmX, tmP, p, stream) : launch_t<BN, true, false>(tmX, tmP, p, stream);
+  return awq ? launch_t<BN, false, true>(tmX, tmP, p, stream) : launch_t<BN, false, false>(tmX, tmP, p, stream);
+}
+
+}  // namespace tc_impl
+
+cudaError_t launch_gemm_tc(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, bool x_bf16, int bn,
+                           cudaStream_t stream) {
+  switch (bn) {
+    case 64: return tc_impl::launch_bn<64>(tmX, tmP, p, x_bf16, stream);
+    case 128: return tc_impl::launch_bn<128>(tmX, tmP, p, x_bf16, stream);
+    default: return tc_impl::launch_bn<256>(tmX, tmP, p, x_bf16, stream);
+  }
+}
+
+}  // namespace w4

@@ -1,0 +1,440 @@
+// libw4.cu -- the C ABI of libw4 (declared in include/w4.h) and the single
+// translation unit that holds every kernel of the library.
+//
+// Host side only: argument validation (before anything is launched), the
+// per-call launch plan (which kernel, how many k-slices, grid), TMA
+// descriptor encoding, and error reporting.  The arithmetic is in the kernels.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "gemm_tc.cu"
+#include "gemv_mma.cu"
+#include "quantize.cu"
+#include "w4.h"
+
+namespace w4 {
+cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, uint8_t *packed,
+                            uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count, cudaStream_t stream);
+cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,
+                        cudaStream_t stream);
+}  // namespace w4
+
+namespace {
+
+thread_local std::string t_last_error;
+
+w4_status fail(w4_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+w4_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(W4_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+std::mutex g_mu;
+
+// SM count of the current device (148 on B200); cached per device.
+cudaError_t current_sm_count(int *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    g_sm_count[dev] = n;
+  }
+  *out = g_sm_count[dev];
+  return cudaSuccess;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+
+enum Path { kPathGemv = 1, kPathTc = 2 };
+
+// Workspace layout: [0, 64 KiB) split-K arrival counters, then fp32 partials.
+// The counter region is the same for every call, so partials left behind by
+// one call never land on the counters of the next; counters are reset to zero
+// by the last CTA (or warp) that uses them.
+constexpr size_t kCounterBytes = 65536;
+constexpr int64_t kMaxCounters = kCounterBytes / 4;
+
+struct GemmPlan {
+  int path = 0;
+  // K1
+  int t8 = 1, ks = 1, kslices = 1, grid_x = 1;
+  bool sc_tma = false;
+  // K2
+  int bn = 256, splits = 1, kb_per_split = 1;
+  size_t ws_bytes = 0;
+};
+
+int t8_for(int64_t M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
+
+// Path forced through the environment (W4_FORCE_PATH=gemv|tc), for tests and tuning.
+int forced_path() {
+  const char *e = getenv("W4_FORCE_PATH");
+  if (!e) return 0;
+  if (!strcmp(e, "gemv")) return kPathGemv;
+  if (!strcmp(e, "tc")) return kPathTc;
+  return 0;
+}
+
+// CTAs of the decode kernel that fit on one SM (shared memory bound).
+int gemv_ctas_per_sm(int ks) {
+  const int per = w4::gemv_smem_bytes(ks) + 1024;
+  int n = (228 * 1024) / per;
+  return n < 1 ? 1 : (n > 4 ? 4 : n);
+}
+
+GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
+  GemmPlan p;
+  p.path = kPathGemv;
+  p.t8 = t8_for(M);
+  const int64_t Kg = K / w4::kGroup;
+  const int64_t RT = cdiv(N, 64);
+  const int64_t RB16 = cdiv(N, 16);
+  p.sc_tma = (Kg % 8) == 0;
+  double best = 1e300;
+  for (int ks = w4::gemv_max_ks(p.t8, awq); ks >= 1; ks /= 2) {
+    const int64_t kslices = cdiv(Kg, ks);
+    if (kslices > 1 && RB16 > kMaxCounters) continue;
+    const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(ks);
+    const double task_bytes = 64.0 * ks * (64 + 4);
+    const double split_bytes = kslices > 1 ? 2.0 * 4.0 * (double)kslices * M * N / sm : 0.0;
+    for (int64_t gx = std::min<int64_t>(RT, std::max<int64_t>(1, slots / kslices)); gx >= 1; --gx) {
+      const int64_t c = cdiv(RT, gx);
+      if (gx < RT && cdiv(RT, gx + 1) == c) continue;  // same tasks per CTA with more CTAs: keep the larger grid
+      const int64_t ctas = gx * kslices;
+      // bytes streamed by the busiest SM (+ split-K partials), + a per-wave start cost
+      const double est = (double)cdiv(ctas, sm) * c * task_bytes + split_bytes +
+                         4096.0 * (double)(cdiv(ctas, slots) - 1) * 64;
+      if (est < best * (1 - 1e-9)) {
+        best = est;
+        p.ks = ks;
+        p.kslices = (int)kslices;
+        p.grid_x = (int)gx;
+      }
+      if (c > 4 * cdiv(RT * kslices, sm) + 8) break;
+    }
+  }
+  // tuning overrides: W4_GEMV_KS (groups per task) and W4_GEMV_GX (CTAs per k-slice)
+  if (const char *e = getenv("W4_GEMV_KS")) {
+    const int ks = atoi(e);
+    if ((ks == 1 || ks == 2 || ks == 4) && ks <= w4::gemv_max_ks(p.t8, awq)) {
+      p.ks = ks;
+      p.kslices = (int)cdiv(Kg, ks);
+      p.grid_x = (int)std::min<int64_t>(RT, std::max<int64_t>(1, (int64_t)sm * gemv_ctas_per_sm(ks) / p.kslices));
+    }
+  }
+  if (const char *e = getenv("W4_GEMV_GX")) {
+    const int gx = atoi(e);
+    if (gx >= 1) p.grid_x = (int)std::min<int64_t>(RT, gx);
+  }
+  if (p.kslices > 1 && RB16 > kMaxCounters) {  // overrides may not exceed the counter region
+    p.ks = w4::gemv_max_ks(p.t8, awq);
+    p.kslices = (int)cdiv(Kg, p.ks);
+  }
+  if (p.kslices > 1) p.ws_bytes = kCounterBytes + (size_t)p.kslices * M * N * 4;
+  return p;
+}
+
+GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, int sm) {
+  GemmPlan p;
+  p.path = kPathTc;
+  p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
+  const int64_t total_kb = K / 64;
+  int64_t splits = 1;
+  if (tiles < sm && tiles <= kMaxCounters) splits = std::max<int64_t>(1, std::min<int64_t>(sm / tiles, total_kb / 8));
+  int64_t kbps = cdiv(total_kb, splits);
+  splits = cdiv(total_kb, kbps);
+  p.splits = (int)splits;
+  p.kb_per_split = (int)kbps;
+  if (splits > 1) p.ws_bytes = kCounterBytes + (size_t)splits * M * N * 4;
+  return p;
+}
+
+bool gemv_fits(int64_t M, int64_t N, bool awq) {
+  return w4::gemv_supports(M, awq);
+}
+
+GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
+  int f = forced_path();
+  if (f == kPathTc) return plan_tc(M, N, K, sm);
+  if (f == kPathGemv || gemv_fits(M, N, awq)) return plan_gemv(M, N, K, awq, sm);
+  return plan_tc(M, N, K, sm);
+}
+
+// W4_DEBUG_PLAN=1 prints every launch plan to stderr (tuning aid).
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
+  GemmPlan p = plan_gemm_raw(M, N, K, awq, sm);
+  if (getenv("W4_DEBUG_PLAN")) {
+    if (p.path == kPathGemv)
+      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld decode: t8=%d ks=%d kslices=%d grid_x=%d scale_tma=%d ws=%zu\n",
+              (long long)M, (long long)N, (long long)K, p.t8, p.ks, p.kslices, p.grid_x, (int)p.sc_tma, p.ws_bytes);
+    else
+      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld tensor-core: bn=%d splits=%d kb_per_split=%d ws=%zu\n",
+              (long long)M, (long long)N, (long long)K, p.bn, p.splits, p.kb_per_split, p.ws_bytes);
+  }
+  return p;
+}
+
+size_t ws_size_all(int64_t M, int64_t N, int64_t K, int sm) {
+  size_t ws = plan_tc(M, N, K, sm).ws_bytes;
+  if (M <= 64) {
+    ws = std::max(ws, plan_gemv(M, N, K, false, sm).ws_bytes);
+    if (M <= 32) ws = std::max(ws, plan_gemv(M, N, K, true, sm).ws_bytes);
+  }
+  return ws;
+}
+
+w4_status check_shape(int64_t M, int64_t N, int64_t K, int group) {
+  if (N < 1 || K < 1 || M < 1) return fail(W4_ERR_INVALID_ARG, "sizes must be >= 1 (M=%lld N=%lld K=%lld)",
+                                           (long long)M, (long long)N, (long long)K);
+  if (group != w4::kGroup) return fail(W4_ERR_UNSUPPORTED, "group=%d: only 128 is served", group);
+  if (K % group != 0) return fail(W4_ERR_INVALID_ARG, "K=%lld is not a multiple of the group (%d)", (long long)K, group);
+  const int64_t lim = (int64_t)1 << 40;
+  if (N > lim || K > lim || M > lim || (double)N * (double)K > 9.0e18 || (double)M * (double)N > 4.0e18 ||
+      (double)M * (double)K > 4.0e18)
+    return fail(W4_ERR_INVALID_ARG, "sizes overflow 64-bit indexing");
+  if (K / 64 > INT32_MAX || N > INT32_MAX || M > INT32_MAX)
+    return fail(W4_ERR_INVALID_ARG, "M, N and K/64 must each fit in 31 bits");
+  return W4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *w4_status_string(w4_status s) {
+  switch (s) {
+    case W4_OK: return "W4_OK";
+    case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG";
+    case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED";
+    case W4_ERR_CUDA: return "W4_ERR_CUDA";
+  }
+  return "W4_ERR_UNKNOWN";
+}
+
+const char *w4_last_error(void) { return t_last_error.c_str(); }
+
+w4_status w4_quantize(const void *W, w4_dtype w_dtype, const float *awq_s, int64_t N, int64_t K, int group,
+                      uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(1, N, K, group);
+  if (st != W4_OK) return st;
+  if (w_dtype != W4_F32 && w_dtype != W4_F16 && w_dtype != W4_BF16)
+    return fail(W4_ERR_UNSUPPORTED, "weight dtype %d not served", (int)w_dtype);
+  if (!W || !packed || !scales || !zeros) return fail(W4_ERR_INVALID_ARG, "null W, packed, scales or zeros");
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros) ||
+      (awq_s && !aligned16(awq_s)) || (codes && !aligned16(codes)))
+    return fail(W4_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  e = w4::launch_quantize(W, (int)w_dtype, awq_s, N, K, packed, scales, zeros, codes, sm,
+                          reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return W4_OK;
+}
+
+w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, w4_stream_t stream) {
+  t_last_error.clear();
+  if (N < 1 || K < 1) return fail(W4_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (K % 32 != 0) return fail(W4_ERR_INVALID_ARG, "K=%lld must be a multiple of 32", (long long)K);
+  if ((double)N * (double)K > 9.0e18) return fail(W4_ERR_INVALID_ARG, "sizes overflow");
+  if (!codes || !packed) return fail(W4_ERR_INVALID_ARG, "null codes or packed");
+  if (!aligned16(codes) || !aligned16(packed)) return fail(W4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  e = w4::launch_pack(codes, N, K, packed, sm, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return W4_OK;
+}
+
+size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1 || K % w4::kGroup != 0) return 0;
+  int sm = 0;
+  if (current_sm_count(&sm) != cudaSuccess) sm = 148;
+  return ws_size_all(M, N, K, sm);
+}
+
+w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
+                     const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros, const float *awq_s,
+                     void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(M, N, K, group);
+  if (st != W4_OK) return st;
+  if (x_dtype != W4_F16 && x_dtype != W4_BF16)
+    return fail(W4_ERR_UNSUPPORTED, "activation dtype must be F16 or BF16");
+  if (y_dtype != W4_F32 && y_dtype != W4_BF16) return fail(W4_ERR_UNSUPPORTED, "output dtype must be F32 or BF16");
+  if (!X || !packed || !scales || !zeros || !Y) return fail(W4_ERR_INVALID_ARG, "null X, packed, scales, zeros or Y");
+  if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y) ||
+      (awq_s && !aligned16(awq_s)) || (workspace && !aligned16(workspace)))
+    return fail(W4_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const bool awq = awq_s != nullptr;
+  const GemmPlan plan = plan_gemm(M, N, K, awq, sm);
+  if (plan.path == kPathGemv && !w4::gemv_supports(M, awq))
+    return fail(W4_ERR_UNSUPPORTED, "W4_FORCE_PATH=gemv cannot serve M=%lld%s", (long long)M, awq ? " with AWQ" : "");
+  if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes))
+    return fail(W4_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", plan.ws_bytes,
+                workspace ? workspace_bytes : (size_t)0);
+  uint32_t *counters = static_cast<uint32_t *>(workspace);
+  float *partials = workspace ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kCounterBytes) : nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool xbf16 = x_dtype == W4_BF16;
+
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return fail(W4_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+
+  if (plan.path == kPathGemv) {
+    CUtensorMap tmP, tmS, tmZ;
+    const cuuint32_t estr[2] = {1, 1};
+    {
+      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+      const cuuint32_t box[2] = {plan.ks == 1 ? 64u : 128u, 64u};
+      CUresult r = enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       plan.ks == 1 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
+    }
+    tmS = tmP;
+    tmZ = tmP;
+    if (plan.sc_tma) {
+      const cuuint64_t dims[2] = {(cuuint64_t)(K / w4::kGroup), (cuuint64_t)N};
+      const cuuint64_t strides[1] = {(cuuint64_t)(K / w4::kGroup) * 2};
+      const cuuint32_t box[2] = {8u, 64u};
+      CUresult r = enc(&tmS, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(scales), dims, strides, box,
+                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for scales failed (CUresult %d)", (int)r);
+      r = enc(&tmZ, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(zeros), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for zeros failed (CUresult %d)", (int)r);
+    }
+    w4::GemvParams p{};
+    p.X = X; p.M = M; p.N = N; p.K = K;
+    p.scales = scales; p.zeros = zeros; p.awq_s = awq_s;
+    p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
+    p.ws = partials; p.counters = counters; p.kslices = plan.kslices; p.grid_x = plan.grid_x;
+    e = w4::launch_gemv(tmP, tmS, tmZ, p, xbf16, plan.t8, plan.ks, plan.sc_tma, s);
+    if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
+    return W4_OK;
+  }
+
+  CUtensorMap tmX, tmP;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)plan.bn};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&tmX, xbf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void *>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for X failed (CUresult %d)", (int)r);
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {32, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
+  }
+  w4::TcParams p{};
+  p.M = M; p.N = N; p.K = K;
+  p.scales = scales; p.zeros = zeros; p.awq_s = awq_s;
+  p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
+  p.ws = partials; p.counters = counters; p.splits = plan.splits; p.kb_per_split = plan.kb_per_split;
+  e = w4::launch_gemm_tc(tmX, tmP, p, xbf16, plan.bn, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tensor-core gemm launch");
+  return W4_OK;
+}
+
+w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K,
+                          int group, const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros,
+                          const float *awq_s, void *Y_host, void *Y_dev, w4_dtype y_dtype, void *workspace,
+                          size_t workspace_bytes, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(M, N, K, group);
+  if (st != W4_OK) return st;
+  if (!X_host || !Y_host || !X_dev || !Y_dev) return fail(W4_ERR_INVALID_ARG, "null host or staging buffer");
+  if (x_dtype != W4_F16 && x_dtype != W4_BF16)
+    return fail(W4_ERR_UNSUPPORTED, "activation dtype must be F16 or BF16");
+  if (y_dtype != W4_F32 && y_dtype != W4_BF16) return fail(W4_ERR_UNSUPPORTED, "output dtype must be F32 or BF16");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xb = (size_t)M * K * 2;
+  const size_t yb = (size_t)M * N * (y_dtype == W4_F32 ? 4 : 2);
+  cudaError_t e = cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy X to device");
+  st = w4a16_gemm(X_dev, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y_dev, y_dtype, workspace,
+                  workspace_bytes, stream);
+  if (st != W4_OK) return st;
+  e = cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy Y to host");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return W4_OK;
+}
+
+w4_status w4_device_error(int *flag) {
+  t_last_error.clear();
+  if (!flag) return fail(W4_ERR_INVALID_ARG, "null flag");
+  int v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "device synchronize");
+  e = cudaMemcpyFromSymbol(&v, w4::g_error_flag, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(w4::g_error_flag, &zero, sizeof zero);
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  *flag = v;
+  return W4_OK;
+}
+
+}  // extern "C"

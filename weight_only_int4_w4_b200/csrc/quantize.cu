@@ -1,0 +1,194 @@
+// quantize.cu -- K0: per-group asymmetric uint4 RTN quantize + nibble pack.
+//
+// One warp owns one group of 128 consecutive input channels of one output
+// row (affine map through a scale and a zero point, per group of 128:
+// "LLM inference acceleration" article, section 2.1); each lane holds 4
+// weights.  Optional AWQ prescale w / s[k] is applied on load (ch. 22
+// "Advanced inference optimisation", section 22.3, AWQ equation).  Every
+// step uses IEEE fp32 round-to-nearest intrinsics so the results are bit-exact
+// with the definition in w4.h.  The kernel is HBM-bound: it reads W once and
+// writes 0.5 B of codes + 4 B of scale/zero per 128 weights.
+#include "common.cuh"
+
+namespace w4 {
+
+namespace quant_impl {
+
+template <typename T>
+struct Load4;
+
+template <>
+struct Load4<float> {
+  static __device__ __forceinline__ void run(const float *p, float (&v)[4]) {
+    float4 t = __ldcs(reinterpret_cast<const float4 *>(p));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  }
+};
+
+template <>
+struct Load4<__half> {
+  static __device__ __forceinline__ void run(const __half *p, float (&v)[4]) {
+    uint2 t = __ldcs(reinterpret_cast<const uint2 *>(p));
+    v[0] = __half2float(__ushort_as_half((unsigned short)(t.x & 0xFFFF)));
+    v[1] = __half2float(__ushort_as_half((unsigned short)(t.x >> 16)));
+    v[2] = __half2float(__ushort_as_half((unsigned short)(t.y & 0xFFFF)));
+    v[3] = __half2float(__ushort_as_half((unsigned short)(t.y >> 16)));
+  }
+};
+
+template <>
+struct Load4<__nv_bfloat16> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16 *p, float (&v)[4]) {
+    uint2 t = __ldcs(reinterpret_cast<const uint2 *>(p));
+    v[0] = __uint_as_float(t.x << 16);
+    v[1] = __uint_as_float(t.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(t.y << 16);
+    v[3] = __uint_as_float(t.y & 0xFFFF0000u);
+  }
+};
+
+__device__ __forceinline__ float clamp15(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
+
+constexpr int kQuantUnroll = 4;  // groups in flight per warp
+
+template <typename TW, bool kAwq, bool kCodes>
+__global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W, const float *__restrict__ awq_s,
+                                                       int64_t total_groups, int64_t groups_per_row,
+                                                       uint8_t *__restrict__ packed, uint16_t *__restrict__ scales,
+                                                       uint16_t *__restrict__ zeros, uint8_t *__restrict__ codes) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+
+  for (int64_t base = warp * kQuantUnroll; base < total_groups; base += nwarps * kQuantUnroll) {
+    float v[kQuantUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int64_t gid = base + u;
+      if (gid < total_groups) {
+        Load4<TW>::run(W + gid * kGroup + lane * 4, v[u]);
+        if (kAwq) {
+          const int64_t k = (gid % groups_per_row) * kGroup + lane * 4;
+          const float4 s = __ldg(reinterpret_cast<const float4 *>(awq_s + k));
+          v[u][0] = __fdiv_rn(v[u][0], s.x);
+          v[u][1] = __fdiv_rn(v[u][1], s.y);
+          v[u][2] = __fdiv_rn(v[u][2], s.z);
+          v[u][3] = __fdiv_rn(v[u][3], s.w);
+        }
+      } else {
+        v[u][0] = v[u][1] = v[u][2] = v[u][3] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int64_t gid = base + u;
+      float mn = fminf(fminf(v[u][0], v[u][1]), fminf(v[u][2], v[u][3]));
+      float mx = fmaxf(fmaxf(v[u][0], v[u][1]), fmaxf(v[u][2], v[u][3]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      // scale = fp16((mx - mn) / 15); a zero fp16 scale is taken as 1.0
+      const float sc32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+      __half sc16 = __float2half_rn(sc32);
+      float sc = __half2float(sc16);
+      if (sc == 0.0f) {
+        sc = 1.0f;
+        sc16 = __float2half_rn(1.0f);
+      }
+      const float z = clamp15(rintf(__fdiv_rn(-mn, sc)));
+      uint32_t q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[j] = (uint32_t)clamp15(__fadd_rn(rintf(__fdiv_rn(v[u][j], sc)), z));
+      if (gid < total_groups) {
+        const uint16_t pk = (uint16_t)(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
+        reinterpret_cast<uint16_t *>(packed + gid * (kGroup / 2))[lane] = pk;
+        if (kCodes)
+          reinterpret_cast<uint32_t *>(codes + gid * kGroup)[lane] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+        if (lane == 0) {
+          scales[gid] = __half_as_ushort(sc16);
+          zeros[gid] = __half_as_ushort(__float2half_rn(z));
+        }
+      }
+    }
+  }
+}
+
+// 32 codes (two 16-B loads) -> 16 packed bytes (one 16-B store).
+__global__ void __launch_bounds__(256) pack_kernel(const uint8_t *__restrict__ codes, int64_t chunks,
+                                                   uint8_t *__restrict__ packed) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 a = __ldcs(reinterpret_cast<const uint4 *>(codes + i * 32));
+    const uint4 b = __ldcs(reinterpret_cast<const uint4 *>(codes + i * 32 + 16));
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t r = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t c = in[2 * w + h] & 0x0F0F0F0Fu;  // 4 codes, masked to 4 bits
+        // bytes c0 c1 c2 c3 -> (c0 | c1 << 4) and (c2 | c3 << 4)
+        const uint32_t lo = (c & 0xFFu) | ((c >> 4) & 0xF0u);
+        const uint32_t hi = ((c >> 16) & 0xFFu) | ((c >> 20) & 0xF0u);
+        r |= (lo | (hi << 8)) << (16 * h);
+      }
+      out[w] = r;
+    }
+    __stcs(reinterpret_cast<uint4 *>(packed + i * 16), make_uint4(out[0], out[1], out[2], out[3]));
+  }
+}
+
+int grid_for(int64_t work_items, int items_per_block, int sm_count, int blocks_per_sm) {
+  int64_t need = (work_items + items_per_block - 1) / items_per_block;
+  int64_t cap = (int64_t)sm_count * blocks_per_sm;
+  if (need > cap) need = cap;
+  if (need < 1) need = 1;
+  return (int)need;
+}
+
+template <typename TW>
+cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, uint8_t *packed,
+                              uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
+                              cudaStream_t stream) {
+  const int64_t gpr = K / kGroup;
+  const int64_t total = N * gpr;
+  const int grid = grid_for(total, 8 * kQuantUnroll, sm_count, 8);
+  const TW *w = static_cast<const TW *>(W);
+  if (awq_s) {
+    if (codes)
+      quantize_kernel<TW, true, true><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+    else
+      quantize_kernel<TW, true, false><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+  } else {
+    if (codes)
+      quantize_kernel<TW, false, true><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+    else
+      quantize_kernel<TW, false, false><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace quant_impl
+
+// dtype: 0 = fp32, 1 = fp16, 2 = bf16
+cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, uint8_t *packed,
+                            uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count, cudaStream_t stream) {
+  switch (dtype) {
+    case 0: return quant_impl::launch_quantize_t<float>(W, awq_s, N, K, packed, scales, zeros, codes, sm_count, stream);
+    case 1: return quant_impl::launch_quantize_t<__half>(W, awq_s, N, K, packed, scales, zeros, codes, sm_count, stream);
+    default: return quant_impl::launch_quantize_t<__nv_bfloat16>(W, awq_s, N, K, packed, scales, zeros, codes, sm_count, stream);
+  }
+}
+
+cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,
+                        cudaStream_t stream) {
+  const int64_t chunks = N * K / 32;
+  const int grid = quant_impl::grid_for(chunks, 256, sm_count, 8);
+  quant_impl::pack_kernel<<<grid, 256, 0, stream>>>(codes, chunks, packed);
+  return cudaGetLastError();
+}
+
+}  // namespace w4

@@ -1,0 +1,158 @@
+"""Python binding of libw4 (argument marshalling only).
+
+Every function here forwards torch tensors' device pointers, sizes and the
+current CUDA stream to the C ABI declared in ``include/w4.h``; all arithmetic
+runs in the library's CUDA kernels.  There is no fallback: if ``libw4.so`` is
+not built, importing this module raises.
+
+Names follow the C ABI: ``w4_quantize``, ``w4_pack``, ``w4a16_gemm``,
+``w4a16_gemm_workspace_size``, ``w4a16_gemm_host``, ``w4_device_error``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libw4.so is not built ({_LIB_PATH}); run weight_only_int4_w4_b200.build.build_library()")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+_P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+_lib.w4_quantize.argtypes = [_P, ctypes.c_int, _P, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P]
+_lib.w4_pack.argtypes = [_P, _I64, _I64, _P, _P]
+_lib.w4a16_gemm.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, ctypes.c_int,
+                            _P, _SZ, _P]
+_lib.w4a16_gemm_host.argtypes = [_P, _P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, _P,
+                                 ctypes.c_int, _P, _SZ, _P]
+_lib.w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
+_lib.w4a16_gemm_workspace_size.restype = _SZ
+_lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+_lib.w4_status_string.argtypes = [ctypes.c_int]
+_lib.w4_status_string.restype = ctypes.c_char_p
+_lib.w4_last_error.restype = ctypes.c_char_p
+for _f in ("w4_quantize", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4_device_error"):
+    getattr(_lib, _f).restype = ctypes.c_int
+
+W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
+W4_F32, W4_F16, W4_BF16 = 0, 1, 2
+_DT = {torch.float32: W4_F32, torch.float16: W4_F16, torch.bfloat16: W4_BF16}
+GROUP = 128
+
+LIB_PATH = _LIB_PATH
+lib = _lib
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.w4_last_error().decode()
+        super().__init__(f"{where}: {_lib.w4_status_string(status).decode()}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != W4_OK:
+        raise W4Error(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def w4_status_string(status: int) -> str:
+    return _lib.w4_status_string(status).decode()
+
+
+def w4_quantize(W: torch.Tensor, awq_s: torch.Tensor | None = None, group: int = GROUP,
+                return_codes: bool = False, stream=None):
+    """Quantize + pack W [N, K] (fp32/fp16/bf16, CUDA).  Returns (packed u8 [N,K/2],
+    scales f16 [N,K/G], zeros f16 [N,K/G]) and, with return_codes, codes u8 [N,K]."""
+    assert W.is_cuda and W.dim() == 2 and W.is_contiguous() and W.dtype in _DT
+    N, K = W.shape
+    dev = W.device
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    zeros = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    codes = torch.empty((N, K), dtype=torch.uint8, device=dev) if return_codes else None
+    if awq_s is not None:
+        assert awq_s.is_cuda and awq_s.dtype == torch.float32 and awq_s.is_contiguous()
+    _check(_lib.w4_quantize(_ptr(W), _DT[W.dtype], _ptr(awq_s), N, K, group, _ptr(packed), _ptr(scales),
+                            _ptr(zeros), _ptr(codes), _stream(stream)), "w4_quantize")
+    return (packed, scales, zeros, codes) if return_codes else (packed, scales, zeros)
+
+
+def w4_pack(codes: torch.Tensor, stream=None) -> torch.Tensor:
+    assert codes.is_cuda and codes.dtype == torch.uint8 and codes.dim() == 2 and codes.is_contiguous()
+    N, K = codes.shape
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=codes.device)
+    _check(_lib.w4_pack(_ptr(codes), N, K, _ptr(packed), _stream(stream)), "w4_pack")
+    return packed
+
+
+def w4a16_gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.w4a16_gemm_workspace_size(M, N, K))
+
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def workspace(M: int, N: int, K: int, device, stream=None) -> torch.Tensor | None:
+    """A zero-filled workspace (cached per device and stream) large enough for (M, N, K).
+    The library leaves it zero-filled after every call, so it can be reused."""
+    need = w4a16_gemm_workspace_size(M, N, K)
+    if need == 0:
+        return None
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (torch.device(device), s.cuda_stream)
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < need:
+            buf = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=device)
+            _ws_cache[key] = buf
+    return buf
+
+
+def w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+               awq_s: torch.Tensor | None = None, out_dtype=torch.float32, out: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None, group: int = GROUP, stream=None) -> torch.Tensor:
+    """Y = X . W^T with W^ dequantized on the fly.  X [M,K] fp16/bf16 (CUDA)."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.dtype in (torch.float16, torch.bfloat16)
+    M, K = X.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    if ws is None:
+        ws = workspace(M, N, K, X.device, stream)
+    _check(_lib.w4a16_gemm(_ptr(X), _DT[X.dtype], M, N, K, group, _ptr(packed), _ptr(scales), _ptr(zeros),
+                           _ptr(awq_s), _ptr(out), _DT[out.dtype], _ptr(ws), 0 if ws is None else ws.numel(),
+                           _stream(stream)), "w4a16_gemm")
+    return out
+
+
+def w4a16_gemm_host(X_host: torch.Tensor, X_dev: torch.Tensor, packed, scales, zeros, Y_host: torch.Tensor,
+                    Y_dev: torch.Tensor, awq_s=None, ws=None, group: int = GROUP, stream=None) -> torch.Tensor:
+    """End-to-end call with pinned host X and Y: H2D copy, fused GEMM, D2H copy, wait."""
+    M, K = X_host.shape
+    N = packed.shape[0]
+    if ws is None:
+        ws = workspace(M, N, K, X_dev.device, stream)
+    _check(_lib.w4a16_gemm_host(_ptr(X_host), _ptr(X_dev), _DT[X_host.dtype], M, N, K, group, _ptr(packed),
+                                _ptr(scales), _ptr(zeros), _ptr(awq_s), _ptr(Y_host), _ptr(Y_dev),
+                                _DT[Y_host.dtype], _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "w4a16_gemm_host")
+    return Y_host
+
+
+def w4_device_error() -> int:
+    flag = ctypes.c_int(0)
+    _check(_lib.w4_device_error(ctypes.byref(flag)), "w4_device_error")
+    return flag.value
