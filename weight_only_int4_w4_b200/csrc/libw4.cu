@@ -87,17 +87,22 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 enum Path { kPathGemv = 1, kPathTc = 2 };
 
-// Workspace layout: [0, 64 KiB) split-K arrival counters, then fp32 partials.
-// The counter region is the same for every call, so partials left behind by
-// one call never land on the counters of the next; counters are reset to zero
-// by the last CTA (or warp) that uses them.
-constexpr size_t kCounterBytes = 65536;
-constexpr int64_t kMaxCounters = kCounterBytes / 4;
+// Workspace layout: [0, 64 KiB) split-K arrival counters (one per 16-row block),
+// [64 KiB, 128 KiB) decode scheduler counters (two per k-slice), then fp32
+// partials.  The counter regions are the same for every call, so partials left
+// behind by one call never land on the counters of the next; every counter is
+// reset to zero by the last CTA (or warp) that uses it.
+constexpr size_t kSplitCounterBytes = 65536;
+constexpr size_t kSchedBytes = 65536;
+constexpr size_t kCounterBytes = kSplitCounterBytes + kSchedBytes;
+constexpr int64_t kMaxSplitCounters = kSplitCounterBytes / 4;
+constexpr int64_t kMaxKslices = kSchedBytes / 8;
+constexpr int kGemvXsMax = 40 * 1024;  // staged-activation budget per CTA
 
 struct GemmPlan {
   int path = 0;
   // K1
-  int t8 = 1, ks = 1, kslices = 1, grid_x = 1;
+  int t8 = 1, kr = 2, kslices = 1, grid_x = 1, xs_bytes = 0;
   bool sc_tma = false;
   // K2
   int bn = 256, splits = 1, kb_per_split = 1;
@@ -115,9 +120,9 @@ int forced_path() {
   return 0;
 }
 
-// CTAs of the decode kernel that fit on one SM (shared memory bound).
-int gemv_ctas_per_sm(int ks) {
-  const int per = w4::gemv_smem_bytes(ks) + 1024;
+// CTAs of the decode kernel resident per SM (shared memory and a 4-CTA register budget).
+int gemv_ctas_per_sm(int xs_bytes) {
+  const int per = w4::gemv_smem_bytes(xs_bytes) + 1024;
   int n = (228 * 1024) / per;
   return n < 1 ? 1 : (n > 4 ? 4 : n);
 }
@@ -130,47 +135,36 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   const int64_t RT = cdiv(N, 64);
   const int64_t RB16 = cdiv(N, 16);
   p.sc_tma = (Kg % 8) == 0;
-  double best = 1e300;
-  for (int ks = w4::gemv_max_ks(p.t8, awq); ks >= 1; ks /= 2) {
-    const int64_t kslices = cdiv(Kg, ks);
-    if (kslices > 1 && RB16 > kMaxCounters) continue;
-    const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(ks);
-    const double task_bytes = 64.0 * ks * (64 + 4);
-    const double split_bytes = kslices > 1 ? 2.0 * 4.0 * (double)kslices * M * N / sm : 0.0;
-    for (int64_t gx = std::min<int64_t>(RT, std::max<int64_t>(1, slots / kslices)); gx >= 1; --gx) {
-      const int64_t c = cdiv(RT, gx);
-      if (gx < RT && cdiv(RT, gx + 1) == c) continue;  // same tasks per CTA with more CTAs: keep the larger grid
-      const int64_t ctas = gx * kslices;
-      // bytes streamed by the busiest SM (+ split-K partials), + a per-wave start cost
-      const double est = (double)cdiv(ctas, sm) * c * task_bytes + split_bytes +
-                         4096.0 * (double)(cdiv(ctas, slots) - 1) * 64;
-      if (est < best * (1 - 1e-9)) {
-        best = est;
-        p.ks = ks;
-        p.kslices = (int)kslices;
-        p.grid_x = (int)gx;
-      }
-      if (c > 4 * cdiv(RT * kslices, sm) + 8) break;
-    }
+  // longest even k-slice whose activations fit the staging budget
+  int64_t kr_max = std::min<int64_t>(Kg + (Kg & 1), 4096);
+  while (kr_max > 2 && w4::gemv_xs_bytes((int)kr_max, M, awq) > kGemvXsMax) kr_max -= 2;
+  // shortest k-slices that still leave ~1.5 tiles per resident CTA (dynamic scheduling balances the rest)
+  int64_t kr = kr_max;
+  for (;;) {
+    const int64_t ks = cdiv(Kg, kr);
+    const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(w4::gemv_xs_bytes((int)kr, M, awq));
+    if (RT * ks * 2 >= slots * 3 || kr <= 2) break;
+    kr -= 2;
   }
-  // tuning overrides: W4_GEMV_KS (groups per task) and W4_GEMV_GX (CTAs per k-slice)
-  if (const char *e = getenv("W4_GEMV_KS")) {
-    const int ks = atoi(e);
-    if ((ks == 1 || ks == 2 || ks == 4) && ks <= w4::gemv_max_ks(p.t8, awq)) {
-      p.ks = ks;
-      p.kslices = (int)cdiv(Kg, ks);
-      p.grid_x = (int)std::min<int64_t>(RT, std::max<int64_t>(1, (int64_t)sm * gemv_ctas_per_sm(ks) / p.kslices));
-    }
+  if (const char *e = getenv("W4_GEMV_KR")) {  // tuning override
+    const int64_t v = atoi(e);
+    if (v >= 2 && v % 2 == 0 && v <= kr_max) kr = v;
   }
-  if (const char *e = getenv("W4_GEMV_GX")) {
-    const int gx = atoi(e);
-    if (gx >= 1) p.grid_x = (int)std::min<int64_t>(RT, gx);
+  int64_t ks = cdiv(Kg, kr);
+  if ((ks > 1 && RB16 > kMaxSplitCounters) || ks > kMaxKslices) {  // counters: fall back to the longest slices
+    kr = kr_max;
+    ks = cdiv(Kg, kr);
   }
-  if (p.kslices > 1 && RB16 > kMaxCounters) {  // overrides may not exceed the counter region
-    p.ks = w4::gemv_max_ks(p.t8, awq);
-    p.kslices = (int)cdiv(Kg, p.ks);
+  p.kr = (int)kr;
+  p.kslices = (int)ks;
+  p.xs_bytes = w4::gemv_xs_bytes(p.kr, M, awq);
+  const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(p.xs_bytes);
+  p.grid_x = (int)std::min<int64_t>(RT, std::max<int64_t>(1, slots / ks));
+  if (const char *e = getenv("W4_GEMV_GX")) {  // tuning override
+    const int v = atoi(e);
+    if (v >= 1) p.grid_x = (int)std::min<int64_t>(RT, v);
   }
-  if (p.kslices > 1) p.ws_bytes = kCounterBytes + (size_t)p.kslices * M * N * 4;
+  p.ws_bytes = kCounterBytes + (ks > 1 ? (size_t)ks * M * N * 4 : 0);
   return p;
 }
 
@@ -181,7 +175,7 @@ GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, int sm) {
   const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
   const int64_t total_kb = K / 64;
   int64_t splits = 1;
-  if (tiles < sm && tiles <= kMaxCounters) splits = std::max<int64_t>(1, std::min<int64_t>(sm / tiles, total_kb / 8));
+  if (tiles < sm && tiles <= kMaxSplitCounters) splits = std::max<int64_t>(1, std::min<int64_t>(sm / tiles, total_kb / 8));
   int64_t kbps = cdiv(total_kb, splits);
   splits = cdiv(total_kb, kbps);
   p.splits = (int)splits;
@@ -206,8 +200,9 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   GemmPlan p = plan_gemm_raw(M, N, K, awq, sm);
   if (getenv("W4_DEBUG_PLAN")) {
     if (p.path == kPathGemv)
-      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld decode: t8=%d ks=%d kslices=%d grid_x=%d scale_tma=%d ws=%zu\n",
-              (long long)M, (long long)N, (long long)K, p.t8, p.ks, p.kslices, p.grid_x, (int)p.sc_tma, p.ws_bytes);
+      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld decode: t8=%d kr=%d kslices=%d grid_x=%d xs=%d scale_tma=%d ws=%zu\n",
+              (long long)M, (long long)N, (long long)K, p.t8, p.kr, p.kslices, p.grid_x, p.xs_bytes, (int)p.sc_tma,
+              p.ws_bytes);
     else
       fprintf(stderr, "[w4] M=%lld N=%lld K=%lld tensor-core: bn=%d splits=%d kb_per_split=%d ws=%zu\n",
               (long long)M, (long long)N, (long long)K, p.bn, p.splits, p.kb_per_split, p.ws_bytes);
@@ -333,11 +328,10 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
     {
       const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
       const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      const cuuint32_t box[2] = {plan.ks == 1 ? 64u : 128u, 64u};
+      const cuuint32_t box[2] = {128u, 64u};
       CUresult r = enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       plan.ks == 1 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
       if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
     }
     tmS = tmP;
@@ -359,8 +353,11 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
     p.X = X; p.M = M; p.N = N; p.K = K;
     p.scales = scales; p.zeros = zeros; p.awq_s = awq_s;
     p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
-    p.ws = partials; p.counters = counters; p.kslices = plan.kslices; p.grid_x = plan.grid_x;
-    e = w4::launch_gemv(tmP, tmS, tmZ, p, xbf16, plan.t8, plan.ks, plan.sc_tma, s);
+    p.ws = partials; p.counters = counters;
+    p.sched = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kSplitCounterBytes);
+    p.kslices = plan.kslices; p.kr = plan.kr; p.grid_x = plan.grid_x; p.xs_bytes = plan.xs_bytes;
+    p.x_bf16 = xbf16;
+    e = w4::launch_gemv(tmP, tmS, tmZ, p, plan.t8, plan.sc_tma, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
     return W4_OK;
   }
