@@ -94,7 +94,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 // read stays off the normal path) if another wait has already given up, so a
 // broken pipeline ends quickly instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int err_bit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
@@ -107,6 +107,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int er
   atomicOr(&g_error_flag, err_bit);
   return false;
 }
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Wait until the grids this one depends on have completed and their writes are
+// visible (returns at once when the launch had no programmatic dependency).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel in the stream start launching (its CTAs still wait for free resources).
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,

@@ -7,36 +7,39 @@
 // eight weights on dequantization.
 //
 //   * Grid: (CTAs per k-slice) x (k-slices).  A CTA owns one k-slice of KR
-//     quantization groups (KR x 128 input channels).  At start its 4 compute
+//     quantization groups (KR x 128 input channels).  At start its compute
 //     warps stage the activations of that k-slice in shared memory as fp16
 //     mma.sync B fragments (see "activation staging" below).
 //   * Work unit ("task"): 64 output rows x the CTA's k-slice.  Row tiles are
 //     handed out by an atomic counter per k-slice, so faster CTAs take more.
-//     Warp 4 (producer) streams each tile's packed codes [64 rows x 128 B =
-//     2 groups per stage, 128-byte swizzle] and fp16 scales / zeros [64 rows x
-//     8 groups] through an NST-deep shared-memory ring with TMA; a header per
-//     stage tells the compute warps which tile and k-chunk it holds.
-//   * Warps 0..3 (compute) own 16 rows each.  Dequantization: a 32-bit word
-//     holds 8 codes; with the fp16 magic 0x6400 one LOP3 yields the exact fp16
-//     pairs 1024 + q for the low nibbles (even k) and 1024 + 16 q for the high
-//     nibbles (odd k) in place, and one shift exposes the other byte pair: one
-//     SHF + four LOP3 per 8 weights.  The tensor core then computes
+//     Warp 8 (producer) streams each tile's packed codes [64 rows x 256 B =
+//     4 groups per stage, two 128-byte-swizzled boxes] and fp16 scales / zeros
+//     [64 rows x 8 groups] through an NST-deep shared-memory ring with TMA; a
+//     header per stage tells the compute warps which tile and k-chunk it holds.
+//   * Warps 0..7 (compute): warp (b, h) owns rows 16b..16b+15 of the tile and
+//     groups 2h, 2h+1 of every stage (two independent MMA streams).  A 32-bit
+//     word holds 8 codes; with the fp16 magic 0x6400 one LOP3 yields the exact
+//     fp16 pairs 1024 + q for the low nibbles (even k) and 1024 + 16 q for the
+//     high nibbles (odd k) in place, and one shift exposes the other byte pair:
+//     one SHF + four LOP3 per 8 weights.  The tensor core then computes
 //         D = sum_even (1024 + q) x' + sum_odd (1024 + 16 q) (x'/16)
 //           = sum_k q x' + 1024 * sum_k B_k          (B = the staged fragment values)
 //     exactly up to fp32 accumulation, and per group the result is promoted
 //     once:  y' += scale * (D - P - z * S),  P = 1024 * sum B, S = sum x',
 //     i.e. scale * sum_k (q - z) x': the dequantize-then-matmul of the
 //     weight-only path (ch. 22, section 22.3) without rounding any weight.
+//     At the end of a tile the two warps of a row block add their halves
+//     through shared memory (bounded mbarrier hand-off).
 //   * Activation staging: x' = x * s (AWQ, ch. 22 section 22.3) * 2^e, with a
 //     power of two e per token and k-slice chosen so max|x'| lies in
 //     [2^13, 2^14): bf16 and fp16 inputs both convert exactly to fp16 (bar
 //     values 2^27 times below the token's maximum), and the result is scaled
 //     back by 2^-e exactly.  With AWQ, x' is split into fp16 high + low parts.
-//   * Split-K (k-slices > 1): each warp stores its fp32 partials for a tile,
-//     then one lane announces them with a release atomic on the tile's 16-row
-//     block counter; the ticket is read one task later (hiding the round trip)
-//     and the last of the k-slices sums the partials into Y.  No warp ever
-//     waits on another CTA.
+//   * Split-K (k-slices > 1): the row block's fp32 partials are stored, then
+//     one lane announces them with a release atomic on the 16-row block's
+//     counter; the ticket is read one tile later (hiding the round trip) and
+//     the last of the k-slices sums the partials into Y.  No warp ever waits
+//     on another CTA.
 //
 // mma.sync m16n8k16 fragments (g = lane / 4, t = lane % 4):
 //   A regs: {row g, k 2t..2t+1}, {row g+8, k 2t..}, {row g, k 2t+8..}, {row g+8, k 2t+8..}
@@ -58,25 +61,27 @@ struct GemvParams {
   const float *awq_s;
   void *Y;
   int y_bf16;
-  int x_bf16;
   float *ws;           // [kslices][M][N] fp32 partials (split-K only)
   uint32_t *counters;  // [ceil(N/16)] split-K arrival counters
   uint32_t *sched;     // [2 * kslices]: next row tile, CTAs done fetching (per k-slice)
   int kslices;
-  int kr;              // groups per k-slice (even)
+  int kr;              // groups per k-slice (multiple of 4)
   int grid_x;          // CTAs per k-slice
   int xs_bytes;        // shared-memory bytes of the staged activations
 };
 
 namespace gemv_impl {
 
-constexpr int kRows = 64;     // rows per task (4 compute warps x 16)
-constexpr int kSG = 2;        // groups per pipeline stage (128 bytes of codes per row)
-constexpr int kNst = 6;       // pipeline stages
-constexpr int kPBytes = kRows * kSG * 64;  // 8 KiB of codes per stage
+constexpr int kRows = 64;      // rows per task
+constexpr int kSG = 4;         // groups per pipeline stage (256 bytes of codes per row)
+constexpr int kNst = 4;        // pipeline stages
+constexpr int kBox = kRows * 128;          // one 128-byte-swizzled box: 2 groups x 64 rows
+constexpr int kPBytes = 2 * kBox;          // 16 KiB of codes per stage
 constexpr int kSBytes = kRows * 8 * 2;     // 8-group scale (or zero) box per stage
 constexpr int kStage = kPBytes + 2 * kSBytes;
 constexpr int kMaxTok = 64;
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = kComputeWarps * 32;
 
 // Staged activations for KR groups and M tokens: B fragments [g][tok][part][t][16 u32],
 // then (P, S) float pairs [g][tok], then the per-token exponents.
@@ -84,8 +89,10 @@ __host__ __device__ constexpr int xs_frag_bytes(int kr, int m, bool awq) { retur
 __host__ __device__ constexpr int xs_bytes_for(int kr, int m, bool awq) {
   return xs_frag_bytes(kr, m, awq) + kr * m * 8 + kMaxTok * 4;
 }
-__host__ __device__ constexpr int smem_bytes_for(int xs_bytes) {
-  return 1024 + kNst * kStage + xs_bytes + kNst * 16 + 2 * kNst * 8 + 64;
+// pair-reduction buffer: [4 row blocks][32 lanes][T8 octets][4] floats
+__host__ __device__ constexpr int pair_bytes_for(int t8) { return 4 * 32 * t8 * 4 * 4; }
+__host__ __device__ constexpr int smem_bytes_for(int xs_bytes, int t8) {
+  return 1024 + kNst * kStage + xs_bytes + pair_bytes_for(t8) + kNst * 16 + 2 * kNst * 8 + 8 * 8 + 64;
 }
 
 // D (+)= A * B on fp16 operands with fp32 accumulation; `first` starts from zero.
@@ -105,23 +112,33 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
   }
 }
 
-__device__ __forceinline__ void named_bar_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ void atom_release_add(uint32_t *addr, uint32_t v, uint32_t &old) {
   asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ float x_to_f32(uint32_t bits16, bool bf16) {
-  return bf16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((unsigned short)bits16));
+// Two 16-bit inputs of a 32-bit word (channel 2j in the low half) -> two floats.
+template <bool kBf16>
+__device__ __forceinline__ float2 pair_to_f32(uint32_t w) {
+  if constexpr (kBf16) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  } else {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+  }
 }
 
-__device__ __forceinline__ uint32_t f16_bits(float v) { return (uint32_t)__half_as_ushort(__float2half_rn(v)); }
+// fp32 pair -> fp16x2 word (round to nearest even), low half = first.
+__device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
 
 // 2^e with e an integer in [-126, 127], exact.
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
 
-template <int T8, bool kAwq, bool kScTma>
-__global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUtensorMap tmP,
+template <int T8, bool kBf16, bool kAwq, bool kScTma>
+__global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_kernel(const __grid_constant__ CUtensorMap tmP,
                                                    const __grid_constant__ CUtensorMap tmS,
                                                    const __grid_constant__ CUtensorMap tmZ, const GemvParams p) {
   constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
@@ -134,9 +151,12 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
   uint32_t *xs = reinterpret_cast<uint32_t *>(smem + kNst * kStage);
   float2 *ps = reinterpret_cast<float2 *>(smem + kNst * kStage + xs_frag_bytes(p.kr, Mi, kAwq));
   int *xexp = reinterpret_cast<int *>(smem + kNst * kStage + xs_frag_bytes(p.kr, Mi, kAwq) + p.kr * Mi * 8);
-  int *hdr = reinterpret_cast<int *>(smem + kNst * kStage + p.xs_bytes);  // [kNst][4]
+  float *pairbuf = reinterpret_cast<float *>(smem + kNst * kStage + p.xs_bytes);  // [4][32][T8][4]
+  int *hdr = reinterpret_cast<int *>(smem + kNst * kStage + p.xs_bytes + pair_bytes_for(T8));  // [kNst][4]
   uint64_t *full = reinterpret_cast<uint64_t *>(hdr + 4 * kNst);
   uint64_t *empty = full + kNst;
+  uint64_t *pair_full = empty + kNst;    // [4]
+  uint64_t *pair_empty = pair_full + 4;  // [4]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -152,14 +172,18 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNst; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 4);
+      mbar_init(&empty[s], kComputeWarps);
+    }
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(&pair_full[b], 1);
+      mbar_init(&pair_empty[b], 1);
     }
     fence_barrier_init();
   }
   if (threadIdx.x < kMaxTok) xexp[threadIdx.x] = 0;  // max |x'| bits per token (first pass)
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == kComputeWarps) {
     // ---------------- producer: fetch row tiles, drive the TMA ring
     if (lane == 0) {
       prefetch_tensormap(&tmP);
@@ -169,15 +193,21 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
       }
       uint32_t *next = p.sched + 2 * kslice;
       uint32_t *fin = next + 1;
-      int64_t rt = atomicAdd(next, 1u);
-      int64_t it = 0;
+      // The first tile of every CTA is static (tile = blockIdx.x), so its weights
+      // can stream before the preceding kernel in the stream has finished; the
+      // scheduler counters (workspace) are touched only after the dependency wait.
+      int64_t rt = blockIdx.x;
+      bool waited = false;
+      int s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       while (ok) {
         const bool have = rt < RT;
-        const int64_t rt_next = have ? (int64_t)atomicAdd(next, 1u) : RT;  // overlaps the issue below
+        int64_t rt_next = RT;
+        if (waited && have) rt_next = (int64_t)gridDim.x + atomicAdd(next, 1u);  // overlaps the issue below
         if (!have) {
-          const int s = (int)(it % kNst);
-          const uint32_t ph = (uint32_t)(it / kNst) & 1u;
+          if (!waited) grid_dependency_wait();
+          waited = true;
           if (mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) {
             hdr[4 * s] = -1;  // end of work
             mbar_arrive(&full[s]);
@@ -185,9 +215,7 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
           break;
         }
         const int32_t row0 = (int32_t)(rt * kRows);
-        for (int c = 0; c < nst_task; ++c, ++it) {
-          const int s = (int)(it % kNst);
-          const uint32_t ph = (uint32_t)(it / kNst) & 1u;
+        for (int c = 0; c < nst_task; ++c) {
           if (!mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) { ok = false; break; }
           hdr[4 * s + 0] = (int)rt;
           hdr[4 * s + 1] = c;
@@ -195,14 +223,25 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
           mbar_arrive_expect_tx(&full[s], kScTma ? kStage : kPBytes);
           const int64_t gs = g_first + (int64_t)c * kSG;
           tma_load_2d(st, &tmP, &full[s], (int32_t)(gs * 64), row0);
+          tma_load_2d(st + kBox, &tmP, &full[s], (int32_t)(gs * 64 + 128), row0);
           if constexpr (kScTma) {
             const int32_t gx0 = (int32_t)(gs & ~(int64_t)7);
             tma_load_2d(st + kPBytes, &tmS, &full[s], gx0, row0);
             tma_load_2d(st + kPBytes + kSBytes, &tmZ, &full[s], gx0, row0);
           }
+          if (++s == kNst) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!waited) {  // first (static) tile issued: now wait, then fetch the next one
+          grid_dependency_wait();
+          waited = true;
+          rt_next = (int64_t)gridDim.x + atomicAdd(next, 1u);
         }
         rt = rt_next;
       }
+      grid_launch_dependents();  // all of this CTA's loads are issued
       // every CTA of this k-slice is done fetching: the last one resets the scheduler
       const uint32_t prev = atomicAdd(fin, 1u);
       if (prev == gridDim.x - 1) {
@@ -213,29 +252,40 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
     return;
   }
 
-  // ---------------- compute warps: activation staging
+  // ---------------- compute warps: activation staging.  A unit is 32 channels
+  // (group gl, token tok, quarter tt); every lane runs the same number of rounds
+  // (the shuffles need whole warps) and a round's 4-lane quads are all valid or
+  // all idle, since the thread count and the unit count are multiples of 4.
+  grid_dependency_wait();  // X (and Y, the workspace) may come from the preceding kernel
   const uint16_t *xg = static_cast<const uint16_t *>(p.X);
-  const int units = ng * Mi * 4;  // (group, token, t): 32 channels each
+  const int units = ng * Mi * 4;
   // pass 1: per-token max |x * s| over the k-slice -> power-of-two exponent
-  for (int u = threadIdx.x; u < units; u += 128) {
-    const int tt = u & 3;
-    const int tok = (u >> 2) % Mi;
-    const int gl = (u >> 2) / Mi;
-    const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
-    const uint16_t *src = xg + (int64_t)tok * K + k0;
-    float mx = 0.0f;
+  for (int r0 = 0; r0 < units; r0 += kComputeThreads) {
+    const int u = r0 + threadIdx.x;
+    if (u < units) {
+      const int tt = u & 3;
+      const int tok = (u >> 2) % Mi;
+      const int gl = (u >> 2) / Mi;
+      const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
+      const uint4 *src = reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + k0);
+      float mx = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + 8 * c));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      for (int c = 0; c < 4; ++c) {
+        const uint4 v = __ldg(src + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float xv = x_to_f32((w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, p.x_bf16);
-        if (kAwq) xv *= __ldg(p.awq_s + k0 + 8 * c + e);
-        mx = fmaxf(mx, fabsf(xv));
+        for (int e = 0; e < 4; ++e) {
+          float2 f = pair_to_f32<kBf16>(w[e]);
+          if constexpr (kAwq) {
+            const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 8 * c + 2 * e));
+            f.x *= s2.x;
+            f.y *= s2.y;
+          }
+          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
       }
+      atomicMax(&xexp[tok], __float_as_int(mx));  // non-negative floats order like their bits
     }
-    atomicMax(&xexp[tok], __float_as_int(mx));  // non-negative floats order like their bits
   }
   named_bar_compute();
   if (threadIdx.x < Mi) {
@@ -247,64 +297,68 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
     xexp[threadIdx.x] = e;
   }
   named_bar_compute();
-  // pass 2: x' = x * s * 2^e as fp16 fragments (odd channels / 16), group sums P and S.
-  // Every lane runs the same number of rounds (the shuffles below need the whole
-  // warp); a round's 4-lane (group, token) quads are all valid or all idle
-  // because both 128 and the unit count are multiples of 4.
-  for (int r0 = 0; r0 < units; r0 += 128) {
+  // pass 2: x' = x * s * 2^e as fp16 fragments (odd channels / 16), group sums P and S
+  for (int r0 = 0; r0 < units; r0 += kComputeThreads) {
     const int u = r0 + threadIdx.x;
     const bool valid = u < units;
     const int tt = u & 3;
     const int tok = valid ? (u >> 2) % Mi : 0;
     const int gl = valid ? (u >> 2) / Mi : 0;
-    const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
-    const uint16_t *src = xg + (int64_t)tok * K + k0;
-    const float sc2 = exp2i(xexp[tok]);
-    uint32_t hbits[kParts][32];
     float sumB = 0.0f, sumX = 0.0f;
     if (valid) {
+      const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
+      const uint4 *src = reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + k0);
+      const int e = xexp[tok];
+      const float se = exp2i(e), so = exp2i(e - 4);  // even channels x 2^e, odd x 2^(e-4)
+      uint32_t hw[kParts][16];  // fp16 pairs (channels 2j, 2j+1) of the 32
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + 8 * c));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      for (int c = 0; c < 4; ++c) {
+        const uint4 v = __ldg(src + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = 8 * c + e;  // channel offset within the 32
-        float xv = x_to_f32((w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, p.x_bf16);
-        if (kAwq) xv *= __ldg(p.awq_s + k0 + j);
-        float xp = xv * sc2;                   // exact power-of-two scaling
-        if (j & 1) xp *= 0.0625f;              // odd channels pair with 1024 + 16 q
-        const uint32_t hb = f16_bits(xp);
-        const float hv = __half2float(__ushort_as_half((unsigned short)hb));
-        hbits[0][j] = hb;
-        float used = hv;
-        if constexpr (kAwq) {
-          const uint32_t lb = f16_bits(xp - hv);
-          hbits[kParts - 1][j] = lb;
-          used += __half2float(__ushort_as_half((unsigned short)lb));
+        for (int e2 = 0; e2 < 4; ++e2) {
+          float2 f = pair_to_f32<kBf16>(w[e2]);
+          if constexpr (kAwq) {
+            const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 8 * c + 2 * e2));
+            f.x *= s2.x;
+            f.y *= s2.y;
+          }
+          f.x *= se;  // exact power-of-two scaling
+          f.y *= so;
+          const uint32_t hi = f16x2_bits(f.x, f.y);
+          const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+          hw[0][4 * c + e2] = hi;
+          float be = hv.x, bo = hv.y;
+          if constexpr (kAwq) {
+            const uint32_t lo = f16x2_bits(f.x - hv.x, f.y - hv.y);
+            const float2 lv = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+            hw[kParts - 1][4 * c + e2] = lo;
+            be += lv.x;
+            bo += lv.y;
+          }
+          sumB += be + bo;
+          sumX += fmaf(16.0f, bo, be);
         }
-        sumB += used;
-        sumX += (j & 1) ? used * 16.0f : used;
+      }
+      // B fragments for MMA block b = 2i + h: B0 = (v[8i+2h], v[8i+2h+4]), B1 = (v[8i+2h+1], v[8i+2h+5]);
+      // word 4i + h holds channels (8i+2h, 8i+2h+1) and word 4i + h + 2 holds (8i+2h+4, 8i+2h+5)
+#pragma unroll
+      for (int pp = 0; pp < kParts; ++pp) {
+        uint32_t o16[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t wa = hw[pp][4 * i + h], wb = hw[pp][4 * i + h + 2];
+            o16[4 * i + 2 * h + 0] = __byte_perm(wa, wb, 0x5410);
+            o16[4 * i + 2 * h + 1] = __byte_perm(wa, wb, 0x7632);
+          }
+        uint4 *dst = reinterpret_cast<uint4 *>(xs + ((((gl * Mi + tok) * kParts + pp) * 4 + tt) * 16));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o16[4 * c], o16[4 * c + 1], o16[4 * c + 2], o16[4 * c + 3]);
       }
     }
-    // B fragments for MMA block b = 2i + h: B0 = (v[8i+2h], v[8i+2h+4]), B1 = (v[8i+2h+1], v[8i+2h+5])
-#pragma unroll
-    for (int pp = 0; pp < kParts; ++pp) {
-      uint32_t o16[16];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int base = 8 * i + 2 * h;
-          o16[4 * i + 2 * h + 0] = hbits[pp][base] | (hbits[pp][base + 4] << 16);
-          o16[4 * i + 2 * h + 1] = hbits[pp][base + 1] | (hbits[pp][base + 5] << 16);
-        }
-      uint4 *dst = reinterpret_cast<uint4 *>(xs + ((((gl * Mi + tok) * kParts + pp) * 4 + tt) * 16));
-#pragma unroll
-      for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o16[4 * c], o16[4 * c + 1], o16[4 * c + 2], o16[4 * c + 3]);
-    }
-    }  // valid
-    // sums over the 4 t-units of (group, token): lanes 4q..4q+3 hold them
+    // sums over the 4 quarters of (group, token): lanes 4q..4q+3 hold them
     sumB += __shfl_xor_sync(0xffffffffu, sumB, 1);
     sumB += __shfl_xor_sync(0xffffffffu, sumB, 2);
     sumX += __shfl_xor_sync(0xffffffffu, sumX, 1);
@@ -316,9 +370,12 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
   // ---------------- stream row tiles
   const int g = lane >> 2;
   const int t = lane & 3;
-  const int ra = warp * 16 + g;  // smem rows of this lane's A fragments
+  const int blk4 = warp & 3;     // 16-row block of the tile
+  const int half = warp >> 2;    // this warp takes groups 2*half, 2*half+1 of every stage
+  const int ra = blk4 * 16 + g;  // smem rows of this lane's A fragments
   const int rb = ra + 8;
   const bool split = p.kslices > 1;
+  const int kslices = p.kslices;
   const uint32_t stage_base = smem_u32(stages);
   const uint32_t xs_base = smem_u32(xs);
   const uint32_t ps_base = smem_u32(ps);
@@ -326,15 +383,16 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
   float acc[T8][4];
 #pragma unroll
   for (int o = 0; o < T8; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.0f;
+  int64_t tiles_done = 0;
   int64_t pend_row0 = -1;  // split-K arrival of the previous tile, read one tile later
   uint32_t pend_ticket = 0;
 
   auto finish_pending = [&]() {
     if (pend_row0 < 0) return;
     const uint32_t prev = __shfl_sync(0xffffffffu, pend_ticket, 0);
-    if (prev == (uint32_t)(p.kslices - 1)) {
+    if (prev == (uint32_t)(kslices - 1)) {
       __threadfence();
-      const int64_t blk = pend_row0 / 16 + warp;
+      const int64_t blk = pend_row0 / 16 + blk4;
 #pragma unroll
       for (int o = 0; o < T8; ++o)
 #pragma unroll
@@ -343,7 +401,7 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
           const int64_t tok = o * 8 + 2 * t + (c & 1);
           if (row < N && tok < M) {
             float v = 0.0f;
-            for (int sl = 0; sl < p.kslices; ++sl) v += __ldcg(p.ws + ((int64_t)sl * M + tok) * N + row);
+            for (int sl = 0; sl < kslices; ++sl) v += __ldcg(p.ws + ((int64_t)sl * M + tok) * N + row);
             if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[tok * N + row] = __float2bfloat16_rn(v);
             else static_cast<float *>(p.Y)[tok * N + row] = v;
           }
@@ -354,108 +412,165 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
     pend_row0 = -1;
   };
 
-  // per-lane constant parts of the shared-memory addresses
-  const uint32_t a_off0 = (uint32_t)(ra * 128), b_off0 = (uint32_t)(rb * 128);
-  const uint32_t sw_a = (uint32_t)(ra & 7), sw_b = (uint32_t)(rb & 7);
+  // per-lane constants: every shared-memory address below is one of these plus a
+  // per-stage or per-group increment (no index arithmetic in the hot loop)
+  const int Mi1 = Mi - 1;
+  const int g_first_i = (int)g_first;
+  const uint32_t box_off = (uint32_t)(half * kBox);
+  const uint32_t a_off0 = box_off + (uint32_t)(ra * 128) + (((uint32_t)t ^ (uint32_t)(ra & 7)) << 4);
+  const uint32_t a_off1 = box_off + (uint32_t)(ra * 128) + (((uint32_t)(4 + t) ^ (uint32_t)(ra & 7)) << 4);
+  const uint32_t b_off0 = box_off + (uint32_t)(rb * 128) + (((uint32_t)t ^ (uint32_t)(rb & 7)) << 4);
+  const uint32_t b_off1 = box_off + (uint32_t)(rb * 128) + (((uint32_t)(4 + t) ^ (uint32_t)(rb & 7)) << 4);
+  const uint32_t sa_off = (uint32_t)(kPBytes + ra * 16), sb_off = (uint32_t)(kPBytes + rb * 16);
+  const uint32_t gstride_x = (uint32_t)(Mi * kParts * 256);  // staged-fragment bytes per group
+  const uint32_t gstride_p = (uint32_t)(Mi * 8);             // (P, S) bytes per group
+  // Token columns beyond M read a real token's data (clamped): a B column only
+  // feeds its own D column, and those columns are never stored.
+  uint32_t bofs[T8], pofs0[T8], pofs1[T8];
+#pragma unroll
+  for (int o = 0; o < T8; ++o) {
+    const int tb = min(o * 8 + g, Mi1);
+    bofs[o] = xs_base + (uint32_t)(tb * kParts * 256 + t * 64);
+    pofs0[o] = ps_base + (uint32_t)(min(o * 8 + 2 * t, Mi1) * 8);
+    pofs1[o] = ps_base + (uint32_t)(min(o * 8 + 2 * t + 1, Mi1) * 8);
+  }
+  const uint32_t hdr_base = smem_u32(hdr);
 
-  for (int64_t it = 0;; ++it) {
-    const int s = (int)(it % kNst);
-    const uint32_t ph = (uint32_t)(it / kNst) & 1u;
+  int s = 0;
+  uint32_t ph = 0;
+  for (;;) {
     if (!mbar_wait(&full[s], ph, kErrTimeoutDequant)) break;
-    const int rt = hdr[4 * s + 0];
+    int rt, c;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(rt), "=r"(c) : "r"(hdr_base + (uint32_t)(s * 16)));
     if (rt < 0) break;
-    const int c = hdr[4 * s + 1];
     const uint32_t st = stage_base + (uint32_t)(s * kStage);
     const int64_t row0 = (int64_t)rt * kRows;
-    const int ngs = min(kSG, ng - c * kSG);  // groups in this stage (warp-uniform)
+    const int gl0 = c * kSG + 2 * half;  // first of this warp's two groups
+
+    if (gl0 < ng) {
+      const bool two = gl0 + 1 < ng;  // warp-uniform
+      // packed codes: one 16-byte chunk per row and group
+      const uint4 pa0 = lds128(st + a_off0), pb0 = lds128(st + b_off0);
+      const uint4 pa1 = lds128(st + a_off1), pb1 = lds128(st + b_off1);
+      // scales and zeros of both groups (adjacent fp16 in one 32-bit word)
+      uint32_t sa2, sb2, za2, zb2;
+      if constexpr (kScTma) {
+        const uint32_t off = (uint32_t)((g_first_i + gl0) & 7) * 2;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sa2) : "r"(st + sa_off + off));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb2) : "r"(st + sb_off + off));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(za2) : "r"(st + sa_off + kSBytes + off));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(zb2) : "r"(st + sb_off + kSBytes + off));
+      } else {
+        const int64_t kg = g_first + gl0;
+        const int64_t na = row0 + ra, nb = row0 + rb;
+        const uint32_t a0 = na < N ? __ldg(p.scales + na * Kg + kg) : 0u;
+        const uint32_t b0 = nb < N ? __ldg(p.scales + nb * Kg + kg) : 0u;
+        const uint32_t c0 = na < N ? __ldg(p.zeros + na * Kg + kg) : 0u;
+        const uint32_t d0 = nb < N ? __ldg(p.zeros + nb * Kg + kg) : 0u;
+        const uint32_t a1 = (two && na < N) ? __ldg(p.scales + na * Kg + kg + 1) : 0u;
+        const uint32_t b1 = (two && nb < N) ? __ldg(p.scales + nb * Kg + kg + 1) : 0u;
+        const uint32_t c1 = (two && na < N) ? __ldg(p.zeros + na * Kg + kg + 1) : 0u;
+        const uint32_t d1 = (two && nb < N) ? __ldg(p.zeros + nb * Kg + kg + 1) : 0u;
+        sa2 = a0 | (a1 << 16);
+        sb2 = b0 | (b1 << 16);
+        za2 = c0 | (c1 << 16);
+        zb2 = d0 | (d1 << 16);
+      }
+      const float2 sca = __half22float2(*reinterpret_cast<const __half2 *>(&sa2));
+      const float2 scb = __half22float2(*reinterpret_cast<const __half2 *>(&sb2));
+      const float2 zfa = __half22float2(*reinterpret_cast<const __half2 *>(&za2));
+      const float2 zfb = __half22float2(*reinterpret_cast<const __half2 *>(&zb2));
 
 #pragma unroll
-    for (int gl2 = 0; gl2 < kSG; ++gl2) {
-      if (gl2 >= ngs) break;
-      const int gl = c * kSG + gl2;  // group within the k-slice
-      const uint32_t chunk = (uint32_t)(gl2 * 4 + t);
-      const uint4 pa = lds128(st + a_off0 + ((chunk ^ sw_a) << 4));
-      const uint4 pb = lds128(st + b_off0 + ((chunk ^ sw_b) << 4));
-      uint32_t sa, sb, za, zb;
-      const int64_t kg = g_first + gl;
-      if constexpr (kScTma) {
-        const uint32_t off = (uint32_t)(kg & 7) * 2;
-        sa = lds_u16(st + kPBytes + ra * 16 + off);
-        sb = lds_u16(st + kPBytes + rb * 16 + off);
-        za = lds_u16(st + kPBytes + kSBytes + ra * 16 + off);
-        zb = lds_u16(st + kPBytes + kSBytes + rb * 16 + off);
-      } else {
-        const int64_t na = row0 + ra, nb = row0 + rb;
-        sa = na < N ? __ldg(p.scales + na * Kg + kg) : 0u;
-        sb = nb < N ? __ldg(p.scales + nb * Kg + kg) : 0u;
-        za = na < N ? __ldg(p.zeros + na * Kg + kg) : 0u;
-        zb = nb < N ? __ldg(p.zeros + nb * Kg + kg) : 0u;
-      }
-      // A fragments: one SHF + four LOP3 per 32-bit word (8 codes)
-      uint32_t A[8][4];
-      const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
-      const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
+      for (int j = 0; j < 2; ++j) {
+        if (j == 1 && !two) break;
+        const uint4 pa = j ? pa1 : pa0, pb = j ? pb1 : pb0;
+        // A fragments: one SHF + four LOP3 per 32-bit word (8 codes)
+        uint32_t A[8][4];
+        const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
+        const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t wa8 = wa[i] >> 8, wb8 = wb[i] >> 8;
-        A[2 * i][0] = lop3_and_or(wa[i], 0x000F000Fu, kMagic);
-        A[2 * i][2] = lop3_and_or(wa[i], 0x00F000F0u, kMagic);
-        A[2 * i][1] = lop3_and_or(wb[i], 0x000F000Fu, kMagic);
-        A[2 * i][3] = lop3_and_or(wb[i], 0x00F000F0u, kMagic);
-        A[2 * i + 1][0] = lop3_and_or(wa8, 0x000F000Fu, kMagic);
-        A[2 * i + 1][2] = lop3_and_or(wa8, 0x00F000F0u, kMagic);
-        A[2 * i + 1][1] = lop3_and_or(wb8, 0x000F000Fu, kMagic);
-        A[2 * i + 1][3] = lop3_and_or(wb8, 0x00F000F0u, kMagic);
-      }
-      const float sca = half_bits_to_float((uint16_t)sa);
-      const float scb = half_bits_to_float((uint16_t)sb);
-      const float zfa = half_bits_to_float((uint16_t)za);
-      const float zfb = half_bits_to_float((uint16_t)zb);
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t wa8 = wa[i] >> 8, wb8 = wb[i] >> 8;
+          A[2 * i][0] = lop3_and_or(wa[i], 0x000F000Fu, kMagic);
+          A[2 * i][2] = lop3_and_or(wa[i], 0x00F000F0u, kMagic);
+          A[2 * i][1] = lop3_and_or(wb[i], 0x000F000Fu, kMagic);
+          A[2 * i][3] = lop3_and_or(wb[i], 0x00F000F0u, kMagic);
+          A[2 * i + 1][0] = lop3_and_or(wa8, 0x000F000Fu, kMagic);
+          A[2 * i + 1][2] = lop3_and_or(wa8, 0x00F000F0u, kMagic);
+          A[2 * i + 1][1] = lop3_and_or(wb8, 0x000F000Fu, kMagic);
+          A[2 * i + 1][3] = lop3_and_or(wb8, 0x00F000F0u, kMagic);
+        }
+        const float sa = j ? sca.y : sca.x, sb = j ? scb.y : scb.x;
+        const float za = j ? zfa.y : zfa.x, zb = j ? zfb.y : zfb.x;
+        const uint32_t xg_off = (uint32_t)(gl0 + j) * gstride_x;
+        const uint32_t pg_off = (uint32_t)(gl0 + j) * gstride_p;
 #pragma unroll
-      for (int o = 0; o < T8; ++o) {
-        if (o * 8 >= Mi) break;  // octet without real tokens (warp-uniform)
-        const int tok = o * 8 + g;
-        float d0[4], d1[4];
+        for (int o = 0; o < T8; ++o) {
+          if (o * 8 >= Mi) break;  // octet without real tokens (warp-uniform)
+          float d0[4], d1[4];
 #pragma unroll
-        for (int pp = 0; pp < kParts; ++pp) {
-          uint32_t Bv[16];
-          if (tok < Mi) {
-            const uint32_t bad = xs_base + (uint32_t)(((((gl * Mi + tok) * kParts + pp) * 4 + t) * 16) * 4);
+          for (int pp = 0; pp < kParts; ++pp) {
+            uint32_t Bv[16];
+            const uint32_t bad = bofs[o] + xg_off + (uint32_t)(pp * 256);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const uint4 v = lds128(bad + 16 * q);
               Bv[4 * q] = v.x; Bv[4 * q + 1] = v.y; Bv[4 * q + 2] = v.z; Bv[4 * q + 3] = v.w;
             }
-          } else {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) Bv[q] = 0u;
+            for (int b = 0; b < 8; ++b) {
+              if (b & 1) mma_f16(d1, A[b], Bv[2 * b], Bv[2 * b + 1], pp == 0 && b == 1);
+              else mma_f16(d0, A[b], Bv[2 * b], Bv[2 * b + 1], pp == 0 && b == 0);
+            }
           }
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            if (b & 1) mma_f16(d1, A[b], Bv[2 * b], Bv[2 * b + 1], pp == 0 && b == 1);
-            else mma_f16(d0, A[b], Bv[2 * b], Bv[2 * b + 1], pp == 0 && b == 0);
-          }
+          // promotion: y' += scale * (D - P - z S) for tokens 2t, 2t+1 of this octet
+          const float2 q0 = lds_f2(pofs0[o] + pg_off);
+          const float2 q1 = lds_f2(pofs1[o] + pg_off);
+          acc[o][0] = fmaf(-sa, fmaf(za, q0.y, q0.x), fmaf(sa, d0[0] + d1[0], acc[o][0]));
+          acc[o][1] = fmaf(-sa, fmaf(za, q1.y, q1.x), fmaf(sa, d0[1] + d1[1], acc[o][1]));
+          acc[o][2] = fmaf(-sb, fmaf(zb, q0.y, q0.x), fmaf(sb, d0[2] + d1[2], acc[o][2]));
+          acc[o][3] = fmaf(-sb, fmaf(zb, q1.y, q1.x), fmaf(sb, d0[3] + d1[3], acc[o][3]));
         }
-        // promotion: y' += scale * (D - P - z S) for tokens 2t, 2t+1 of this octet
-        const int t0 = o * 8 + 2 * t;
-        float2 q0 = make_float2(0.f, 0.f), q1 = make_float2(0.f, 0.f);
-        if (t0 < Mi) q0 = lds_f2(ps_base + (uint32_t)((gl * Mi + t0) * 8));
-        if (t0 + 1 < Mi) q1 = lds_f2(ps_base + (uint32_t)((gl * Mi + t0 + 1) * 8));
-        acc[o][0] = fmaf(-sca, fmaf(zfa, q0.y, q0.x), fmaf(sca, d0[0] + d1[0], acc[o][0]));
-        acc[o][1] = fmaf(-sca, fmaf(zfa, q1.y, q1.x), fmaf(sca, d0[1] + d1[1], acc[o][1]));
-        acc[o][2] = fmaf(-scb, fmaf(zfb, q0.y, q0.x), fmaf(scb, d0[2] + d1[2], acc[o][2]));
-        acc[o][3] = fmaf(-scb, fmaf(zfb, q1.y, q1.x), fmaf(scb, d0[3] + d1[3], acc[o][3]));
       }
     }
     // release the stage (all lanes' shared-memory reads are consumed above)
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == kNst) {
+      s = 0;
+      ph ^= 1u;
+    }
     if (c != nst_task - 1) continue;
 
-    // ---------------- tile done: outputs of this warp's 16 rows (scaled back by 2^-e)
-    finish_pending();
-    const int64_t blk = row0 / 16 + warp;
-    if (blk < RB16) {
+    // ---------------- tile done: the two warps of a row block combine their groups
+    // through shared memory, handing off with (bounded) mbarrier waits
+    {
+      const uint32_t pph = (uint32_t)(tiles_done & 1);
+      if (half == 1) {
+        if (!mbar_wait(&pair_empty[blk4], pph ^ 1u, kErrTimeoutDequant)) break;
+#pragma unroll
+        for (int o = 0; o < T8; ++o)
+          *reinterpret_cast<float4 *>(pairbuf + ((blk4 * 32 + lane) * T8 + o) * 4) =
+              make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pair_full[blk4]);
+      } else {
+        if (!mbar_wait(&pair_full[blk4], pph, kErrTimeoutDequant)) break;
+#pragma unroll
+        for (int o = 0; o < T8; ++o) {
+          const float4 v = *reinterpret_cast<const float4 *>(pairbuf + ((blk4 * 32 + lane) * T8 + o) * 4);
+          acc[o][0] += v.x; acc[o][1] += v.y; acc[o][2] += v.z; acc[o][3] += v.w;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pair_empty[blk4]);
+      }
+      ++tiles_done;
+    }
+    // outputs of this row block (scaled back by 2^-e), written by the half-0 warp
+    const int64_t blk = row0 / 16 + blk4;
+    if (half == 0) finish_pending();
+    if (half == 0 && blk < RB16) {
       const int64_t rowa = row0 + ra, rowb = row0 + rb;
 #pragma unroll
       for (int o = 0; o < T8; ++o)
@@ -483,27 +598,44 @@ __global__ void __launch_bounds__(160) gemv_kernel(const __grid_constant__ CUten
 #pragma unroll
     for (int o = 0; o < T8; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.0f;
   }
-  finish_pending();
+  if (half == 0) finish_pending();
 }
 
-template <int T8, bool kAwq, bool kScTma>
+template <int T8, bool kBf16, bool kAwq, bool kScTma>
 cudaError_t launch_t(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUtensorMap &tmZ, const GemvParams &p,
                      cudaStream_t stream) {
-  auto kern = gemv_kernel<T8, kAwq, kScTma>;
-  const int smem = smem_bytes_for(p.xs_bytes);
+  auto kern = gemv_kernel<T8, kBf16, kAwq, kScTma>;
+  const int smem = smem_bytes_for(p.xs_bytes, T8);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)p.grid_x, (unsigned)p.kslices);
-  kern<<<grid, 160, smem, stream>>>(tmP, tmS, tmZ, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid_x, (unsigned)p.kslices);
+  cfg.blockDim = dim3(kComputeThreads + 32);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmP, tmS, tmZ, p);
+}
+
+template <int T8, bool kBf16>
+cudaError_t launch_x(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUtensorMap &tmZ, const GemvParams &p,
+                     bool sc_tma, cudaStream_t stream) {
+  if (p.awq_s)
+    return sc_tma ? launch_t<T8, kBf16, true, true>(tmP, tmS, tmZ, p, stream)
+                  : launch_t<T8, kBf16, true, false>(tmP, tmS, tmZ, p, stream);
+  return sc_tma ? launch_t<T8, kBf16, false, true>(tmP, tmS, tmZ, p, stream)
+                : launch_t<T8, kBf16, false, false>(tmP, tmS, tmZ, p, stream);
 }
 
 template <int T8>
 cudaError_t launch_s(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUtensorMap &tmZ, const GemvParams &p,
-                     bool sc_tma, cudaStream_t stream) {
-  if (p.awq_s)
-    return sc_tma ? launch_t<T8, true, true>(tmP, tmS, tmZ, p, stream) : launch_t<T8, true, false>(tmP, tmS, tmZ, p, stream);
-  return sc_tma ? launch_t<T8, false, true>(tmP, tmS, tmZ, p, stream) : launch_t<T8, false, false>(tmP, tmS, tmZ, p, stream);
+                     bool x_bf16, bool sc_tma, cudaStream_t stream) {
+  return x_bf16 ? launch_x<T8, true>(tmP, tmS, tmZ, p, sc_tma, stream)
+                : launch_x<T8, false>(tmP, tmS, tmZ, p, sc_tma, stream);
 }
 
 }  // namespace gemv_impl
@@ -512,16 +644,16 @@ bool gemv_supports(int64_t M, bool awq) { return M <= 64 && !(awq && M > 32); }
 
 // Shared-memory bytes of the staged activations for a k-slice of kr groups.
 int gemv_xs_bytes(int kr, int64_t M, bool awq) { return gemv_impl::xs_bytes_for(kr, (int)M, awq); }
-int gemv_smem_bytes(int xs_bytes) { return gemv_impl::smem_bytes_for(xs_bytes); }
+int gemv_smem_bytes(int xs_bytes, int t8) { return gemv_impl::smem_bytes_for(xs_bytes, t8); }
 
 cudaError_t launch_gemv(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUtensorMap &tmZ, const GemvParams &p,
-                        int t8, bool sc_tma, cudaStream_t stream) {
+                        int t8, bool x_bf16, bool sc_tma, cudaStream_t stream) {
   using namespace gemv_impl;
   switch (t8) {
-    case 1: return launch_s<1>(tmP, tmS, tmZ, p, sc_tma, stream);
-    case 2: return launch_s<2>(tmP, tmS, tmZ, p, sc_tma, stream);
-    case 4: return launch_s<4>(tmP, tmS, tmZ, p, sc_tma, stream);
-    default: return launch_s<8>(tmP, tmS, tmZ, p, sc_tma, stream);
+    case 1: return launch_s<1>(tmP, tmS, tmZ, p, x_bf16, sc_tma, stream);
+    case 2: return launch_s<2>(tmP, tmS, tmZ, p, x_bf16, sc_tma, stream);
+    case 4: return launch_s<4>(tmP, tmS, tmZ, p, x_bf16, sc_tma, stream);
+    default: return launch_s<8>(tmP, tmS, tmZ, p, x_bf16, sc_tma, stream);
   }
 }
 

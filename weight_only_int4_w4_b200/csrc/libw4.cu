@@ -120,11 +120,12 @@ int forced_path() {
   return 0;
 }
 
-// CTAs of the decode kernel resident per SM (shared memory and a 4-CTA register budget).
-int gemv_ctas_per_sm(int xs_bytes) {
-  const int per = w4::gemv_smem_bytes(xs_bytes) + 1024;
+// CTAs of the decode kernel resident per SM (shared memory, and at most 3 CTAs of
+// 288 threads for the register file).
+int gemv_ctas_per_sm(int xs_bytes, int t8) {
+  const int per = w4::gemv_smem_bytes(xs_bytes, t8) + 1024;
   int n = (228 * 1024) / per;
-  return n < 1 ? 1 : (n > 4 ? 4 : n);
+  return n < 1 ? 1 : (n > 3 ? 3 : n);
 }
 
 GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
@@ -135,20 +136,38 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   const int64_t RT = cdiv(N, 64);
   const int64_t RB16 = cdiv(N, 16);
   p.sc_tma = (Kg % 8) == 0;
-  // longest even k-slice whose activations fit the staging budget
-  int64_t kr_max = std::min<int64_t>(Kg + (Kg & 1), 4096);
-  while (kr_max > 2 && w4::gemv_xs_bytes((int)kr_max, M, awq) > kGemvXsMax) kr_max -= 2;
-  // shortest k-slices that still leave ~1.5 tiles per resident CTA (dynamic scheduling balances the rest)
+  // k-slices are whole pipeline stages of 4 groups.  Longest one whose activations
+  // fit the staging budget:
+  int64_t kr_max = std::min<int64_t>(cdiv(Kg, 4) * 4, 4096);
+  while (kr_max > 4 && w4::gemv_xs_bytes((int)kr_max, M, awq) > kGemvXsMax) kr_max -= 4;
+  // Slice length from a cost model fitted to B200 measurements of this kernel: a CTA
+  // streams at ~20 GB/s (its TMA ring depth over the loaded memory latency), the
+  // whole GPU at ~6.5 TB/s, a launch costs ~4 us, and every extra k-slice adds
+  // activation staging plus split-K partials (~3 us, then ~1.2 us per slice).
   int64_t kr = kr_max;
-  for (;;) {
-    const int64_t ks = cdiv(Kg, kr);
-    const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(w4::gemv_xs_bytes((int)kr, M, awq));
-    if (RT * ks * 2 >= slots * 3 || kr <= 2) break;
-    kr -= 2;
+  {
+    const double bytes = (double)N * (double)K * (0.5 + 4.0 / w4::kGroup);
+    double best = 1e300;
+    int64_t prev = -1;
+    for (int64_t ks = cdiv(Kg, kr_max); ks <= 8; ++ks) {
+      const int64_t cand = cdiv(cdiv(Kg, ks), 4) * 4;  // balanced slices, whole stages
+      if (cand == prev || cand > kr_max) continue;
+      prev = cand;
+      const int64_t nks = cdiv(Kg, cand);
+      const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(w4::gemv_xs_bytes((int)cand, M, awq), p.t8);
+      const double ctas = (double)std::min<int64_t>(RT * nks, slots);
+      const double stream_us = std::max(bytes / (ctas * 20e9), bytes / 6.5e12) * 1e6;
+      const double est = 4.0 + stream_us + (nks > 1 ? 3.0 + 1.2 * (double)nks : 0.0);
+      if (est < best) {
+        best = est;
+        kr = cand;
+      }
+      if (cand <= 4) break;
+    }
   }
   if (const char *e = getenv("W4_GEMV_KR")) {  // tuning override
     const int64_t v = atoi(e);
-    if (v >= 2 && v % 2 == 0 && v <= kr_max) kr = v;
+    if (v >= 4 && v % 4 == 0 && v <= kr_max) kr = v;
   }
   int64_t ks = cdiv(Kg, kr);
   if ((ks > 1 && RB16 > kMaxSplitCounters) || ks > kMaxKslices) {  // counters: fall back to the longest slices
@@ -158,7 +177,7 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   p.kr = (int)kr;
   p.kslices = (int)ks;
   p.xs_bytes = w4::gemv_xs_bytes(p.kr, M, awq);
-  const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(p.xs_bytes);
+  const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(p.xs_bytes, p.t8);
   p.grid_x = (int)std::min<int64_t>(RT, std::max<int64_t>(1, slots / ks));
   if (const char *e = getenv("W4_GEMV_GX")) {  // tuning override
     const int v = atoi(e);
@@ -356,8 +375,7 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
     p.ws = partials; p.counters = counters;
     p.sched = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kSplitCounterBytes);
     p.kslices = plan.kslices; p.kr = plan.kr; p.grid_x = plan.grid_x; p.xs_bytes = plan.xs_bytes;
-    p.x_bf16 = xbf16;
-    e = w4::launch_gemv(tmP, tmS, tmZ, p, plan.t8, plan.sc_tma, s);
+    e = w4::launch_gemv(tmP, tmS, tmZ, p, plan.t8, xbf16, plan.sc_tma, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
     return W4_OK;
   }
