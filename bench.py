@@ -165,20 +165,33 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(v, world):
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+def _all_reduce(v, op):
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(v, world):
+    """Slowest rank's time: the job is done when every rank is done."""
+    return v if world == 1 else _all_reduce(v, torch.distributed.ReduceOp.MAX)
 
 
 def sum_over_ranks(v, world):
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t)
-    return float(t.item())
+    """Total work of all ranks (weak scaling: each rank runs its own copy of the step)."""
+    return v if world == 1 else _all_reduce(v, torch.distributed.ReduceOp.SUM)
+
+
+def job_throughput(bytes_per_rank, ms_per_rank, world):
+    """Whole-job GB/s: all ranks' bytes over the slowest rank's device time."""
+    ms = max_over_ranks(ms_per_rank, world)
+    return sum_over_ranks(bytes_per_rank, world) / (ms * 1e-3) / 1e9, ms
+
+
+def decode_config(world):
+    return {"workload": "decode_8b: Llama-3-8B qkv/o_proj/gate_up/down, M=1, bf16 X ~N(0,1), "
+                        "W ~N(0,0.02) with 0.1% N(0,0.4) outliers, uint4 G=128",
+            "global_batch": world, "seq_len": 1, "parallelism": f"replicas{world}"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -236,7 +249,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32xu4->f64", "data": "synthetic",
-        "config": {"workload": "decode_8b (oracle sample)", "global_batch": 1, "seq_len": 1, "parallelism": "none"},
+        "config": decode_config(world),
         "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"{rows} output rows of each of the 4 Llama-3-8B layers per step (dequant + fp64 matmul, M=1)"},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -430,8 +443,7 @@ def main():
     step_bytes = sum(gemm_bytes(1, layers[n]["N"], layers[n]["K"]) for n in LAYERS)
 
     ms, dom, clocks = decode_leg(w4, layers, args.steps, args.warmup, world)
-    ms = max_over_ranks(ms, world)
-    value = sum_over_ranks(step_bytes * args.steps, world) / (ms * 1e-3) / 1e9
+    value, ms = job_throughput(step_bytes * args.steps, ms, world)
 
     K, N = synthetic.SHAPES_8B[DOMINANT]
     dom_bytes = gemm_bytes(1, N, K)
@@ -439,9 +451,7 @@ def main():
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
 
     e2e_ms, h2d, d2h = e2e_leg(w4, layers, max(20, args.steps // 4), args.warmup, world)
-    e2e_ms = max_over_ranks(e2e_ms, world)
-    e2e_steps = max(20, args.steps // 4)
-    e2e_value = sum_over_ranks(step_bytes * e2e_steps, world) / (e2e_ms * 1e-3) / 1e9
+    e2e_value, e2e_ms = job_throughput(step_bytes * max(20, args.steps // 4), e2e_ms, world)
     del layers
     torch.cuda.empty_cache()
 
@@ -469,9 +479,7 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16xu4->f32", "data": "synthetic",
-            "config": {"workload": "decode_8b: Llama-3-8B qkv/o_proj/gate_up/down, M=1, bf16 X ~N(0,1), "
-                                   "W ~N(0,0.02) with 0.1% N(0,0.4) outliers, uint4 G=128",
-                       "global_batch": world, "seq_len": 1, "parallelism": f"replicas{world}",
+            "config": {**decode_config(world),
                        "l2": f"{N_COPIES} rotating weight copies ({N_COPIES * step_bytes / 1e6:.0f} MB > 4x L2): "
                              "each step reads weights not touched for 4 steps",
                        "graph": "timed steps captured in one CUDA graph"},
