@@ -139,6 +139,35 @@ w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype,
                           w4_stream_t stream);
 
 /*
+ * Decode GEMM with library-owned scratch: the same computation, kernel and
+ * result as w4a16_gemm for decode shapes, with no workspace argument.  The
+ * source pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory where they run the layer (an engine plugin
+ * with no allocator of its own, a loop that must not take cudaMalloc).
+ *   Arguments as for w4a16_gemm.  M <= 64 (M <= 32 with awq_s), else
+ *   W4_ERR_UNSUPPORTED.
+ *   Scratch: a fixed array of w4a16_gemm_decode_static_capacity() bytes
+ *   (8 MiB) per device, part of the library's own module.  A shape whose plan
+ *   needs more returns W4_ERR_UNSUPPORTED with the sizes in w4_last_error()
+ *   and launches nothing; use w4a16_gemm with a workspace for it.
+ *   The first call on a device looks up the scratch address on that device
+ *   (the device must be current); make it before any stream capture.
+ *   The scratch starts zero-filled and every completed call leaves its
+ *   counters at zero.  Calls on one device share it: calls that overlap in
+ *   time (other streams or threads) race on it and give wrong results.
+ */
+w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M,
+                                   int64_t N, int64_t K, int group,
+                                   const uint8_t *packed,
+                                   const uint16_t *scales,
+                                   const uint16_t *zeros, const float *awq_s,
+                                   void *Y, w4_dtype y_dtype,
+                                   w4_stream_t stream);
+
+/* Bytes of the static scratch behind w4a16_gemm_decode_static. */
+size_t w4a16_gemm_decode_static_capacity(void);
+
+/*
  * Device-side error word: kernels whose bounded waits run out set it instead
  * of hanging.  Copies its value to *flag (0 = no error) and clears it; this
  * call synchronizes the current device.

@@ -453,3 +453,85 @@ w4_status w4_device_error(int *flag) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode GEMM with library-owned scratch.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// layer: a C plugin inside an engine that has already handed the whole device
+// to its own pools (weights, KV cache) and owns no allocator of its own, or a
+// latency-bound decode loop that must not take cudaMalloc/cudaFree, which can
+// synchronize the whole device.  w4a16_gemm_decode_static serves them with a
+// fixed scratch that lives in this module's own device memory: a file-scope
+// array loaded with the module, so no call here allocates anything.
+//
+// What must start at zero: the split-K and scheduler counters at the front of
+// the scratch.  Device globals without an initializer are zero-filled when the
+// module is loaded, and every completed call leaves the counters at zero again.
+// The fp32 partials behind them need no initial value.  A call whose kernel
+// reported a device error (w4_device_error) may leave counters non-zero; the
+// scratch has no reset, so the process should stop using this entry point then.
+//
+// All calls on one device share the one scratch: two calls that overlap in time
+// (different streams or threads) race on it and give wrong results.  Calls on
+// one stream, one after another, are safe.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;  // 128 KiB counters + ~7.9 MiB partials
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+void *g_static_scratch_ptr[kMaxDevices];
+
+// Address of the scratch on the current device.  The first call on a device
+// looks it up (which loads the module there if it is not loaded yet).
+cudaError_t static_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4a16_gemm_decode_static_capacity(void) { return kStaticScratchBytes; }
+
+w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
+                                   const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros,
+                                   const float *awq_s, void *Y, w4_dtype y_dtype, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(M, N, K, group);
+  if (st != W4_OK) return st;
+  const bool awq = awq_s != nullptr;
+  if (!w4::gemv_supports(M, awq))
+    return fail(W4_ERR_UNSUPPORTED, "the static-scratch decode GEMM serves M <= 64 (M <= 32 with AWQ), got M=%lld%s",
+                (long long)M, awq ? " with AWQ" : "");
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const size_t need = plan_gemm(M, N, K, awq, sm).ws_bytes;
+  if (need > kStaticScratchBytes)
+    return fail(W4_ERR_UNSUPPORTED,
+                "M=%lld N=%lld K=%lld needs %zu bytes of scratch; the static scratch holds %zu "
+                "(call w4a16_gemm with a caller-owned workspace instead)",
+                (long long)M, (long long)N, (long long)K, need, kStaticScratchBytes);
+  void *scratch = nullptr;
+  e = static_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
+  return w4a16_gemm(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, scratch,
+                    kStaticScratchBytes, stream);
+}
+
+}  // extern "C"

@@ -6,7 +6,8 @@ runs in the library's CUDA kernels.  There is no fallback: if ``libw4.so`` is
 not built, importing this module raises.
 
 Names follow the C ABI: ``w4_quantize``, ``w4_pack``, ``w4a16_gemm``,
-``w4a16_gemm_workspace_size``, ``w4a16_gemm_host``, ``w4_device_error``.
+``w4a16_gemm_workspace_size``, ``w4a16_gemm_host``, ``w4a16_gemm_decode_static``,
+``w4_device_error``.
 """
 from __future__ import annotations
 
@@ -28,13 +29,17 @@ _lib.w4a16_gemm.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P
                             _P, _SZ, _P]
 _lib.w4a16_gemm_host.argtypes = [_P, _P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, _P,
                                  ctypes.c_int, _P, _SZ, _P]
+_lib.w4a16_gemm_decode_static.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P,
+                                          ctypes.c_int, _P]
+_lib.w4a16_gemm_decode_static_capacity.argtypes = []
+_lib.w4a16_gemm_decode_static_capacity.restype = _SZ
 _lib.w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
 _lib.w4a16_gemm_workspace_size.restype = _SZ
 _lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
 _lib.w4_status_string.argtypes = [ctypes.c_int]
 _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
-for _f in ("w4_quantize", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4_device_error"):
+for _f in ("w4_quantize", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -150,6 +155,26 @@ def w4a16_gemm_host(X_host: torch.Tensor, X_dev: torch.Tensor, packed, scales, z
                                 _DT[Y_host.dtype], _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
            "w4a16_gemm_host")
     return Y_host
+
+
+def w4a16_gemm_decode_static(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                             awq_s: torch.Tensor | None = None, out_dtype=torch.float32,
+                             out: torch.Tensor | None = None, group: int = GROUP, stream=None) -> torch.Tensor:
+    """Decode-shape Y = X . W^T using the library's own fixed scratch (no workspace
+    argument).  Calls on one device must not overlap in time."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.dtype in (torch.float16, torch.bfloat16)
+    M, K = X.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _check(_lib.w4a16_gemm_decode_static(_ptr(X), _DT[X.dtype], M, N, K, group, _ptr(packed), _ptr(scales),
+                                         _ptr(zeros), _ptr(awq_s), _ptr(out), _DT[out.dtype], _stream(stream)),
+           "w4a16_gemm_decode_static")
+    return out
+
+
+def w4a16_gemm_decode_static_capacity() -> int:
+    return int(_lib.w4a16_gemm_decode_static_capacity())
 
 
 def w4_device_error() -> int:
