@@ -8,8 +8,9 @@ bf16 activations with packed uint4 weights resident in HBM.  Throughput is
 algorithmic bytes (packed codes + fp16 scale/zero + X + fp32 Y) per second.
 
 Also reported on the same JSON line:
-  * roofline of the dominant kernel (gate_up), timed by CUDA events recorded
-    inside the same CUDA graph as the timed steps;
+  * roofline of the dominant kernel (gate_up): its average launch duration,
+    from CUDA events around a CUDA graph of back-to-back gate_up launches over
+    the same rotating weight copies;
   * e2e: the same metric through the C ABI's host-buffer entry point
     (pinned X in, fp32 Y out, copies inside the timed region);
   * quantize: the quantize+pack kernel on the same four layers (fp32 W in);
@@ -278,49 +279,66 @@ def build_decode_state(w4, dev):
     return layers
 
 
-def decode_leg(w4, layers, steps, warmup, world):
-    dev = torch.device("cuda")
-    stream = torch.cuda.Stream()
-    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-          for _ in range(steps)]
-
-    def step(i, record=False):
-        for name in LAYERS:
-            L = layers[name]
-            packed, scales, zeros = L["copies"][i % N_COPIES]
-            if record and name == DOMINANT:
-                ev[i][0].record()
-            w4.w4a16_gemm(L["X"], packed, scales, zeros, out=L["Y"], ws=L["ws"])
-            if record and name == DOMINANT:
-                ev[i][1].record()
-
+def _graph_of(fn, steps, warmup, stream):
     with torch.cuda.stream(stream):
         for i in range(warmup):
-            step(i)
+            fn(i)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for i in range(steps):
-            step(i, record=True)
-    # warm replay of the graph itself
-    with torch.cuda.stream(stream):
+            fn(i)
+    with torch.cuda.stream(stream):  # warm replay of the graph itself
         g.replay()
     torch.cuda.synchronize()
+    return g
 
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+def _replay_timed(g, stream):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def decode_leg(w4, layers, steps, warmup, world):
+    """The timed steps: `steps` decode steps (4 fused calls each) in one CUDA graph."""
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        for name in LAYERS:
+            L = layers[name]
+            packed, scales, zeros = L["copies"][i % N_COPIES]
+            w4.w4a16_gemm(L["X"], packed, scales, zeros, out=L["Y"], ws=L["ws"])
+
+    g = _graph_of(step, steps, warmup, stream)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        with torch.cuda.stream(stream):
-            t_start.record(stream)
-            g.replay()
-            t_end.record(stream)
-        torch.cuda.synchronize()
+        ms = _replay_timed(g, stream)
     barrier(world)
-    ms = t_start.elapsed_time(t_end)
-    dom = [a.elapsed_time(b) for a, b in ev]
     del g
-    return ms, dom, clk.summary()
+    return ms, clk.summary()
+
+
+def dominant_leg(w4, layers, launches, warmup):
+    """Average launch duration of the dominant kernel (gate_up, M=1): `launches`
+    launches over the rotating weight copies in one CUDA graph, timed with events
+    on the stream they run on."""
+    stream = torch.cuda.Stream()
+    L = layers[DOMINANT]
+
+    def one(i):
+        packed, scales, zeros = L["copies"][i % N_COPIES]
+        w4.w4a16_gemm(L["X"], packed, scales, zeros, out=L["Y"], ws=L["ws"])
+
+    g = _graph_of(one, launches, warmup, stream)
+    ms = _replay_timed(g, stream)
+    del g
+    return ms / launches
 
 
 def e2e_leg(w4, layers, steps, warmup, world):
@@ -442,12 +460,12 @@ def main():
     layers = build_decode_state(w4, torch.device("cuda"))
     step_bytes = sum(gemm_bytes(1, layers[n]["N"], layers[n]["K"]) for n in LAYERS)
 
-    ms, dom, clocks = decode_leg(w4, layers, args.steps, args.warmup, world)
+    ms, clocks = decode_leg(w4, layers, args.steps, args.warmup, world)
     value, ms = job_throughput(step_bytes * args.steps, ms, world)
 
     K, N = synthetic.SHAPES_8B[DOMINANT]
     dom_bytes = gemm_bytes(1, N, K)
-    dom_ms = sum(dom) / len(dom)
+    dom_ms = dominant_leg(w4, layers, max(20, args.steps), args.warmup)
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
 
     e2e_ms, h2d, d2h = e2e_leg(w4, layers, max(20, args.steps // 4), args.warmup, world)

@@ -601,6 +601,16 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   if (half == 0) finish_pending();
 }
 
+// Programmatic dependent launch is on by default; W4_PDL=0 launches without it
+// (for tools that replay kernels one at a time).
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char *e = getenv("W4_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int T8, bool kBf16, bool kAwq, bool kScTma>
 cudaError_t launch_t(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUtensorMap &tmZ, const GemvParams &p,
                      cudaStream_t stream) {
@@ -617,7 +627,7 @@ cudaError_t launch_t(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUten
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, tmP, tmS, tmZ, p);
 }
 
