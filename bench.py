@@ -439,6 +439,33 @@ def prefill_leg(w4, M=8192, steps=3):
     return res, total_flop / (total_ms * 1e-3) / 1e12, total_ms
 
 
+def stack70b_leg(w4, replays=3):
+    """Whole-model 70B decode step: quantize the 80-layer stack + lm_head on the device, then
+    one step through all 321 linear layers at M=1 and at M=16, each captured in a CUDA graph."""
+    from weight_only_int4_w4_b200 import stack70b
+    layers, q_ms, q_bytes = stack70b.build(w4)
+    out = {"workload": "Llama-3-70B stack: 80 x (qkv, o_proj, gate_up, down) + lm_head, "
+                       "69.50 G params, 36.92 GB packed, W ~N(0,0.015), bf16 X ~N(0,1)",
+           "quantize": {"value": round(q_bytes / (q_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                        "ms_total": round(q_ms, 2), "bytes": q_bytes}}
+    hbm_peak = peaks()[0]
+    for M in (1, 16):
+        X, Y, ws = stack70b.step_buffers(w4, layers, M)
+        stream = torch.cuda.Stream()
+        g = _graph_of(lambda i: stack70b.run_step(w4, layers, X, Y, ws), 1, 1, stream)
+        ms = min(_replay_timed(g, stream) for _ in range(replays))
+        del g
+        nbytes = stack70b.step_bytes(layers, M)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[f"decode_m{M}"] = {"us_per_step": round(ms * 1e3, 1), "GB/s": round(gbs, 1),
+                                "bytes_per_step": nbytes, "roofline_frac": round(gbs / hbm_peak, 4),
+                                "launches": len(layers)}
+        del X, Y, ws
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,6 +509,7 @@ def main():
                               "roofline": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm_peak,
                                            "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4)}}
         pf, pf_all, pf_ms = prefill_leg(w4)
+        extras["stack70b"] = stack70b_leg(w4)
         extras["prefill"] = {"value": round(pf_all, 1), "unit": "TFLOP/s", "ms_per_step": round(pf_ms, 3),
                              "workload": "Llama-3-70B qkv/o_proj/gate_up/down, M=8192, bf16 X",
                              "per_layer_tflops": pf,
