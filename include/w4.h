@@ -66,7 +66,7 @@ extern "C" {
 typedef enum {
   W4_OK = 0,
   W4_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer, short workspace */
-  W4_ERR_UNSUPPORTED = 2, /* valid but not served: group != 128, dtype combination */
+  W4_ERR_UNSUPPORTED = 2, /* valid but not served: group not 32/64/128, dtype combination */
   W4_ERR_CUDA = 3         /* a CUDA call or kernel launch failed */
 } w4_status;
 
@@ -80,8 +80,8 @@ typedef struct CUstream_st *w4_stream_t;
  *   W        device [N][K], dtype w_dtype (F32, F16 or BF16)
  *   awq_s    device [K] fp32 or NULL (no AWQ)
  *   N, K     N >= 1, K >= 1, K % group == 0
- *   group    must be 128
- *   packed   device [N][K/2] out; scales, zeros device [N][K/128] out
+ *   group    128; 32 and 64 are also served (scales, zeros [N][K/group])
+ *   packed   device [N][K/2] out; scales, zeros device [N][K/group] out
  *   codes    device [N][K] out, or NULL (unpacked codes, a test aid)
  * Outputs match the rule above bit for bit.
  */
@@ -89,6 +89,21 @@ w4_status w4_quantize(const void *W, w4_dtype w_dtype, const float *awq_s,
                       int64_t N, int64_t K, int group, uint8_t *packed,
                       uint16_t *scales, uint16_t *zeros, uint8_t *codes,
                       w4_stream_t stream);
+
+/*
+ * Symmetric variant of w4_quantize: INT4 as the symmetric value set
+ * {-7, ..., 7} (mhpq.cn practitioner's article, section 2.1).  Per group:
+ *   amax = max |w'|;  scale = fp16(amax / 7), 1.0 if that is 0;
+ *   q = clamp(rint(w' / scale), -7, 7);  stored code = q + 8 (1..15), zero = 8.
+ * The outputs have the same layout as w4_quantize's (every zero is 8.0), so
+ * w4a16_gemm consumes them unchanged: (code - 8) * scale = q * scale.
+ * Arguments and errors as for w4_quantize.
+ */
+w4_status w4_quantize_symmetric(const void *W, w4_dtype w_dtype,
+                                const float *awq_s, int64_t N, int64_t K,
+                                int group, uint8_t *packed, uint16_t *scales,
+                                uint16_t *zeros, uint8_t *codes,
+                                w4_stream_t stream);
 
 /*
  * Pack one-code-per-byte codes [N][K] (device) into packed [N][K/2]
@@ -102,7 +117,8 @@ w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed,
  * Fused dequantize-matmul Y = X . W^T (a6..a7).
  *   X         device [M][K], x_dtype F16 or BF16
  *   M, N, K   >= 1; K % group == 0
- *   group     must be 128
+ *   group     the group given to w4_quantize: 128, or 32 / 64 (then K must be
+ *             a multiple of 64, and the tensor-core kernel serves every M)
  *   packed, scales, zeros   as produced by w4_quantize
  *   awq_s     device [K] fp32, the SAME vector given to w4_quantize, or NULL
  *   Y         device [M][N], y_dtype F32 or BF16 (overwritten)

@@ -38,6 +38,7 @@ def _load():
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         _lib.w4o_quantize.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
+        _lib.w4o_quantize_sym.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
         _lib.w4o_pack.argtypes = [P, I64, I64, P]
         _lib.w4o_unpack.argtypes = [P, I64, I64, P]
         _lib.w4o_dequant.argtypes = [P, P, P, P, I64, I64, ctypes.c_int, P]
@@ -68,6 +69,20 @@ def quantize(W, awq_s=None, group: int = 128):
     rc = _load().w4o_quantize(_ptr(W), _ptr(s), N, K, group, _ptr(codes), _ptr(scales), _ptr(zeros))
     if rc != 0:
         raise ValueError("w4o_quantize rejected its arguments")
+    return codes, scales.view(np.float16), zeros.view(np.float16)
+
+
+def quantize_symmetric(W, awq_s=None, group: int = 128):
+    """Symmetric variant: codes q + 8 with q in [-7, 7], scale = fp16(max|w'| / 7), zeros all 8."""
+    W = _c(W, np.float32)
+    s = _c(awq_s, np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K), np.uint8)
+    scales = np.empty((N, K // group), np.uint16)
+    zeros = np.empty((N, K // group), np.uint16)
+    rc = _load().w4o_quantize_sym(_ptr(W), _ptr(s), N, K, group, _ptr(codes), _ptr(scales), _ptr(zeros))
+    if rc != 0:
+        raise ValueError("w4o_quantize_sym rejected its arguments")
     return codes, scales.view(np.float16), zeros.view(np.float16)
 
 

@@ -20,6 +20,9 @@
  *                (INT4 = 0.5 B), weight-only quantization (dequantize back to
  *                FP16 then matmul), and the AWQ equation W^ = quant(W/s) * s.
  *
+ *   [Notes 2.1]  mhpq.cn practitioner's article, section 2.1: INT4 weights take
+ *                values in the symmetric set {-7, ..., 7} (the symmetric variant).
+ *
  * Readings taken where the pages are silent (each one is exercised by a test):
  *   - codes are asymmetric uint4 in [0,15]; one fp16 scale and one fp16 zero
  *     point per group of G = 128 consecutive input channels (k) of a row n;
@@ -111,6 +114,60 @@ int w4o_quantize(const float *W, const float *awq_s, int64_t N, int64_t K,
             for (int i = 0; i < group; ++i) {
                 float q = clamp_0_15(rintf(wp[i] / sc) + z);
                 codes[n * K + k0 + i] = (uint8_t)q;
+            }
+        }
+    }
+    return 0;
+}
+
+/* clamp to [-7, 7] */
+static float clamp_pm7(float v) {
+    if (v < -7.0f) return -7.0f;
+    if (v > 7.0f) return 7.0f;
+    return v;
+}
+
+/*
+ * Symmetric variant: INT4 as the symmetric value set {-7, ..., 7} ([Notes 2.1]:
+ * mhpq.cn practitioner's article, section 2.1).  The page gives the value set
+ * only; the scale rule taken here is the plain symmetric one:
+ *   amax  = max |w'| over the group
+ *   scale = fp16(amax / 7), taken as 1.0 if that is 0
+ *   q     = clamp(rint(w' / scale), -7, 7)
+ * and the code stored is q + 8 (1..15) with zero point 8, so the asymmetric
+ * dequantization ((float)code - z) * scale gives q * scale unchanged.
+ */
+int w4o_quantize_sym(const float *W, const float *awq_s, int64_t N, int64_t K,
+                     int group, uint8_t *codes, uint16_t *scales, uint16_t *zeros) {
+    if (N < 0 || K < 0 || group <= 0 || K % group != 0) return -1;
+    fesetround(FE_TONEAREST);
+    const int64_t Kg = K / group;
+    float wp[1024];
+    if (group > 1024) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < Kg; ++g) {
+            const int64_t k0 = g * group;
+            for (int i = 0; i < group; ++i) {
+                float w = W[n * K + k0 + i];
+                wp[i] = awq_s ? w / awq_s[k0 + i] : w;
+            }
+            float amax = 0.0f;
+            for (int i = 0; i < group; ++i) {
+                float a = fabsf(wp[i]);
+                if (a > amax) amax = a;
+            }
+            float sc32 = amax / 7.0f;
+            uint16_t sc_bits = f32_to_f16_bits(sc32);
+            float sc = f16_bits_to_f32(sc_bits);
+            if (sc == 0.0f) {
+                sc = 1.0f;
+                sc_bits = f32_to_f16_bits(1.0f);
+            }
+            scales[n * Kg + g] = sc_bits;
+            zeros[n * Kg + g] = f32_to_f16_bits(8.0f);
+            for (int i = 0; i < group; ++i) {
+                float q = clamp_pm7(rintf(wp[i] / sc));
+                codes[n * K + k0 + i] = (uint8_t)(q + 8.0f);
             }
         }
     }

@@ -64,7 +64,7 @@ def test_status_strings(lib):
     (0, 128, 128, 1),      # empty
     (4, 0, 128, 1),
     (4, 200, 128, 1),      # K not a multiple of the group
-    (4, 256, 64, 2),       # unsupported group size
+    (4, 256, 48, 2),       # unsupported group size (32, 64 and 128 are served)
     (-1, 128, 128, 1),
 ])
 def test_quantize_rejects_bad_shapes(lib, N, K, group, expect):
@@ -98,7 +98,8 @@ def test_gemm_rejects(lib):
                                      kw.get("Y", A), kw.get("yd", 0), None, 0, None)
     assert g(M=0) == 1
     assert g(K=100) == 1
-    assert g(G=32) == 2
+    assert g(G=48) == 2          # group not served
+    assert g(G=32, K=96) == 2    # groups of 32 need K a multiple of 64
     assert g(xd=0) == 2          # fp32 activations are not served
     assert g(yd=1) == 2          # fp16 output not served
     assert g(X=None) == 1

@@ -316,3 +316,70 @@ def test_synthetic_row_blocks_are_consistent():
     assert np.array_equal(full[rows].numpy(), part.numpy())
     frac = (full.abs() > 0.1).float().mean().item()
     assert 0.0002 < frac < 0.003  # ~0.1% N(0,0.4) outliers, a few of them small
+
+
+# ---------------------------------------------------------------- symmetric variant {-7..7}
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_symmetric_grid_properties(group):
+    """Codes lie in {-7..7} + 8 with zero point 8. The scale is the nearest fp16
+    to max|w|/7 (numpy's conversion). Every weight is within scale/2 of its
+    reconstruction (checked in fp64)."""
+    W = _weights(N=32, K=512, outliers=0.002, tag=("sym", group))
+    codes, sc, zp = oracle.quantize_symmetric(W, group=group)
+    assert codes.min() >= 1 and codes.max() <= 15
+    assert np.all(zp.astype(np.float32) == 8.0)
+    Wg = _groups(W.astype(np.float64), group)
+    amax = np.abs(Wg).max(axis=2)
+    expect = (amax.astype(np.float32) / np.float32(7.0)).astype(np.float16)
+    assert np.array_equal(sc.view(np.uint16), expect.view(np.uint16))
+    q = _groups(codes.astype(np.float64), group) - 8.0
+    scale = sc.astype(np.float64)[:, :, None]
+    assert np.all(np.abs(Wg - q * scale) <= scale / 2 + 1e-12)
+
+
+def test_symmetric_on_grid_weights_reconstruct_exactly():
+    """w = q * c with c an fp16 value and +-7 present in every group: the scale is
+    c exactly and the codes are q + 8."""
+    rng = np.random.default_rng(5)
+    N, K = 8, 256
+    q = rng.integers(-7, 8, size=(N, K))
+    q[:, 0], q[:, 128] = 7, -7
+    c = np.float16(0.0078125 * 1.25)
+    W = (q * np.float32(c)).astype(np.float32)
+    codes, sc, zp = oracle.quantize_symmetric(W)
+    assert np.all(sc == c)
+    assert np.array_equal(codes.astype(np.int64), q + 8)
+
+
+def test_symmetric_sign_symmetry():
+    """rint is symmetric and the set {-7..7} is too: quantizing -W negates every q."""
+    W = _weights(N=16, K=384, tag="symneg")
+    c1, s1, _ = oracle.quantize_symmetric(W)
+    c2, s2, _ = oracle.quantize_symmetric(-W)
+    assert np.array_equal(s1.view(np.uint16), s2.view(np.uint16))
+    assert np.array_equal(16 - c1.astype(np.int64), c2.astype(np.int64))
+
+
+def test_symmetric_half_even_ties_and_degenerate():
+    """A worked group: with max|w| = 7 the scale is 1 and +-0.5, +-2.5 round to even
+    (0, +-2). An all-zero group gets scale 1.0 and codes 8."""
+    w = np.zeros((2, 128), np.float32)
+    w[0, :6] = [7.0, -7.0, 0.5, -0.5, 2.5, -2.5]
+    codes, sc, zp = oracle.quantize_symmetric(w)
+    assert sc[0, 0] == 1.0 and sc[1, 0] == 1.0
+    assert list(codes[0, :6].astype(int) - 8) == [7, -7, 0, 0, 2, -2]
+    assert np.all(codes[1] == 8)
+
+
+def test_symmetric_awq_unit_scale_and_dequant_matches_q_times_scale():
+    """s = 1 changes nothing. The shared dequantization ((code - 8) * scale)
+    gives q * scale exactly."""
+    W = _weights(N=8, K=256, tag="symawq")
+    c0, s0, z0 = oracle.quantize_symmetric(W)
+    c1, s1, z1 = oracle.quantize_symmetric(W, np.ones(256, np.float32))
+    assert np.array_equal(c0, c1) and np.array_equal(s0.view(np.uint16), s1.view(np.uint16))
+    What = oracle.dequant(c0, s0, z0)
+    q = c0.astype(np.float32) - 8.0
+    expect = (q.reshape(8, 2, 128) * s0.astype(np.float32)[:, :, None]).reshape(8, 256)
+    assert np.array_equal(What, expect)

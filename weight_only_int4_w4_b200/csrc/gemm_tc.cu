@@ -35,6 +35,7 @@ struct TcParams {
   uint32_t *counters;  // [tiles] arrival counters (split-K only)
   int splits;
   int kb_per_split;  // k-blocks of 64 per split
+  int group;         // quantization group: 32, 64 or 128 input channels
 };
 
 namespace tc_impl {
@@ -57,15 +58,18 @@ struct TcCfg {
 // weight turns them into (q - z) * scale: the offsets -(256 + z) * scale and
 // -(16 + z) * scale are exact in fp32 (9 + 11 significant bits), so the only
 // rounding is that of the final 16-bit conversion.
+// (sc0, z0) serve channels 0..31 of the k-block (w0) and (sc1, z1) channels
+// 32..63 (w1): the same pair for groups of 64 and 128, two pairs for groups of 32.
 template <bool kBf16, bool kAwq>
-__device__ __forceinline__ void dequant_row64(const uint4 &w0, const uint4 &w1, float sc, float z,
-                                              const float *__restrict__ sk, uint32_t (&out)[32]) {
-  const float off_lo = -(256.0f + z) * sc;
-  const float sc16 = sc * 0.0625f;
-  const float off_hi = -(16.0f + z) * sc;
+__device__ __forceinline__ void dequant_row64(const uint4 &w0, const uint4 &w1, float sc0, float z0, float sc1,
+                                              float z1, const float *__restrict__ sk, uint32_t (&out)[32]) {
   const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
   for (int wi = 0; wi < 8; ++wi) {
+    const float sc = wi < 4 ? sc0 : sc1, z = wi < 4 ? z0 : z1;
+    const float off_lo = -(256.0f + z) * sc;
+    const float sc16 = sc * 0.0625f;
+    const float off_hi = -(16.0f + z) * sc;
     const uint32_t w = words[wi];
     const uint32_t tb[4] = {w << 15, w << 7, w >> 1, w >> 9};  // byte b at bits 15..22
 #pragma unroll
@@ -187,24 +191,33 @@ __global__ void __launch_bounds__(256, 1)
     const int r = q * 32 + lane;
     const int64_t n = n0 + r;
     const bool row_ok = n < N;
-    const int64_t Kg = K / kGroup;
+    const int G = p.group;
+    const int64_t Kg = K / G;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    float sc = 0.0f, z = 0.0f;
+    float sc = 0.0f, z = 0.0f, sc1 = 0.0f, z1 = 0.0f;
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
       const int s = i % kNS;
       const uint32_t ph = (uint32_t)(i / kNS) & 1u;
       const int kb = kb0 + i;
-      if (i == 0 || (kb & 1) == 0) {
-        const int64_t grp = kb / 2;
+      if (G == 32) {  // two groups per 64-channel k-block
+        const int64_t grp = 2 * (int64_t)kb;
         sc = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp)) : 0.0f;
         z = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp)) : 0.0f;
+        sc1 = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp + 1)) : 0.0f;
+        z1 = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp + 1)) : 0.0f;
+      } else if (i == 0 || (kb & (G / 64 - 1)) == 0) {  // a group spans G / 64 k-blocks
+        const int64_t grp = kb / (G / 64);
+        sc = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp)) : 0.0f;
+        z = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp)) : 0.0f;
+        sc1 = sc;
+        z1 = z;
       }
       if (!mbar_wait(&full[s], ph, kErrTimeoutDequant)) { ok = false; break; }
       const uint4 *src = reinterpret_cast<const uint4 *>(sP + s * kPStage + r * 32);
       const uint4 w0 = src[0], w1 = src[1];
       uint32_t out[32];
-      dequant_row64<kBf16, kAwq>(w0, w1, sc, z, kAwq ? p.awq_s + (int64_t)kb * kBK : nullptr, out);
+      dequant_row64<kBf16, kAwq>(w0, w1, sc, z, sc1, z1, kAwq ? p.awq_s + (int64_t)kb * kBK : nullptr, out);
       tmem_st_32x32b_x32(lane_base + (uint32_t)(BN + s * 32), out);
       tc_wait_st();
       tc_fence_before();

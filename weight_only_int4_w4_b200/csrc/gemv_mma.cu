@@ -61,10 +61,10 @@ struct GemvParams {
   const float *awq_s;
   void *Y;
   int y_bf16;
-  float *ws;           // [kslices][M][N] fp32 partials (split-K only)
+  float *ws;           // [kslices][slots][M][N] fp32 partials (row tiles shared by CTAs)
   uint32_t *counters;  // [ceil(N/16)] split-K arrival counters
-  uint32_t *sched;     // [2 * kslices]: next row tile, CTAs done fetching (per k-slice)
   int kslices;
+  int slots;           // partial slots per k-slice and row tile (see the static partition)
   int kr;              // groups per k-slice (multiple of 4)
   int grid_x;          // CTAs per k-slice
   int xs_bytes;        // shared-memory bytes of the staged activations
@@ -137,8 +137,29 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
 // 2^e with e an integer in [-126, 127], exact.
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
 
+// Static balanced partition of a k-slice's work.  The iterations of a k-slice
+// are its (row tile, stage) pairs in tile-major order, T = RT * S of them; CTA
+// c of the slice's C CTAs takes iterations [floor(c T / C), floor((c+1) T / C)).
+// The planner keeps C <= T, so every range is non-empty.
+__device__ __forceinline__ int64_t part_begin(int64_t c, int64_t T, int64_t C) { return (c * T) / C; }
+// The CTA whose range holds iteration i.
+__device__ __forceinline__ int64_t part_owner(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
+// Stages of k-slice ks (the last slice may hold fewer groups).
+__device__ __forceinline__ int64_t slice_stages(int ks, int kr, int64_t Kg) {
+  const int64_t ng = min((int64_t)kr, Kg - (int64_t)ks * kr);
+  return (ng + kSG - 1) / kSG;
+}
+// CTAs of k-slice ks that hold part of row tile rt, and the first of them.
+__device__ __forceinline__ void tile_owners(int64_t rt, int64_t RT, int64_t C, int ks, int kr, int64_t Kg,
+                                            int64_t &first, int64_t &count) {
+  const int64_t S = slice_stages(ks, kr, Kg);
+  const int64_t T = RT * S;
+  first = part_owner(rt * S, T, C);
+  count = part_owner(rt * S + S - 1, T, C) - first + 1;
+}
+
 template <int T8, bool kBf16, bool kAwq, bool kScTma>
-__global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_kernel(const __grid_constant__ CUtensorMap tmP,
+__global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __grid_constant__ CUtensorMap tmP,
                                                    const __grid_constant__ CUtensorMap tmS,
                                                    const __grid_constant__ CUtensorMap tmZ, const GemvParams p) {
   constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
@@ -167,7 +188,8 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   const int kslice = blockIdx.y;
   const int64_t g_first = (int64_t)kslice * p.kr;
   const int ng = (int)min((int64_t)p.kr, Kg - g_first);  // groups of this k-slice
-  const int nst_task = (ng + kSG - 1) / kSG;                 // stages per task
+  const int S = (ng + kSG - 1) / kSG;                       // stages per row tile
+  const int ng_pad = S * kSG;                               // staged groups (zero beyond ng)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNst; ++s) {
@@ -184,41 +206,44 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   __syncthreads();
 
   if (warp == kComputeWarps) {
-    // ---------------- producer: fetch row tiles, drive the TMA ring
+    // ---------------- producer: walk this CTA's iteration range, drive the TMA ring.
+    // Weights are never written by a preceding kernel, so nothing here waits for it.
     if (lane == 0) {
       prefetch_tensormap(&tmP);
       if (kScTma) {
         prefetch_tensormap(&tmS);
         prefetch_tensormap(&tmZ);
       }
-      uint32_t *next = p.sched + 2 * kslice;
-      uint32_t *fin = next + 1;
-      // The first tile of every CTA is static (tile = blockIdx.x), so its weights
-      // can stream before the preceding kernel in the stream has finished; the
-      // scheduler counters (workspace) are touched only after the dependency wait.
-      int64_t rt = blockIdx.x;
-      bool waited = false;
+      const int64_t C = gridDim.x;
+      const int64_t T = RT * S;
+      const int64_t it1 = part_begin((int64_t)blockIdx.x + 1, T, C);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      while (ok) {
-        const bool have = rt < RT;
-        int64_t rt_next = RT;
-        if (waited && have) rt_next = (int64_t)gridDim.x + atomicAdd(next, 1u);  // overlaps the issue below
-        if (!have) {
-          if (!waited) grid_dependency_wait();
-          waited = true;
-          if (mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) {
-            hdr[4 * s] = -1;  // end of work
-            mbar_arrive(&full[s]);
+      for (int64_t it = part_begin(blockIdx.x, T, C); ok && it < it1;) {
+        const int64_t rt = it / S;
+        const int c0 = (int)(it - rt * S);
+        const int64_t frag_end = min(it1, (rt + 1) * (int64_t)S);
+        const int c1 = (int)(frag_end - rt * S);
+        // the fragment's place among the row tile's contributors
+        const bool direct = c0 == 0 && c1 == S && p.kslices == 1;
+        int slot = 0, ntotal = 0;
+        if (!direct) {
+          int64_t first, count;
+          tile_owners(rt, RT, C, kslice, p.kr, Kg, first, count);
+          slot = (int)((int64_t)blockIdx.x - first);
+          for (int ks = 0; ks < p.kslices; ++ks) {
+            tile_owners(rt, RT, C, ks, p.kr, Kg, first, count);
+            ntotal += (int)count;
           }
-          break;
         }
         const int32_t row0 = (int32_t)(rt * kRows);
-        for (int c = 0; c < nst_task; ++c) {
+        for (int c = c0; c < c1; ++c) {
           if (!mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) { ok = false; break; }
           hdr[4 * s + 0] = (int)rt;
-          hdr[4 * s + 1] = c;
+          hdr[4 * s + 1] = c | ((c == c1 - 1) ? (1 << 16) : 0);
+          hdr[4 * s + 2] = slot | (direct ? (1 << 16) : 0);
+          hdr[4 * s + 3] = ntotal;
           uint8_t *st = stages + s * kStage;
           mbar_arrive_expect_tx(&full[s], kScTma ? kStage : kPBytes);
           const int64_t gs = g_first + (int64_t)c * kSG;
@@ -234,20 +259,13 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
             ph ^= 1u;
           }
         }
-        if (!waited) {  // first (static) tile issued: now wait, then fetch the next one
-          grid_dependency_wait();
-          waited = true;
-          rt_next = (int64_t)gridDim.x + atomicAdd(next, 1u);
-        }
-        rt = rt_next;
+        it = frag_end;
+      }
+      if (ok && mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) {
+        hdr[4 * s] = -1;  // end of work
+        mbar_arrive(&full[s]);
       }
       grid_launch_dependents();  // all of this CTA's loads are issued
-      // every CTA of this k-slice is done fetching: the last one resets the scheduler
-      const uint32_t prev = atomicAdd(fin, 1u);
-      if (prev == gridDim.x - 1) {
-        atomicExch(next, 0u);
-        atomicExch(fin, 0u);
-      }
     }
     return;
   }
@@ -256,9 +274,12 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   // (group gl, token tok, quarter tt); every lane runs the same number of rounds
   // (the shuffles need whole warps) and a round's 4-lane quads are all valid or
   // all idle, since the thread count and the unit count are multiples of 4.
+  // Groups ng..ng_pad-1 (past the end of the k-slice) are staged as zeros, so a
+  // stage always holds whole groups that contribute exactly 0.
   grid_dependency_wait();  // X (and Y, the workspace) may come from the preceding kernel
   const uint16_t *xg = static_cast<const uint16_t *>(p.X);
   const int units = ng * Mi * 4;
+  const int units_pad = ng_pad * Mi * 4;
   // pass 1: per-token max |x * s| over the k-slice -> power-of-two exponent
   for (int r0 = 0; r0 < units; r0 += kComputeThreads) {
     const int u = r0 + threadIdx.x;
@@ -298,46 +319,53 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   }
   named_bar_compute();
   // pass 2: x' = x * s * 2^e as fp16 fragments (odd channels / 16), group sums P and S
-  for (int r0 = 0; r0 < units; r0 += kComputeThreads) {
+  for (int r0 = 0; r0 < units_pad; r0 += kComputeThreads) {
     const int u = r0 + threadIdx.x;
-    const bool valid = u < units;
+    const bool valid = u < units_pad;
     const int tt = u & 3;
     const int tok = valid ? (u >> 2) % Mi : 0;
     const int gl = valid ? (u >> 2) / Mi : 0;
+    const bool real = valid && gl < ng;
     float sumB = 0.0f, sumX = 0.0f;
     if (valid) {
-      const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
-      const uint4 *src = reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + k0);
-      const int e = xexp[tok];
-      const float se = exp2i(e), so = exp2i(e - 4);  // even channels x 2^e, odd x 2^(e-4)
       uint32_t hw[kParts][16];  // fp16 pairs (channels 2j, 2j+1) of the 32
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 v = __ldg(src + c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      for (int pp = 0; pp < kParts; ++pp)
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          float2 f = pair_to_f32<kBf16>(w[e2]);
-          if constexpr (kAwq) {
-            const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 8 * c + 2 * e2));
-            f.x *= s2.x;
-            f.y *= s2.y;
+        for (int j = 0; j < 16; ++j) hw[pp][j] = 0u;
+      if (real) {
+        const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
+        const uint4 *src = reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + k0);
+        const int e = xexp[tok];
+        const float se = exp2i(e), so = exp2i(e - 4);  // even channels x 2^e, odd x 2^(e-4)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = __ldg(src + c);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float2 f = pair_to_f32<kBf16>(w[e2]);
+            if constexpr (kAwq) {
+              const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 8 * c + 2 * e2));
+              f.x *= s2.x;
+              f.y *= s2.y;
+            }
+            f.x *= se;  // exact power-of-two scaling
+            f.y *= so;
+            const uint32_t hi = f16x2_bits(f.x, f.y);
+            const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+            hw[0][4 * c + e2] = hi;
+            float be = hv.x, bo = hv.y;
+            if constexpr (kAwq) {
+              const uint32_t lo = f16x2_bits(f.x - hv.x, f.y - hv.y);
+              const float2 lv = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+              hw[kParts - 1][4 * c + e2] = lo;
+              be += lv.x;
+              bo += lv.y;
+            }
+            sumB += be + bo;
+            sumX += fmaf(16.0f, bo, be);
           }
-          f.x *= se;  // exact power-of-two scaling
-          f.y *= so;
-          const uint32_t hi = f16x2_bits(f.x, f.y);
-          const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
-          hw[0][4 * c + e2] = hi;
-          float be = hv.x, bo = hv.y;
-          if constexpr (kAwq) {
-            const uint32_t lo = f16x2_bits(f.x - hv.x, f.y - hv.y);
-            const float2 lv = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
-            hw[kParts - 1][4 * c + e2] = lo;
-            be += lv.x;
-            bo += lv.y;
-          }
-          sumB += be + bo;
-          sumX += fmaf(16.0f, bo, be);
         }
       }
       // B fragments for MMA block b = 2i + h: B0 = (v[8i+2h], v[8i+2h+4]), B1 = (v[8i+2h+1], v[8i+2h+5]);
@@ -367,14 +395,13 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   }
   named_bar_compute();
 
-  // ---------------- stream row tiles
+  // ---------------- consume stages
   const int g = lane >> 2;
   const int t = lane & 3;
   const int blk4 = warp & 3;     // 16-row block of the tile
   const int half = warp >> 2;    // this warp takes groups 2*half, 2*half+1 of every stage
   const int ra = blk4 * 16 + g;  // smem rows of this lane's A fragments
   const int rb = ra + 8;
-  const bool split = p.kslices > 1;
   const int kslices = p.kslices;
   const uint32_t stage_base = smem_u32(stages);
   const uint32_t xs_base = smem_u32(xs);
@@ -383,16 +410,39 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   float acc[T8][4];
 #pragma unroll
   for (int o = 0; o < T8; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.0f;
-  int64_t tiles_done = 0;
-  int64_t pend_row0 = -1;  // split-K arrival of the previous tile, read one tile later
+  int64_t frags_done = 0;
+  int64_t pend_row0 = -1;  // arrival of the previous fragment's partials, read one fragment later
+  int pend_total = 0;
   uint32_t pend_ticket = 0;
 
+  // The last contributor of a row block sums every k-slice's and every
+  // fragment's partials in a fixed order (slice-major, then fragment), so the
+  // result does not depend on which CTA finishes last.
   auto finish_pending = [&]() {
     if (pend_row0 < 0) return;
     const uint32_t prev = __shfl_sync(0xffffffffu, pend_ticket, 0);
-    if (prev == (uint32_t)(kslices - 1)) {
+    if (prev == (uint32_t)(pend_total - 1)) {
       __threadfence();
       const int64_t blk = pend_row0 / 16 + blk4;
+      const int64_t rt = pend_row0 / kRows;
+      float v[T8][4];
+#pragma unroll
+      for (int o = 0; o < T8; ++o) v[o][0] = v[o][1] = v[o][2] = v[o][3] = 0.0f;
+      for (int ks = 0; ks < kslices; ++ks) {
+        int64_t first, count;
+        tile_owners(rt, RT, (int64_t)gridDim.x, ks, p.kr, Kg, first, count);
+        for (int64_t sl = 0; sl < count; ++sl) {
+          const float *base = p.ws + ((int64_t)ks * p.slots + sl) * M * N;
+#pragma unroll
+          for (int o = 0; o < T8; ++o)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int64_t row = pend_row0 + ((c < 2) ? ra : rb);
+              const int64_t tok = o * 8 + 2 * t + (c & 1);
+              if (row < N && tok < M) v[o][c] += __ldcg(base + tok * N + row);
+            }
+        }
+      }
 #pragma unroll
       for (int o = 0; o < T8; ++o)
 #pragma unroll
@@ -400,10 +450,8 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
           const int64_t row = pend_row0 + ((c < 2) ? ra : rb);
           const int64_t tok = o * 8 + 2 * t + (c & 1);
           if (row < N && tok < M) {
-            float v = 0.0f;
-            for (int sl = 0; sl < kslices; ++sl) v += __ldcg(p.ws + ((int64_t)sl * M + tok) * N + row);
-            if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[tok * N + row] = __float2bfloat16_rn(v);
-            else static_cast<float *>(p.Y)[tok * N + row] = v;
+            if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[tok * N + row] = __float2bfloat16_rn(v[o][c]);
+            else static_cast<float *>(p.Y)[tok * N + row] = v[o][c];
           }
         }
       __syncwarp();
@@ -440,50 +488,114 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
   uint32_t ph = 0;
   for (;;) {
     if (!mbar_wait(&full[s], ph, kErrTimeoutDequant)) break;
-    int rt, c;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(rt), "=r"(c) : "r"(hdr_base + (uint32_t)(s * 16)));
+    int rt, cw, sw, ntotal;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(rt), "=r"(cw), "=r"(sw), "=r"(ntotal)
+                 : "r"(hdr_base + (uint32_t)(s * 16)));
     if (rt < 0) break;
+    const int c = cw & 0xFFFF;
+    const bool last = (cw >> 16) != 0;
     const uint32_t st = stage_base + (uint32_t)(s * kStage);
-    const int64_t row0 = (int64_t)rt * kRows;
-    const int gl0 = c * kSG + 2 * half;  // first of this warp's two groups
+    const int gl0 = c * kSG + 2 * half;  // first of this warp's two groups (both < ng_pad)
 
-    if (gl0 < ng) {
-      const bool two = gl0 + 1 < ng;  // warp-uniform
-      // packed codes: one 16-byte chunk per row and group
-      const uint4 pa0 = lds128(st + a_off0), pb0 = lds128(st + b_off0);
-      const uint4 pa1 = lds128(st + a_off1), pb1 = lds128(st + b_off1);
-      // scales and zeros of both groups (adjacent fp16 in one 32-bit word)
-      uint32_t sa2, sb2, za2, zb2;
-      if constexpr (kScTma) {
-        const uint32_t off = (uint32_t)((g_first_i + gl0) & 7) * 2;
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sa2) : "r"(st + sa_off + off));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb2) : "r"(st + sb_off + off));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(za2) : "r"(st + sa_off + kSBytes + off));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(zb2) : "r"(st + sb_off + kSBytes + off));
-      } else {
-        const int64_t kg = g_first + gl0;
-        const int64_t na = row0 + ra, nb = row0 + rb;
-        const uint32_t a0 = na < N ? __ldg(p.scales + na * Kg + kg) : 0u;
-        const uint32_t b0 = nb < N ? __ldg(p.scales + nb * Kg + kg) : 0u;
-        const uint32_t c0 = na < N ? __ldg(p.zeros + na * Kg + kg) : 0u;
-        const uint32_t d0 = nb < N ? __ldg(p.zeros + nb * Kg + kg) : 0u;
-        const uint32_t a1 = (two && na < N) ? __ldg(p.scales + na * Kg + kg + 1) : 0u;
-        const uint32_t b1 = (two && nb < N) ? __ldg(p.scales + nb * Kg + kg + 1) : 0u;
-        const uint32_t c1 = (two && na < N) ? __ldg(p.zeros + na * Kg + kg + 1) : 0u;
-        const uint32_t d1 = (two && nb < N) ? __ldg(p.zeros + nb * Kg + kg + 1) : 0u;
-        sa2 = a0 | (a1 << 16);
-        sb2 = b0 | (b1 << 16);
-        za2 = c0 | (c1 << 16);
-        zb2 = d0 | (d1 << 16);
+    // packed codes: one 16-byte chunk per row and group
+    const uint4 pa0 = lds128(st + a_off0), pb0 = lds128(st + b_off0);
+    const uint4 pa1 = lds128(st + a_off1), pb1 = lds128(st + b_off1);
+    // scales and zeros of both groups (adjacent fp16 in one 32-bit word)
+    uint32_t sa2, sb2, za2, zb2;
+    if constexpr (kScTma) {
+      const uint32_t off = (uint32_t)((g_first_i + gl0) & 7) * 2;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sa2) : "r"(st + sa_off + off));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb2) : "r"(st + sb_off + off));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(za2) : "r"(st + sa_off + kSBytes + off));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(zb2) : "r"(st + sb_off + kSBytes + off));
+    } else {
+      const int64_t row0 = (int64_t)rt * kRows;
+      const int64_t kg = g_first + gl0;
+      const bool two = gl0 + 1 < ng;
+      const bool one = gl0 < ng;
+      const int64_t na = row0 + ra, nb = row0 + rb;
+      const uint32_t a0 = (one && na < N) ? __ldg(p.scales + na * Kg + kg) : 0u;
+      const uint32_t b0 = (one && nb < N) ? __ldg(p.scales + nb * Kg + kg) : 0u;
+      const uint32_t c0 = (one && na < N) ? __ldg(p.zeros + na * Kg + kg) : 0u;
+      const uint32_t d0 = (one && nb < N) ? __ldg(p.zeros + nb * Kg + kg) : 0u;
+      const uint32_t a1 = (two && na < N) ? __ldg(p.scales + na * Kg + kg + 1) : 0u;
+      const uint32_t b1 = (two && nb < N) ? __ldg(p.scales + nb * Kg + kg + 1) : 0u;
+      const uint32_t c1 = (two && na < N) ? __ldg(p.zeros + na * Kg + kg + 1) : 0u;
+      const uint32_t d1 = (two && nb < N) ? __ldg(p.zeros + nb * Kg + kg + 1) : 0u;
+      sa2 = a0 | (a1 << 16);
+      sb2 = b0 | (b1 << 16);
+      za2 = c0 | (c1 << 16);
+      zb2 = d0 | (d1 << 16);
+    }
+    const float2 sca = __half22float2(*reinterpret_cast<const __half2 *>(&sa2));
+    const float2 scb = __half22float2(*reinterpret_cast<const __half2 *>(&sb2));
+    const float2 zfa = __half22float2(*reinterpret_cast<const __half2 *>(&za2));
+    const float2 zfb = __half22float2(*reinterpret_cast<const __half2 *>(&zb2));
+    const uint32_t xg_off0 = (uint32_t)gl0 * gstride_x, xg_off1 = xg_off0 + gstride_x;
+    const uint32_t pg_off0 = (uint32_t)gl0 * gstride_p, pg_off1 = pg_off0 + gstride_p;
+
+    if constexpr (T8 <= 2) {
+      // Both groups at once, k-block by k-block: four independent accumulator chains
+      // per token octet (group x even/odd k-block), A fragments built just in time.
+      float d[T8][2][2][4];
+      const uint32_t wa0[4] = {pa0.x, pa0.y, pa0.z, pa0.w}, wb0[4] = {pb0.x, pb0.y, pb0.z, pb0.w};
+      const uint32_t wa1[4] = {pa1.x, pa1.y, pa1.z, pa1.w}, wb1[4] = {pb1.x, pb1.y, pb1.z, pb1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t A[2][2][4];  // [group][k-block parity][fragment reg]
+        {
+          const uint32_t a8 = wa0[i] >> 8, b8 = wb0[i] >> 8, a18 = wa1[i] >> 8, b18 = wb1[i] >> 8;
+          A[0][0][0] = lop3_and_or(wa0[i], 0x000F000Fu, kMagic);
+          A[0][0][2] = lop3_and_or(wa0[i], 0x00F000F0u, kMagic);
+          A[0][0][1] = lop3_and_or(wb0[i], 0x000F000Fu, kMagic);
+          A[0][0][3] = lop3_and_or(wb0[i], 0x00F000F0u, kMagic);
+          A[0][1][0] = lop3_and_or(a8, 0x000F000Fu, kMagic);
+          A[0][1][2] = lop3_and_or(a8, 0x00F000F0u, kMagic);
+          A[0][1][1] = lop3_and_or(b8, 0x000F000Fu, kMagic);
+          A[0][1][3] = lop3_and_or(b8, 0x00F000F0u, kMagic);
+          A[1][0][0] = lop3_and_or(wa1[i], 0x000F000Fu, kMagic);
+          A[1][0][2] = lop3_and_or(wa1[i], 0x00F000F0u, kMagic);
+          A[1][0][1] = lop3_and_or(wb1[i], 0x000F000Fu, kMagic);
+          A[1][0][3] = lop3_and_or(wb1[i], 0x00F000F0u, kMagic);
+          A[1][1][0] = lop3_and_or(a18, 0x000F000Fu, kMagic);
+          A[1][1][2] = lop3_and_or(a18, 0x00F000F0u, kMagic);
+          A[1][1][1] = lop3_and_or(b18, 0x000F000Fu, kMagic);
+          A[1][1][3] = lop3_and_or(b18, 0x00F000F0u, kMagic);
+        }
+#pragma unroll
+        for (int o = 0; o < T8; ++o)
+#pragma unroll
+          for (int pp = 0; pp < kParts; ++pp) {
+            // B words 4i..4i+3 of each group: (x, y) feed k-block 2i, (z, w) feed 2i+1
+            const uint4 B0 = lds128(bofs[o] + xg_off0 + (uint32_t)(pp * 256 + 16 * i));
+            const uint4 B1 = lds128(bofs[o] + xg_off1 + (uint32_t)(pp * 256 + 16 * i));
+            const bool first = i == 0 && pp == 0;
+            mma_f16(d[o][0][0], A[0][0], B0.x, B0.y, first);
+            mma_f16(d[o][1][0], A[1][0], B1.x, B1.y, first);
+            mma_f16(d[o][0][1], A[0][1], B0.z, B0.w, first);
+            mma_f16(d[o][1][1], A[1][1], B1.z, B1.w, first);
+          }
       }
-      const float2 sca = __half22float2(*reinterpret_cast<const __half2 *>(&sa2));
-      const float2 scb = __half22float2(*reinterpret_cast<const __half2 *>(&sb2));
-      const float2 zfa = __half22float2(*reinterpret_cast<const __half2 *>(&za2));
-      const float2 zfb = __half22float2(*reinterpret_cast<const __half2 *>(&zb2));
-
+      // promotion: y' += scale * (D - P - z S) per group, tokens 2t, 2t+1 of each octet
+#pragma unroll
+      for (int o = 0; o < T8; ++o)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t pg = j ? pg_off1 : pg_off0;
+          const float2 q0 = lds_f2(pofs0[o] + pg);
+          const float2 q1 = lds_f2(pofs1[o] + pg);
+          const float sa = j ? sca.y : sca.x, sb = j ? scb.y : scb.x;
+          const float za = j ? zfa.y : zfa.x, zb = j ? zfb.y : zfb.x;
+          acc[o][0] = fmaf(-sa, fmaf(za, q0.y, q0.x), fmaf(sa, d[o][j][0][0] + d[o][j][1][0], acc[o][0]));
+          acc[o][1] = fmaf(-sa, fmaf(za, q1.y, q1.x), fmaf(sa, d[o][j][0][1] + d[o][j][1][1], acc[o][1]));
+          acc[o][2] = fmaf(-sb, fmaf(zb, q0.y, q0.x), fmaf(sb, d[o][j][0][2] + d[o][j][1][2], acc[o][2]));
+          acc[o][3] = fmaf(-sb, fmaf(zb, q1.y, q1.x), fmaf(sb, d[o][j][0][3] + d[o][j][1][3], acc[o][3]));
+        }
+    } else {
+      // Many token octets: one group at a time, its A fragments reused across octets.
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        if (j == 1 && !two) break;
         const uint4 pa = j ? pa1 : pa0, pb = j ? pb1 : pb0;
         // A fragments: one SHF + four LOP3 per 32-bit word (8 codes)
         uint32_t A[8][4];
@@ -503,8 +615,8 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
         }
         const float sa = j ? sca.y : sca.x, sb = j ? scb.y : scb.x;
         const float za = j ? zfa.y : zfa.x, zb = j ? zfb.y : zfb.x;
-        const uint32_t xg_off = (uint32_t)(gl0 + j) * gstride_x;
-        const uint32_t pg_off = (uint32_t)(gl0 + j) * gstride_p;
+        const uint32_t xg_off = j ? xg_off1 : xg_off0;
+        const uint32_t pg_off = j ? pg_off1 : pg_off0;
 #pragma unroll
         for (int o = 0; o < T8; ++o) {
           if (o * 8 >= Mi) break;  // octet without real tokens (warp-uniform)
@@ -524,7 +636,6 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
               else mma_f16(d0, A[b], Bv[2 * b], Bv[2 * b + 1], pp == 0 && b == 0);
             }
           }
-          // promotion: y' += scale * (D - P - z S) for tokens 2t, 2t+1 of this octet
           const float2 q0 = lds_f2(pofs0[o] + pg_off);
           const float2 q1 = lds_f2(pofs1[o] + pg_off);
           acc[o][0] = fmaf(-sa, fmaf(za, q0.y, q0.x), fmaf(sa, d0[0] + d1[0], acc[o][0]));
@@ -541,12 +652,12 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
       s = 0;
       ph ^= 1u;
     }
-    if (c != nst_task - 1) continue;
+    if (!last) continue;
 
-    // ---------------- tile done: the two warps of a row block combine their groups
+    // ---------------- fragment done: the two warps of a row block combine their groups
     // through shared memory, handing off with (bounded) mbarrier waits
     {
-      const uint32_t pph = (uint32_t)(tiles_done & 1);
+      const uint32_t pph = (uint32_t)(frags_done & 1);
       if (half == 1) {
         if (!mbar_wait(&pair_empty[blk4], pph ^ 1u, kErrTimeoutDequant)) break;
 #pragma unroll
@@ -565,13 +676,17 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
         __syncwarp();
         if (lane == 0) mbar_arrive(&pair_empty[blk4]);
       }
-      ++tiles_done;
+      ++frags_done;
     }
     // outputs of this row block (scaled back by 2^-e), written by the half-0 warp
+    const int64_t row0 = (int64_t)rt * kRows;
     const int64_t blk = row0 / 16 + blk4;
     if (half == 0) finish_pending();
     if (half == 0 && blk < RB16) {
+      const bool direct = (sw >> 16) != 0;
+      const int slot = sw & 0xFFFF;
       const int64_t rowa = row0 + ra, rowb = row0 + rb;
+      float *part = p.ws + ((int64_t)kslice * p.slots + slot) * M * N;
 #pragma unroll
       for (int o = 0; o < T8; ++o)
 #pragma unroll
@@ -580,19 +695,20 @@ __global__ void __launch_bounds__(288, (T8 <= 1 ? 3 : (T8 == 2 ? 2 : 1))) gemv_k
           const int tok = o * 8 + 2 * t + (cc & 1);
           if (row < N && tok < Mi) {
             const float v = acc[o][cc] * exp2i(-xexp[tok]);
-            if (!split) {
+            if (direct) {
               if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[(int64_t)tok * N + row] = __float2bfloat16_rn(v);
               else static_cast<float *>(p.Y)[(int64_t)tok * N + row] = v;
             } else {
-              p.ws[((int64_t)kslice * M + tok) * N + row] = v;
+              part[(int64_t)tok * N + row] = v;
             }
           }
         }
-      if (split) {
-        // announce the partials: warp barrier, then one release atomic (read one tile later)
+      if (!direct) {
+        // announce the partials: warp barrier, then one release atomic (read one fragment later)
         __syncwarp();
         if (lane == 0) atom_release_add(&p.counters[blk], 1u, pend_ticket);
         pend_row0 = row0;
+        pend_total = ntotal;
       }
     }
 #pragma unroll

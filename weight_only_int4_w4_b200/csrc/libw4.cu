@@ -21,8 +21,9 @@
 #include "w4.h"
 
 namespace w4 {
-cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, uint8_t *packed,
-                            uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count, cudaStream_t stream);
+cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, int group,
+                            bool symmetric, uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes,
+                            int sm_count, cudaStream_t stream);
 cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,
                         cudaStream_t stream);
 }  // namespace w4
@@ -87,8 +88,8 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 enum Path { kPathGemv = 1, kPathTc = 2 };
 
-// Workspace layout: [0, 64 KiB) split-K arrival counters (one per 16-row block),
-// [64 KiB, 128 KiB) decode scheduler counters (two per k-slice), then fp32
+// Workspace layout: [0, 64 KiB) arrival counters (one per 16-row block),
+// [64 KiB, 128 KiB) reserved, then fp32
 // partials.  The counter regions are the same for every call, so partials left
 // behind by one call never land on the counters of the next; every counter is
 // reset to zero by the last CTA (or warp) that uses it.
@@ -96,13 +97,12 @@ constexpr size_t kSplitCounterBytes = 65536;
 constexpr size_t kSchedBytes = 65536;
 constexpr size_t kCounterBytes = kSplitCounterBytes + kSchedBytes;
 constexpr int64_t kMaxSplitCounters = kSplitCounterBytes / 4;
-constexpr int64_t kMaxKslices = kSchedBytes / 8;
 constexpr int kGemvXsMax = 40 * 1024;  // staged-activation budget per CTA
 
 struct GemmPlan {
   int path = 0;
   // K1
-  int t8 = 1, kr = 2, kslices = 1, grid_x = 1, xs_bytes = 0;
+  int t8 = 1, kr = 2, kslices = 1, grid_x = 1, xs_bytes = 0, slots = 1;
   bool sc_tma = false;
   // K2
   int bn = 256, splits = 1, kb_per_split = 1;
@@ -136,54 +136,52 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   const int64_t RT = cdiv(N, 64);
   const int64_t RB16 = cdiv(N, 16);
   p.sc_tma = (Kg % 8) == 0;
-  // k-slices are whole pipeline stages of 4 groups.  Longest one whose activations
-  // fit the staging budget:
-  int64_t kr_max = std::min<int64_t>(cdiv(Kg, 4) * 4, 4096);
-  while (kr_max > 4 && w4::gemv_xs_bytes((int)kr_max, M, awq) > kGemvXsMax) kr_max -= 4;
-  // Slice length from a cost model fitted to B200 measurements of this kernel: a CTA
-  // streams at ~20 GB/s (its TMA ring depth over the loaded memory latency), the
-  // whole GPU at ~6.5 TB/s, a launch costs ~4 us, and every extra k-slice adds
-  // activation staging plus split-K partials (~3 us, then ~1.2 us per slice).
-  int64_t kr = kr_max;
-  {
-    const double bytes = (double)N * (double)K * (0.5 + 4.0 / w4::kGroup);
-    double best = 1e300;
-    int64_t prev = -1;
-    for (int64_t ks = cdiv(Kg, kr_max); ks <= 8; ++ks) {
-      const int64_t cand = cdiv(cdiv(Kg, ks), 4) * 4;  // balanced slices, whole stages
-      if (cand == prev || cand > kr_max) continue;
-      prev = cand;
-      const int64_t nks = cdiv(Kg, cand);
-      const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(w4::gemv_xs_bytes((int)cand, M, awq), p.t8);
-      const double ctas = (double)std::min<int64_t>(RT * nks, slots);
-      const double stream_us = std::max(bytes / (ctas * 20e9), bytes / 6.5e12) * 1e6;
-      const double est = 4.0 + stream_us + (nks > 1 ? 3.0 + 1.2 * (double)nks : 0.0);
-      if (est < best) {
-        best = est;
-        kr = cand;
-      }
-      if (cand <= 4) break;
-    }
-  }
+  // k-slices are whole pipeline stages of 4 groups; the longest one whose
+  // activations fit the staging budget (every CTA stages its whole k-slice).
+  // The static partition balances the work across CTAs, so K is split only
+  // when the activations do not fit.
+  int64_t kr = std::min<int64_t>(cdiv(Kg, 4) * 4, 4096);
+  while (kr > 4 && w4::gemv_xs_bytes((int)kr, M, awq) > kGemvXsMax) kr -= 4;
   if (const char *e = getenv("W4_GEMV_KR")) {  // tuning override
     const int64_t v = atoi(e);
-    if (v >= 4 && v % 4 == 0 && v <= kr_max) kr = v;
+    if (v >= 4 && v % 4 == 0 && v <= kr) kr = v;
   }
   int64_t ks = cdiv(Kg, kr);
-  if ((ks > 1 && RB16 > kMaxSplitCounters) || ks > kMaxKslices) {  // counters: fall back to the longest slices
-    kr = kr_max;
-    ks = cdiv(Kg, kr);
-  }
   p.kr = (int)kr;
   p.kslices = (int)ks;
   p.xs_bytes = w4::gemv_xs_bytes(p.kr, M, awq);
+  // stages per row tile: S_full for every k-slice but the last, S_last for the last
+  const int64_t S_full = kr / 4;
+  const int64_t S_last = cdiv(Kg - (ks - 1) * kr, 4);
   const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(p.xs_bytes, p.t8);
-  p.grid_x = (int)std::min<int64_t>(RT, std::max<int64_t>(1, slots / ks));
+  int64_t C = std::max<int64_t>(1, slots / ks);
   if (const char *e = getenv("W4_GEMV_GX")) {  // tuning override
     const int v = atoi(e);
-    if (v >= 1) p.grid_x = (int)std::min<int64_t>(RT, v);
+    if (v >= 1) C = v;
   }
-  p.ws_bytes = kCounterBytes + (ks > 1 ? (size_t)ks * M * N * 4 : 0);
+  C = std::min<int64_t>(C, RT * std::min(S_full, S_last));  // every CTA gets >= 1 iteration
+  p.grid_x = (int)C;
+  // Partial slots per (k-slice, row tile): a tile's S iterations meet at most
+  // floor((S - 2) / L) + 2 CTA ranges, L = the shortest range, floor(S * RT / C).
+  auto bound = [&](int64_t S) -> int64_t {
+    if (S <= 1) return 1;
+    const int64_t L = (S * RT) / C;
+    return std::min<int64_t>(C, (S - 2) / L + 2);
+  };
+  p.slots = (int)std::max(bound(S_full), bound(S_last));
+  bool partials = ks > 1 || RT % C != 0;
+  if (partials && RB16 > kMaxSplitCounters) {
+    // more row blocks than arrival counters: one CTA per row tile (no partials) if
+    // K is not split, else not served by this kernel
+    if (ks > 1) {
+      p.path = 0;
+      return p;
+    }
+    p.grid_x = (int)RT;
+    p.slots = 1;
+    partials = false;
+  }
+  p.ws_bytes = kCounterBytes + (partials ? (size_t)ks * p.slots * M * N * 4 : 0);
   return p;
 }
 
@@ -210,7 +208,10 @@ bool gemv_fits(int64_t M, int64_t N, bool awq) {
 GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   int f = forced_path();
   if (f == kPathTc) return plan_tc(M, N, K, sm);
-  if (f == kPathGemv || gemv_fits(M, N, awq)) return plan_gemv(M, N, K, awq, sm);
+  if (f == kPathGemv || gemv_fits(M, N, awq)) {
+    const GemmPlan p = plan_gemv(M, N, K, awq, sm);
+    if (p.path == kPathGemv || f == kPathGemv) return p;
+  }
   return plan_tc(M, N, K, sm);
 }
 
@@ -219,9 +220,10 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   GemmPlan p = plan_gemm_raw(M, N, K, awq, sm);
   if (getenv("W4_DEBUG_PLAN")) {
     if (p.path == kPathGemv)
-      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld decode: t8=%d kr=%d kslices=%d grid_x=%d xs=%d scale_tma=%d ws=%zu\n",
-              (long long)M, (long long)N, (long long)K, p.t8, p.kr, p.kslices, p.grid_x, p.xs_bytes, (int)p.sc_tma,
-              p.ws_bytes);
+      fprintf(stderr,
+              "[w4] M=%lld N=%lld K=%lld decode: t8=%d kr=%d kslices=%d grid_x=%d slots=%d xs=%d scale_tma=%d ws=%zu\n",
+              (long long)M, (long long)N, (long long)K, p.t8, p.kr, p.kslices, p.grid_x, p.slots, p.xs_bytes,
+              (int)p.sc_tma, p.ws_bytes);
     else
       fprintf(stderr, "[w4] M=%lld N=%lld K=%lld tensor-core: bn=%d splits=%d kb_per_split=%d ws=%zu\n",
               (long long)M, (long long)N, (long long)K, p.bn, p.splits, p.kb_per_split, p.ws_bytes);
@@ -241,7 +243,8 @@ size_t ws_size_all(int64_t M, int64_t N, int64_t K, int sm) {
 w4_status check_shape(int64_t M, int64_t N, int64_t K, int group) {
   if (N < 1 || K < 1 || M < 1) return fail(W4_ERR_INVALID_ARG, "sizes must be >= 1 (M=%lld N=%lld K=%lld)",
                                            (long long)M, (long long)N, (long long)K);
-  if (group != w4::kGroup) return fail(W4_ERR_UNSUPPORTED, "group=%d: only 128 is served", group);
+  if (group != 32 && group != 64 && group != 128)
+    return fail(W4_ERR_UNSUPPORTED, "group=%d: 32, 64 and 128 are served", group);
   if (K % group != 0) return fail(W4_ERR_INVALID_ARG, "K=%lld is not a multiple of the group (%d)", (long long)K, group);
   const int64_t lim = (int64_t)1 << 40;
   if (N > lim || K > lim || M > lim || (double)N * (double)K > 9.0e18 || (double)M * (double)N > 4.0e18 ||
@@ -268,8 +271,13 @@ const char *w4_status_string(w4_status s) {
 
 const char *w4_last_error(void) { return t_last_error.c_str(); }
 
-w4_status w4_quantize(const void *W, w4_dtype w_dtype, const float *awq_s, int64_t N, int64_t K, int group,
-                      uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, w4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+w4_status quantize_common(const void *W, w4_dtype w_dtype, const float *awq_s, int64_t N, int64_t K, int group,
+                          bool symmetric, uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes,
+                          w4_stream_t stream) {
   t_last_error.clear();
   w4_status st = check_shape(1, N, K, group);
   if (st != W4_OK) return st;
@@ -282,10 +290,25 @@ w4_status w4_quantize(const void *W, w4_dtype w_dtype, const float *awq_s, int64
   int sm = 0;
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
-  e = w4::launch_quantize(W, (int)w_dtype, awq_s, N, K, packed, scales, zeros, codes, sm,
+  e = w4::launch_quantize(W, (int)w_dtype, awq_s, N, K, group, symmetric, packed, scales, zeros, codes, sm,
                           reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return W4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+w4_status w4_quantize(const void *W, w4_dtype w_dtype, const float *awq_s, int64_t N, int64_t K, int group,
+                      uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, w4_stream_t stream) {
+  return quantize_common(W, w_dtype, awq_s, N, K, group, false, packed, scales, zeros, codes, stream);
+}
+
+w4_status w4_quantize_symmetric(const void *W, w4_dtype w_dtype, const float *awq_s, int64_t N, int64_t K,
+                                int group, uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes,
+                                w4_stream_t stream) {
+  return quantize_common(W, w_dtype, awq_s, N, K, group, true, packed, scales, zeros, codes, stream);
 }
 
 w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, w4_stream_t stream) {
@@ -319,6 +342,11 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
   if (x_dtype != W4_F16 && x_dtype != W4_BF16)
     return fail(W4_ERR_UNSUPPORTED, "activation dtype must be F16 or BF16");
   if (y_dtype != W4_F32 && y_dtype != W4_BF16) return fail(W4_ERR_UNSUPPORTED, "output dtype must be F32 or BF16");
+  // Groups of 32 or 64 are served by the tensor-core kernel (64-channel k-blocks).
+  if (group != w4::kGroup) {
+    if (K % 64 != 0) return fail(W4_ERR_UNSUPPORTED, "group=%d needs K a multiple of 64 (K=%lld)", group, (long long)K);
+    if (forced_path() == kPathGemv) return fail(W4_ERR_UNSUPPORTED, "the decode kernel serves group 128 only");
+  }
   if (!X || !packed || !scales || !zeros || !Y) return fail(W4_ERR_INVALID_ARG, "null X, packed, scales, zeros or Y");
   if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y) ||
       (awq_s && !aligned16(awq_s)) || (workspace && !aligned16(workspace)))
@@ -327,7 +355,10 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const bool awq = awq_s != nullptr;
-  const GemmPlan plan = plan_gemm(M, N, K, awq, sm);
+  const GemmPlan plan = group == w4::kGroup ? plan_gemm(M, N, K, awq, sm) : plan_tc(M, N, K, sm);
+  if (plan.path == 0)
+    return fail(W4_ERR_UNSUPPORTED, "W4_FORCE_PATH=gemv cannot serve N=%lld with K split into k-slices",
+                (long long)N);
   if (plan.path == kPathGemv && !w4::gemv_supports(M, awq))
     return fail(W4_ERR_UNSUPPORTED, "W4_FORCE_PATH=gemv cannot serve M=%lld%s", (long long)M, awq ? " with AWQ" : "");
   if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes))
@@ -373,8 +404,7 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
     p.scales = scales; p.zeros = zeros; p.awq_s = awq_s;
     p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
     p.ws = partials; p.counters = counters;
-    p.sched = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kSplitCounterBytes);
-    p.kslices = plan.kslices; p.kr = plan.kr; p.grid_x = plan.grid_x; p.xs_bytes = plan.xs_bytes;
+    p.kslices = plan.kslices; p.slots = plan.slots; p.kr = plan.kr; p.grid_x = plan.grid_x; p.xs_bytes = plan.xs_bytes;
     e = w4::launch_gemv(tmP, tmS, tmZ, p, plan.t8, xbf16, plan.sc_tma, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
     return W4_OK;
@@ -406,6 +436,7 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
   p.scales = scales; p.zeros = zeros; p.awq_s = awq_s;
   p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
   p.ws = partials; p.counters = counters; p.splits = plan.splits; p.kb_per_split = plan.kb_per_split;
+  p.group = group;
   e = w4::launch_gemm_tc(tmX, tmP, p, xbf16, plan.bn, s);
   if (e != cudaSuccess) return cuda_fail(e, "tensor-core gemm launch");
   return W4_OK;
@@ -515,6 +546,7 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
   w4_status st = check_shape(M, N, K, group);
   if (st != W4_OK) return st;
   const bool awq = awq_s != nullptr;
+  if (group != w4::kGroup) return fail(W4_ERR_UNSUPPORTED, "the static-scratch decode GEMM serves group 128 only");
   if (!w4::gemv_supports(M, awq))
     return fail(W4_ERR_UNSUPPORTED, "the static-scratch decode GEMM serves M <= 64 (M <= 32 with AWQ), got M=%lld%s",
                 (long long)M, awq ? " with AWQ" : "");

@@ -1,9 +1,10 @@
-// quantize.cu -- K0: per-group asymmetric uint4 RTN quantize + nibble pack.
+// quantize.cu -- K0: per-group uint4 RTN quantize + nibble pack.
 //
-// One warp owns one group of 128 consecutive input channels of one output
-// row (affine map through a scale and a zero point, per group of 128:
-// "LLM inference acceleration" article, section 2.1); each lane holds 4
-// weights.  Optional AWQ prescale w / s[k] is applied on load (ch. 22
+// Asymmetric codes: an affine map through a scale and a zero point per group of
+// 128 input channels ("LLM inference acceleration" article, section 2.1), also
+// served with groups of 32 and 64.  Symmetric variant: INT4 as the value set
+// {-7..7} (mhpq.cn practitioner's article, section 2.1), stored as q + 8 with
+// zero point 8.  Each lane holds 4 weights; a group is held by G/4 lanes.  Optional AWQ prescale w / s[k] is applied on load (ch. 22
 // "Advanced inference optimisation", section 22.3, AWQ equation).  Every
 // step uses IEEE fp32 round-to-nearest intrinsics so the results are bit-exact
 // with the definition in w4.h.  The kernel is HBM-bound: it reads W once and
@@ -48,27 +49,35 @@ struct Load4<__nv_bfloat16> {
 };
 
 __device__ __forceinline__ float clamp15(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
+__device__ __forceinline__ float clamp7(float v) { return fminf(fmaxf(v, -7.0f), 7.0f); }
 
-constexpr int kQuantUnroll = 4;  // groups in flight per warp
+constexpr int kQuantUnroll = 4;  // 128-element chunks in flight per warp
 
-template <typename TW, bool kAwq, bool kCodes>
+// The matrix is walked as its flattened N*K elements in chunks of 128: lane l of
+// a warp holds elements 4l..4l+3 of a chunk, and a group of G (32, 64 or 128)
+// consecutive elements (groups never straddle rows, since G divides K) is held
+// by G/4 consecutive lanes, which reduce its min and max with shuffles.  Group j
+// of the flattened order is scales[j] / zeros[j] of the [N][K/G] arrays.
+template <typename TW, bool kAwq, bool kCodes, bool kSym>
 __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W, const float *__restrict__ awq_s,
-                                                       int64_t total_groups, int64_t groups_per_row,
+                                                       int64_t E, int64_t K, int group,
                                                        uint8_t *__restrict__ packed, uint16_t *__restrict__ scales,
                                                        uint16_t *__restrict__ zeros, uint8_t *__restrict__ codes) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t chunks = (E + 127) / 128;
+  const int lg = group >> 2;  // lanes per group
 
-  for (int64_t base = warp * kQuantUnroll; base < total_groups; base += nwarps * kQuantUnroll) {
+  for (int64_t base = warp * kQuantUnroll; base < chunks; base += nwarps * kQuantUnroll) {
     float v[kQuantUnroll][4];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t gid = base + u;
-      if (gid < total_groups) {
-        Load4<TW>::run(W + gid * kGroup + lane * 4, v[u]);
+      const int64_t e = (base + u) * 128 + lane * 4;
+      if (e < E) {
+        Load4<TW>::run(W + e, v[u]);
         if (kAwq) {
-          const int64_t k = (gid % groups_per_row) * kGroup + lane * 4;
+          const int64_t k = e % K;
           const float4 s = __ldg(reinterpret_cast<const float4 *>(awq_s + k));
           v[u][0] = __fdiv_rn(v[u][0], s.x);
           v[u][1] = __fdiv_rn(v[u][1], s.y);
@@ -81,34 +90,48 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
     }
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t gid = base + u;
+      const int64_t e = (base + u) * 128 + lane * 4;
       float mn = fminf(fminf(v[u][0], v[u][1]), fminf(v[u][2], v[u][3]));
       float mx = fmaxf(fmaxf(v[u][0], v[u][1]), fmaxf(v[u][2], v[u][3]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
+      for (int o = lg >> 1; o > 0; o >>= 1) {  // within each aligned run of lg lanes
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
-      // scale = fp16((mx - mn) / 15); a zero fp16 scale is taken as 1.0
-      const float sc32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-      __half sc16 = __float2half_rn(sc32);
-      float sc = __half2float(sc16);
-      if (sc == 0.0f) {
-        sc = 1.0f;
-        sc16 = __float2half_rn(1.0f);
-      }
-      const float z = clamp15(rintf(__fdiv_rn(-mn, sc)));
       uint32_t q[4];
+      __half sc16;
+      float z;
+      if constexpr (kSym) {
+        // scale = fp16(max|w| / 7) (1.0 if 0); q = clamp(rint(w / scale), -7, 7), stored as q + 8
+        const float amax = fmaxf(fabsf(mn), fabsf(mx));
+        sc16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        float sc = __half2float(sc16);
+        if (sc == 0.0f) {
+          sc = 1.0f;
+          sc16 = __float2half_rn(1.0f);
+        }
+        z = 8.0f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) q[j] = (uint32_t)clamp15(__fadd_rn(rintf(__fdiv_rn(v[u][j], sc)), z));
-      if (gid < total_groups) {
+        for (int j = 0; j < 4; ++j) q[j] = (uint32_t)(clamp7(rintf(__fdiv_rn(v[u][j], sc))) + 8.0f);
+      } else {
+        // scale = fp16((mx - mn) / 15); a zero fp16 scale is taken as 1.0
+        sc16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+        float sc = __half2float(sc16);
+        if (sc == 0.0f) {
+          sc = 1.0f;
+          sc16 = __float2half_rn(1.0f);
+        }
+        z = clamp15(rintf(__fdiv_rn(-mn, sc)));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) q[j] = (uint32_t)clamp15(__fadd_rn(rintf(__fdiv_rn(v[u][j], sc)), z));
+      }
+      if (e < E) {
         const uint16_t pk = (uint16_t)(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
-        reinterpret_cast<uint16_t *>(packed + gid * (kGroup / 2))[lane] = pk;
-        if (kCodes)
-          reinterpret_cast<uint32_t *>(codes + gid * kGroup)[lane] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
-        if (lane == 0) {
-          scales[gid] = __half_as_ushort(sc16);
-          zeros[gid] = __half_as_ushort(__float2half_rn(z));
+        reinterpret_cast<uint16_t *>(packed)[e >> 2] = pk;
+        if (kCodes) reinterpret_cast<uint32_t *>(codes)[e >> 2] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+        if ((lane & (lg - 1)) == 0) {
+          const int64_t gi = e / group;
+          scales[gi] = __half_as_ushort(sc16);
+          zeros[gi] = __half_as_ushort(__float2half_rn(z));
         }
       }
     }
@@ -149,38 +172,50 @@ int grid_for(int64_t work_items, int items_per_block, int sm_count, int blocks_p
   return (int)need;
 }
 
-template <typename TW>
-cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, uint8_t *packed,
+template <typename TW, bool kSym>
+cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, int group, uint8_t *packed,
                               uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
                               cudaStream_t stream) {
-  const int64_t gpr = K / kGroup;
-  const int64_t total = N * gpr;
-  const int grid = grid_for(total, 8 * kQuantUnroll, sm_count, 8);
+  const int64_t E = N * K;
+  const int64_t chunks = (E + 127) / 128;
+  const int grid = grid_for(chunks, 8 * kQuantUnroll, sm_count, 8);
   const TW *w = static_cast<const TW *>(W);
   if (awq_s) {
     if (codes)
-      quantize_kernel<TW, true, true><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+      quantize_kernel<TW, true, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
     else
-      quantize_kernel<TW, true, false><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+      quantize_kernel<TW, true, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
   } else {
     if (codes)
-      quantize_kernel<TW, false, true><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+      quantize_kernel<TW, false, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
     else
-      quantize_kernel<TW, false, false><<<grid, 256, 0, stream>>>(w, awq_s, total, gpr, packed, scales, zeros, codes);
+      quantize_kernel<TW, false, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
   }
   return cudaGetLastError();
 }
 
+template <bool kSym>
+cudaError_t launch_quantize_s(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, int group,
+                              uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
+                              cudaStream_t stream) {
+  switch (dtype) {
+    case 0: return launch_quantize_t<float, kSym>(W, awq_s, N, K, group, packed, scales, zeros, codes, sm_count, stream);
+    case 1: return launch_quantize_t<__half, kSym>(W, awq_s, N, K, group, packed, scales, zeros, codes, sm_count, stream);
+    default:
+      return launch_quantize_t<__nv_bfloat16, kSym>(W, awq_s, N, K, group, packed, scales, zeros, codes, sm_count, stream);
+  }
+}
+
 }  // namespace quant_impl
 
-// dtype: 0 = fp32, 1 = fp16, 2 = bf16
-cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, uint8_t *packed,
-                            uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count, cudaStream_t stream) {
-  switch (dtype) {
-    case 0: return quant_impl::launch_quantize_t<float>(W, awq_s, N, K, packed, scales, zeros, codes, sm_count, stream);
-    case 1: return quant_impl::launch_quantize_t<__half>(W, awq_s, N, K, packed, scales, zeros, codes, sm_count, stream);
-    default: return quant_impl::launch_quantize_t<__nv_bfloat16>(W, awq_s, N, K, packed, scales, zeros, codes, sm_count, stream);
-  }
+// dtype: 0 = fp32, 1 = fp16, 2 = bf16; group 32, 64 or 128; symmetric selects the {-7..7} variant
+cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, int group,
+                            bool symmetric, uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes,
+                            int sm_count, cudaStream_t stream) {
+  return symmetric ? quant_impl::launch_quantize_s<true>(W, dtype, awq_s, N, K, group, packed, scales, zeros, codes,
+                                                         sm_count, stream)
+                   : quant_impl::launch_quantize_s<false>(W, dtype, awq_s, N, K, group, packed, scales, zeros, codes,
+                                                          sm_count, stream);
 }
 
 cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,

@@ -5,7 +5,7 @@ current CUDA stream to the C ABI declared in ``include/w4.h``; all arithmetic
 runs in the library's CUDA kernels.  There is no fallback: if ``libw4.so`` is
 not built, importing this module raises.
 
-Names follow the C ABI: ``w4_quantize``, ``w4_pack``, ``w4a16_gemm``,
+Names follow the C ABI: ``w4_quantize`` (and ``w4_quantize_symmetric``), ``w4_pack``, ``w4a16_gemm``,
 ``w4a16_gemm_workspace_size``, ``w4a16_gemm_host``, ``w4a16_gemm_decode_static``,
 ``w4_device_error``.
 """
@@ -24,6 +24,7 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 _P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 _lib.w4_quantize.argtypes = [_P, ctypes.c_int, _P, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P]
+_lib.w4_quantize_symmetric.argtypes = [_P, ctypes.c_int, _P, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P]
 _lib.w4_pack.argtypes = [_P, _I64, _I64, _P, _P]
 _lib.w4a16_gemm.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, ctypes.c_int,
                             _P, _SZ, _P]
@@ -39,7 +40,7 @@ _lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
 _lib.w4_status_string.argtypes = [ctypes.c_int]
 _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
-for _f in ("w4_quantize", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
+for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -77,9 +78,10 @@ def w4_status_string(status: int) -> str:
 
 
 def w4_quantize(W: torch.Tensor, awq_s: torch.Tensor | None = None, group: int = GROUP,
-                return_codes: bool = False, stream=None):
+                return_codes: bool = False, stream=None, symmetric: bool = False):
     """Quantize + pack W [N, K] (fp32/fp16/bf16, CUDA).  Returns (packed u8 [N,K/2],
-    scales f16 [N,K/G], zeros f16 [N,K/G]) and, with return_codes, codes u8 [N,K]."""
+    scales f16 [N,K/G], zeros f16 [N,K/G]) and, with return_codes, codes u8 [N,K].
+    symmetric=True calls w4_quantize_symmetric (codes q + 8, q in [-7, 7])."""
     assert W.is_cuda and W.dim() == 2 and W.is_contiguous() and W.dtype in _DT
     N, K = W.shape
     dev = W.device
@@ -89,8 +91,9 @@ def w4_quantize(W: torch.Tensor, awq_s: torch.Tensor | None = None, group: int =
     codes = torch.empty((N, K), dtype=torch.uint8, device=dev) if return_codes else None
     if awq_s is not None:
         assert awq_s.is_cuda and awq_s.dtype == torch.float32 and awq_s.is_contiguous()
-    _check(_lib.w4_quantize(_ptr(W), _DT[W.dtype], _ptr(awq_s), N, K, group, _ptr(packed), _ptr(scales),
-                            _ptr(zeros), _ptr(codes), _stream(stream)), "w4_quantize")
+    fn, name = (_lib.w4_quantize_symmetric, "w4_quantize_symmetric") if symmetric else (_lib.w4_quantize, "w4_quantize")
+    _check(fn(_ptr(W), _DT[W.dtype], _ptr(awq_s), N, K, group, _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(codes),
+              _stream(stream)), name)
     return (packed, scales, zeros, codes) if return_codes else (packed, scales, zeros)
 
 
