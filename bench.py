@@ -466,6 +466,34 @@ def stack70b_leg(w4, replays=3):
     return out
 
 
+def awq_search_leg(w4, repeats=3):
+    """AWQ exponent search on the Llama-3-8B gate_up weights with a 512-row calibration batch
+    (1% of the channels x10), 21 exponents in [-1, 1]: device time per search."""
+    dev = torch.device("cuda")
+    K, N = synthetic.SHAPES_8B["gate_up"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synthetic.seed_of("bench", "awq-search") % (2 ** 62))
+    W = torch.randn((N, K), generator=gen, device=dev) * 0.02
+    X = torch.randn((512, K), generator=gen, device=dev)
+    X[:, torch.randperm(K, generator=gen, device=dev)[: K // 100]] *= 10.0
+    X = X.to(torch.bfloat16)
+    w4.w4_awq_search(W, X)  # warm-up
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(repeats):
+        _, best, errs = w4.w4_awq_search(W, X)
+    b.record()
+    torch.cuda.synchronize()
+    zero = errs[w4.AWQ_EXPONENTS.index(0.0)]
+    out = {"ms_per_search": round(a.elapsed_time(b) / repeats, 3), "exponents": len(w4.AWQ_EXPONENTS),
+           "best_exponent": best, "error_vs_plain_rtn": round(min(errs) / zero, 4),
+           "workload": "gate_up 4096->28672 fp32 W, 512 x 4096 bf16 calibration with 1% channels x10"}
+    del W, X
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -510,6 +538,7 @@ def main():
                                            "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4)}}
         pf, pf_all, pf_ms = prefill_leg(w4)
         extras["stack70b"] = stack70b_leg(w4)
+        extras["awq_search"] = awq_search_leg(w4)
         extras["prefill"] = {"value": round(pf_all, 1), "unit": "TFLOP/s", "ms_per_step": round(pf_ms, 3),
                              "workload": "Llama-3-70B qkv/o_proj/gate_up/down, M=8192, bf16 X",
                              "per_layer_tflops": pf,

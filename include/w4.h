@@ -155,6 +155,39 @@ w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype,
                           w4_stream_t stream);
 
 /*
+ * AWQ scale search (offline, before w4_quantize).  AWQ quantizes W / s and
+ * multiplies back by s, with s a per-input-channel activation magnitude from
+ * calibration data (ch. 22 "Advanced inference optimisation", section 22.3);
+ * a quantized layer is judged by its output error || X W^T - X W^^T ||_F^2 on
+ * calibration activations X (same section).  Here s = m^a with
+ * m_k = mean over the calibration rows of |x_k| (fp64; s = 1 where m_k = 0),
+ * and a is the exponent of `alphas` with the smallest error (the first on ties).
+ *   W         device [N][K] fp32 (the dense weights)
+ *   Xcal      device [Mc][K] F16 or BF16 calibration activations
+ *   group     32, 64 or 128 (as for w4_quantize)
+ *   alphas    HOST array of 1..256 finite exponents (negative ones protect the
+ *             channels with large activations: W / s is then larger there)
+ *   awq_s     device [K] fp32 out: s for the best exponent, to be given to
+ *             w4_quantize and w4a16_gemm
+ *   errors    HOST [n_alpha] out (fp64 output error per exponent), or NULL
+ *   best      HOST out: index of the best exponent
+ *   workspace device scratch of w4_awq_search_workspace_size(Mc, N, K, group)
+ *             bytes, zero-filled before its first use (it holds a w4a16_gemm
+ *             workspace, left zero-filled by every call).
+ * Runs the quantizer and w4a16_gemm once per exponent and a dense fp32
+ * reference GEMM once; synchronizes `stream` before returning.
+ */
+w4_status w4_awq_search(const float *W, int64_t N, int64_t K, int group,
+                        const void *Xcal, w4_dtype x_dtype, int64_t Mc,
+                        const float *alphas, int n_alpha, float *awq_s,
+                        double *errors, int *best, void *workspace,
+                        size_t workspace_bytes, w4_stream_t stream);
+
+/* Bytes of workspace w4_awq_search needs (0 for invalid sizes). */
+size_t w4_awq_search_workspace_size(int64_t Mc, int64_t N, int64_t K,
+                                    int group);
+
+/*
  * Decode GEMM with library-owned scratch: the same computation, kernel and
  * result as w4a16_gemm for decode shapes, with no workspace argument.  The
  * source pages have no counterpart to this call; it exists for callers that

@@ -39,6 +39,7 @@ def _load():
         I64 = ctypes.c_int64
         _lib.w4o_quantize.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
         _lib.w4o_quantize_sym.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
+        _lib.w4o_awq_search.argtypes = [P, I64, I64, ctypes.c_int, P, I64, P, ctypes.c_int, P, P, P]
         _lib.w4o_pack.argtypes = [P, I64, I64, P]
         _lib.w4o_unpack.argtypes = [P, I64, I64, P]
         _lib.w4o_dequant.argtypes = [P, P, P, P, I64, I64, ctypes.c_int, P]
@@ -84,6 +85,24 @@ def quantize_symmetric(W, awq_s=None, group: int = 128):
     if rc != 0:
         raise ValueError("w4o_quantize_sym rejected its arguments")
     return codes, scales.view(np.float16), zeros.view(np.float16)
+
+
+def awq_search(W, X, alphas, group: int = 128):
+    """AWQ exponent search: W [N,K] fp32, X [Mc,K] (values of 16-bit inputs, as floats),
+    alphas (exponent grid) -> (errors fp64 [n_alpha], s fp32 [K] of the best, best index)."""
+    W = _c(W, np.float32)
+    X = _c(X, np.float32)
+    a = _c(np.asarray(alphas, np.float64), np.float64)
+    N, K = W.shape
+    Mc = X.shape[0]
+    errors = np.empty(len(a), np.float64)
+    s = np.empty(K, np.float32)
+    best = ctypes.c_int(-1)
+    rc = _load().w4o_awq_search(_ptr(W), N, K, group, _ptr(X), Mc, _ptr(a), len(a), _ptr(errors), _ptr(s),
+                                ctypes.byref(best))
+    if rc != 0:
+        raise ValueError("w4o_awq_search rejected its arguments")
+    return errors, s, best.value
 
 
 def pack(codes):

@@ -42,6 +42,7 @@
 #include <fenv.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* fp32 -> IEEE binary16, round-to-nearest-even (compiler conversion). */
@@ -244,4 +245,61 @@ int w4o_gemm(const float *X, const float *What, int64_t M, int64_t N,
             if (bound) bound[m * N + n] = abs_acc;
         }
     return 0;
+}
+
+/*
+ * AWQ scale search.  AWQ takes a per-input-channel activation magnitude s from
+ * calibration data and quantizes W / s ([Ch22 22.3], AWQ); the quality
+ * measure of a quantized layer is its output error on calibration activations,
+ * || X W^T - X W^^T ||_F^2 ([Ch22 22.3], the objective stated for GPTQ).
+ * Reading taken (the page gives no formula for s): s_k = m_k^a with
+ * m_k = mean over the calibration rows of |x_k| (fp64), rounded to fp32 (1 where
+ * m_k = 0), and the exponent a is the one of the given grid with the smallest
+ * error (the first one on ties).
+ *
+ * X [Mc][K] holds the calibration activations as floats; W [N][K] fp32.
+ * Outputs: errors [n_alpha] (fp64), s_out [K] for the best exponent, *best.
+ * Plain loops: the error of each exponent is the fp64 sum of squared
+ * differences between the fp64 products X W^T and X W^^T.
+ */
+int w4o_awq_search(const float *W, int64_t N, int64_t K, int group,
+                   const float *X, int64_t Mc, const double *alphas,
+                   int n_alpha, double *errors, float *s_out, int *best) {
+    if (N < 1 || K < 1 || Mc < 1 || n_alpha < 1 || group <= 0 || K % group != 0) return -1;
+    double *m = (double *)malloc(sizeof(double) * (size_t)K);
+    float *s = (float *)malloc(sizeof(float) * (size_t)K);
+    uint8_t *codes = (uint8_t *)malloc((size_t)(N * K));
+    uint16_t *sc = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(N * (K / group)));
+    uint16_t *zp = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(N * (K / group)));
+    float *What = (float *)malloc(sizeof(float) * (size_t)(N * K));
+    double *Yref = (double *)malloc(sizeof(double) * (size_t)(Mc * N));
+    double *Yq = (double *)malloc(sizeof(double) * (size_t)(Mc * N));
+    int rc = -1;
+    if (!m || !s || !codes || !sc || !zp || !What || !Yref || !Yq) goto done;
+    for (int64_t k = 0; k < K; ++k) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < Mc; ++r) acc += fabs((double)X[r * K + k]);
+        m[k] = acc / (double)Mc;
+    }
+    w4o_gemm(X, W, Mc, N, K, Yref, NULL);
+    int arg = 0;
+    for (int i = 0; i < n_alpha; ++i) {
+        for (int64_t k = 0; k < K; ++k) s[k] = m[k] > 0.0 ? (float)pow(m[k], alphas[i]) : 1.0f;
+        w4o_quantize(W, s, N, K, group, codes, sc, zp);
+        w4o_dequant(codes, sc, zp, s, N, K, group, What);
+        w4o_gemm(X, What, Mc, N, K, Yq, NULL);
+        double e = 0.0;
+        for (int64_t j = 0; j < Mc * N; ++j) {
+            double d = Yref[j] - Yq[j];
+            e += d * d;
+        }
+        errors[i] = e;
+        if (e < errors[arg]) arg = i;
+    }
+    for (int64_t k = 0; k < K; ++k) s_out[k] = m[k] > 0.0 ? (float)pow(m[k], alphas[arg]) : 1.0f;
+    *best = arg;
+    rc = 0;
+done:
+    free(m); free(s); free(codes); free(sc); free(zp); free(What); free(Yref); free(Yq);
+    return rc;
 }

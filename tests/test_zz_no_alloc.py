@@ -53,9 +53,10 @@ def test_static_scratch_matches_workspace_entry(w4, M, N, K, awq):
 
 
 def test_static_scratch_rejects_oversized_plan(w4):
-    """M=64 needs several k-slices, and 64 x 65536 fp32 partials per slice exceed
-    the fixed scratch: rejected on the host with the sizes in the message."""
-    M, N, K = 64, 65536, 4096
+    """M=8 on a wide, deep layer splits K into slices, and its fp32 partials
+    (slices x 2 slots x 8 x 65536 floats) exceed the fixed scratch: rejected on
+    the host with the sizes in the message (buffers are full-size all the same)."""
+    M, N, K = 8, 65536, 8192
     assert w4.w4a16_gemm_workspace_size(M, N, K) > w4.w4a16_gemm_decode_static_capacity()
     X = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
     packed = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
@@ -64,6 +65,8 @@ def test_static_scratch_rejects_oversized_plan(w4):
         w4.w4a16_gemm_decode_static(X, packed, sc, sc)
     assert ei.value.status == w4.W4_ERR_UNSUPPORTED
     assert "static scratch" in str(ei.value)
+    del packed, sc
+    torch.cuda.empty_cache()
 
 
 def test_static_scratch_rejects_prefill_shapes(w4):

@@ -74,7 +74,7 @@ namespace gemv_impl {
 
 constexpr int kRows = 64;      // rows per task
 constexpr int kSG = 4;         // groups per pipeline stage (256 bytes of codes per row)
-constexpr int kNst = 4;        // pipeline stages
+constexpr int kNst = 5;        // pipeline stages (5 x 18 KiB in flight per CTA)
 constexpr int kBox = kRows * 128;          // one 128-byte-swizzled box: 2 groups x 64 rows
 constexpr int kPBytes = 2 * kBox;          // 16 KiB of codes per stage
 constexpr int kSBytes = kRows * 8 * 2;     // 8-group scale (or zero) box per stage
@@ -141,9 +141,16 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t
 // are its (row tile, stage) pairs in tile-major order, T = RT * S of them; CTA
 // c of the slice's C CTAs takes iterations [floor(c T / C), floor((c+1) T / C)).
 // The planner keeps C <= T, so every range is non-empty.
-__device__ __forceinline__ int64_t part_begin(int64_t c, int64_t T, int64_t C) { return (c * T) / C; }
+// (32-bit arithmetic whenever the products fit, which is every realistic layer.)
+__device__ __forceinline__ int64_t part_begin(int64_t c, int64_t T, int64_t C) {
+  if (T * C < (int64_t(1) << 32)) return (int64_t)((uint32_t)(c * T) / (uint32_t)C);
+  return (c * T) / C;
+}
 // The CTA whose range holds iteration i.
-__device__ __forceinline__ int64_t part_owner(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
+__device__ __forceinline__ int64_t part_owner(int64_t i, int64_t T, int64_t C) {
+  if (T * C < (int64_t(1) << 32)) return (int64_t)((uint32_t)((i + 1) * C - 1) / (uint32_t)T);
+  return ((i + 1) * C - 1) / T;
+}
 // Stages of k-slice ks (the last slice may hold fewer groups).
 __device__ __forceinline__ int64_t slice_stages(int ks, int kr, int64_t Kg) {
   const int64_t ng = min((int64_t)kr, Kg - (int64_t)ks * kr);
@@ -193,7 +200,7 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNst; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 2);  // the expect-tx arrival, then the header's
       mbar_init(&empty[s], kComputeWarps);
     }
     for (int b = 0; b < 4; ++b) {
@@ -225,25 +232,10 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         const int c0 = (int)(it - rt * S);
         const int64_t frag_end = min(it1, (rt + 1) * (int64_t)S);
         const int c1 = (int)(frag_end - rt * S);
-        // the fragment's place among the row tile's contributors
         const bool direct = c0 == 0 && c1 == S && p.kslices == 1;
-        int slot = 0, ntotal = 0;
-        if (!direct) {
-          int64_t first, count;
-          tile_owners(rt, RT, C, kslice, p.kr, Kg, first, count);
-          slot = (int)((int64_t)blockIdx.x - first);
-          for (int ks = 0; ks < p.kslices; ++ks) {
-            tile_owners(rt, RT, C, ks, p.kr, Kg, first, count);
-            ntotal += (int)count;
-          }
-        }
         const int32_t row0 = (int32_t)(rt * kRows);
         for (int c = c0; c < c1; ++c) {
           if (!mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) { ok = false; break; }
-          hdr[4 * s + 0] = (int)rt;
-          hdr[4 * s + 1] = c | ((c == c1 - 1) ? (1 << 16) : 0);
-          hdr[4 * s + 2] = slot | (direct ? (1 << 16) : 0);
-          hdr[4 * s + 3] = ntotal;
           uint8_t *st = stages + s * kStage;
           mbar_arrive_expect_tx(&full[s], kScTma ? kStage : kPBytes);
           const int64_t gs = g_first + (int64_t)c * kSG;
@@ -254,6 +246,23 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
             tma_load_2d(st + kPBytes, &tmS, &full[s], gx0, row0);
             tma_load_2d(st + kPBytes + kSBytes, &tmZ, &full[s], gx0, row0);
           }
+          // Header: the fragment's place among the row tile's contributors is only
+          // read at its last stage, so it is worked out after that stage's loads.
+          int slot = 0, ntotal = 0;
+          if (c == c1 - 1 && !direct) {
+            int64_t first, count;
+            tile_owners(rt, RT, C, kslice, p.kr, Kg, first, count);
+            slot = (int)((int64_t)blockIdx.x - first);
+            for (int ks = 0; ks < p.kslices; ++ks) {
+              tile_owners(rt, RT, C, ks, p.kr, Kg, first, count);
+              ntotal += (int)count;
+            }
+          }
+          hdr[4 * s + 0] = (int)rt;
+          hdr[4 * s + 1] = c | ((c == c1 - 1) ? (1 << 16) : 0);
+          hdr[4 * s + 2] = slot | (direct ? (1 << 16) : 0);
+          hdr[4 * s + 3] = ntotal;
+          mbar_arrive(&full[s]);
           if (++s == kNst) {
             s = 0;
             ph ^= 1u;
@@ -262,7 +271,8 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         it = frag_end;
       }
       if (ok && mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) {
-        hdr[4 * s] = -1;  // end of work
+        hdr[4 * s] = -1;  // end of work (no loads: both arrivals here)
+        mbar_arrive(&full[s]);
         mbar_arrive(&full[s]);
       }
       grid_launch_dependents();  // all of this CTA's loads are issued
@@ -280,47 +290,31 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
   const uint16_t *xg = static_cast<const uint16_t *>(p.X);
   const int units = ng * Mi * 4;
   const int units_pad = ng_pad * Mi * 4;
-  // pass 1: per-token max |x * s| over the k-slice -> power-of-two exponent
-  for (int r0 = 0; r0 < units; r0 += kComputeThreads) {
-    const int u = r0 + threadIdx.x;
-    if (u < units) {
-      const int tt = u & 3;
-      const int tok = (u >> 2) % Mi;
-      const int gl = (u >> 2) / Mi;
-      const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
-      const uint4 *src = reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + k0);
-      float mx = 0.0f;
+  // Unit u -> (group gl, token tok, quarter tt); its 32 channels start at k0.
+  auto unit_src = [&](int u) -> const uint4 * {
+    const int tt = u & 3, tok = (u >> 2) % Mi, gl = (u >> 2) / Mi;
+    return reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + (g_first + gl) * kGroup + 32 * tt);
+  };
+  auto unit_max = [&](int u, const uint32_t (&w)[16]) {  // max |x * s| of the unit -> its token's running max
+    const int tt = u & 3, tok = (u >> 2) % Mi, gl = (u >> 2) / Mi;
+    const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
+    float mx = 0.0f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 v = __ldg(src + c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float2 f = pair_to_f32<kBf16>(w[e]);
-          if constexpr (kAwq) {
-            const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 8 * c + 2 * e));
-            f.x *= s2.x;
-            f.y *= s2.y;
-          }
-          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
+    for (int e = 0; e < 16; ++e) {
+      float2 f = pair_to_f32<kBf16>(w[e]);
+      if constexpr (kAwq) {
+        const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 2 * e));
+        f.x *= s2.x;
+        f.y *= s2.y;
       }
-      atomicMax(&xexp[tok], __float_as_int(mx));  // non-negative floats order like their bits
+      mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
     }
-  }
-  named_bar_compute();
-  if (threadIdx.x < Mi) {
-    const int bits = xexp[threadIdx.x];
-    // max|x'| in [2^13, 2^14): e = 13 - floor(log2 max); 0 for an all-zero token
-    const int E = (bits >> 23) & 0xFF;  // biased exponent of the max (finite inputs)
-    int e = (bits == 0) ? 0 : 13 - (E - 127);
-    e = max(-100, min(100, e));
-    xexp[threadIdx.x] = e;
-  }
-  named_bar_compute();
-  // pass 2: x' = x * s * 2^e as fp16 fragments (odd channels / 16), group sums P and S
-  for (int r0 = 0; r0 < units_pad; r0 += kComputeThreads) {
-    const int u = r0 + threadIdx.x;
+    atomicMax(&xexp[tok], __float_as_int(mx));  // non-negative floats order like their bits
+  };
+  // x' = x * s * 2^e as fp16 B fragments (odd channels / 16) plus the group sums P and S.
+  // Every lane of the warp calls this (the shuffles need whole warps); units past
+  // units_pad are idle, and units of the zero padding (gl >= ng) write zeros.
+  auto unit_convert = [&](int u, const uint32_t (&w)[16]) {
     const bool valid = u < units_pad;
     const int tt = u & 3;
     const int tok = valid ? (u >> 2) % Mi : 0;
@@ -335,37 +329,31 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         for (int j = 0; j < 16; ++j) hw[pp][j] = 0u;
       if (real) {
         const int64_t k0 = (g_first + gl) * kGroup + 32 * tt;
-        const uint4 *src = reinterpret_cast<const uint4 *>(xg + (int64_t)tok * K + k0);
         const int e = xexp[tok];
         const float se = exp2i(e), so = exp2i(e - 4);  // even channels x 2^e, odd x 2^(e-4)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v = __ldg(src + c);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            float2 f = pair_to_f32<kBf16>(w[e2]);
-            if constexpr (kAwq) {
-              const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 8 * c + 2 * e2));
-              f.x *= s2.x;
-              f.y *= s2.y;
-            }
-            f.x *= se;  // exact power-of-two scaling
-            f.y *= so;
-            const uint32_t hi = f16x2_bits(f.x, f.y);
-            const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
-            hw[0][4 * c + e2] = hi;
-            float be = hv.x, bo = hv.y;
-            if constexpr (kAwq) {
-              const uint32_t lo = f16x2_bits(f.x - hv.x, f.y - hv.y);
-              const float2 lv = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
-              hw[kParts - 1][4 * c + e2] = lo;
-              be += lv.x;
-              bo += lv.y;
-            }
-            sumB += be + bo;
-            sumX += fmaf(16.0f, bo, be);
+        for (int j = 0; j < 16; ++j) {
+          float2 f = pair_to_f32<kBf16>(w[j]);
+          if constexpr (kAwq) {
+            const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.awq_s + k0 + 2 * j));
+            f.x *= s2.x;
+            f.y *= s2.y;
           }
+          f.x *= se;  // exact power-of-two scaling
+          f.y *= so;
+          const uint32_t hi = f16x2_bits(f.x, f.y);
+          const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+          hw[0][j] = hi;
+          float be = hv.x, bo = hv.y;
+          if constexpr (kAwq) {
+            const uint32_t lo = f16x2_bits(f.x - hv.x, f.y - hv.y);
+            const float2 lv = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+            hw[kParts - 1][j] = lo;
+            be += lv.x;
+            bo += lv.y;
+          }
+          sumB += be + bo;
+          sumX += fmaf(16.0f, bo, be);
         }
       }
       // B fragments for MMA block b = 2i + h: B0 = (v[8i+2h], v[8i+2h+4]), B1 = (v[8i+2h+1], v[8i+2h+5]);
@@ -392,6 +380,57 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
     sumX += __shfl_xor_sync(0xffffffffu, sumX, 1);
     sumX += __shfl_xor_sync(0xffffffffu, sumX, 2);
     if (valid && tt == 0) ps[gl * Mi + tok] = make_float2(1024.0f * sumB, sumX);
+  };
+  auto load_unit = [&](int u, uint32_t (&w)[16]) {
+    const uint4 *src = unit_src(u);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = __ldg(src + c);
+      w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+    }
+  };
+  auto set_exponents = [&]() {
+    named_bar_compute();
+    if (threadIdx.x < Mi) {
+      const int bits = xexp[threadIdx.x];
+      // max|x'| in [2^13, 2^14): e = 13 - floor(log2 max); 0 for an all-zero token
+      const int E = (bits >> 23) & 0xFF;  // biased exponent of the max (finite inputs)
+      int e = (bits == 0) ? 0 : 13 - (E - 127);
+      e = max(-100, min(100, e));
+      xexp[threadIdx.x] = e;
+    }
+    named_bar_compute();
+  };
+  if (!kAwq && units_pad <= 2 * kComputeThreads) {
+    // one read of X: both rounds' words stay in registers across the exponent step
+    uint32_t w0[16], w1[16];
+    const int u0 = threadIdx.x, u1 = kComputeThreads + threadIdx.x;
+    if (u0 < units) { load_unit(u0, w0); unit_max(u0, w0); }
+    if (u1 < units) { load_unit(u1, w1); unit_max(u1, w1); }
+    set_exponents();
+    unit_convert(u0, w0);
+    if (units_pad > kComputeThreads) unit_convert(u1, w1);
+  } else {
+    // pass 1: per-token max over the k-slice; pass 2 reads X again and converts
+    for (int r0 = 0; r0 < units; r0 += kComputeThreads) {
+      const int u = r0 + threadIdx.x;
+      if (u < units) {
+        uint32_t w[16];
+        load_unit(u, w);
+        unit_max(u, w);
+      }
+    }
+    set_exponents();
+    for (int r0 = 0; r0 < units_pad; r0 += kComputeThreads) {
+      const int u = r0 + threadIdx.x;
+      uint32_t w[16];
+      if (u < units) load_unit(u, w);
+      else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) w[j] = 0u;
+      }
+      unit_convert(u, w);
+    }
   }
   named_bar_compute();
 

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -18,12 +19,26 @@
 #include "gemm_tc.cu"
 #include "gemv_mma.cu"
 #include "quantize.cu"
+#include "awq_search.cu"
+#include "outliers.cu"
 #include "w4.h"
 
 namespace w4 {
+cudaError_t launch_mean_abs(const void *X, bool x_bf16, int64_t Mc, int64_t K, double *m, cudaStream_t stream);
+cudaError_t launch_awq_scale(const double *m, int64_t K, double a, float *s, cudaStream_t stream);
+cudaError_t launch_dense_ref(const void *X, bool x_bf16, const float *W, int64_t Mc, int64_t N, int64_t K, float *Y,
+                             cudaStream_t stream);
+cudaError_t launch_sq_err(const float *A, const float *B, int64_t count, double *partial, double *err,
+                          cudaStream_t stream);
 cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, int group,
-                            bool symmetric, uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes,
-                            int sm_count, cudaStream_t stream);
+                            bool symmetric, const uint32_t *tau, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
+                            uint8_t *codes, int sm_count, cudaStream_t stream);
+cudaError_t launch_outlier_threshold(const float *W, int64_t E, int64_t count, uint32_t *state, uint32_t *hist,
+                                     int sm_count, cudaStream_t stream);
+cudaError_t launch_outlier_csr(const float *W, int64_t N, int64_t K, const uint32_t *state, int32_t *counts,
+                               int32_t *row_ptr, int64_t cap, int32_t *col, uint16_t *val, cudaStream_t stream);
+cudaError_t launch_sparse_add(const void *X, bool x_bf16, int64_t M, int64_t N, int64_t K, const int32_t *row_ptr,
+                              const int32_t *col, const uint16_t *val, void *Y, bool y_bf16, cudaStream_t stream);
 cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,
                         cudaStream_t stream);
 }  // namespace w4
@@ -140,11 +155,34 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   // activations fit the staging budget (every CTA stages its whole k-slice).
   // The static partition balances the work across CTAs, so K is split only
   // when the activations do not fit.
-  int64_t kr = std::min<int64_t>(cdiv(Kg, 4) * 4, 4096);
-  while (kr > 4 && w4::gemv_xs_bytes((int)kr, M, awq) > kGemvXsMax) kr -= 4;
+  int64_t kr_max = std::min<int64_t>(cdiv(Kg, 4) * 4, 4096);
+  while (kr_max > 4 && w4::gemv_xs_bytes((int)kr_max, M, awq) > kGemvXsMax) kr_max -= 4;
+  const int64_t ks0 = cdiv(Kg, kr_max);
+  // balanced slices: the shortest slice length (whole stages) that gives ks slices
+  auto kr_for = [&](int64_t ks) { return cdiv(cdiv(Kg, ks), 4) * 4; };
+  auto slots_for = [&](int64_t kr_c) {
+    return (int64_t)sm * gemv_ctas_per_sm(w4::gemv_xs_bytes((int)kr_c, M, awq), p.t8);
+  };
+  int64_t kr = kr_for(ks0);
+  int64_t C = -1;
+  if (RT * ks0 <= slots_for(kr)) {
+    // Few row tiles: one whole tile per CTA (no tile is shared, outputs written
+    // directly when K is not split), with K split into the most slices that keep
+    // RT * slices CTAs resident and at least 6 stages per slice.
+    for (int64_t ks = ks0 + 1;; ++ks) {
+      const int64_t kr_c = kr_for(ks);
+      if (cdiv(Kg, kr_c) != ks) {
+        if (kr_c <= 4) break;
+        continue;
+      }
+      if (kr_c / 4 < 6 || RT * ks > slots_for(kr_c)) break;
+      kr = kr_c;
+    }
+    C = RT;
+  }
   if (const char *e = getenv("W4_GEMV_KR")) {  // tuning override
     const int64_t v = atoi(e);
-    if (v >= 4 && v % 4 == 0 && v <= kr) kr = v;
+    if (v >= 4 && v % 4 == 0 && v <= kr_max) kr = v;
   }
   int64_t ks = cdiv(Kg, kr);
   p.kr = (int)kr;
@@ -153,8 +191,8 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   // stages per row tile: S_full for every k-slice but the last, S_last for the last
   const int64_t S_full = kr / 4;
   const int64_t S_last = cdiv(Kg - (ks - 1) * kr, 4);
-  const int64_t slots = (int64_t)sm * gemv_ctas_per_sm(p.xs_bytes, p.t8);
-  int64_t C = std::max<int64_t>(1, slots / ks);
+  const int64_t slots = slots_for(kr);
+  if (C < 0) C = std::max<int64_t>(1, slots / ks);  // many row tiles: balanced partition
   if (const char *e = getenv("W4_GEMV_GX")) {  // tuning override
     const int v = atoi(e);
     if (v >= 1) C = v;
@@ -201,8 +239,11 @@ GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, int sm) {
   return p;
 }
 
+// Measured on B200 (8B layer shapes): the decode kernel wins up to M = 8; from
+// M = 16 on, the tensor-core kernel is faster at every shape (its dequant is
+// amortized over the token tile, while the decode kernel's k-slices shrink with M).
 bool gemv_fits(int64_t M, int64_t N, bool awq) {
-  return w4::gemv_supports(M, awq);
+  return M <= 8 && w4::gemv_supports(M, awq);
 }
 
 GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
@@ -290,7 +331,7 @@ w4_status quantize_common(const void *W, w4_dtype w_dtype, const float *awq_s, i
   int sm = 0;
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
-  e = w4::launch_quantize(W, (int)w_dtype, awq_s, N, K, group, symmetric, packed, scales, zeros, codes, sm,
+  e = w4::launch_quantize(W, (int)w_dtype, awq_s, N, K, group, symmetric, nullptr, packed, scales, zeros, codes, sm,
                           reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return W4_OK;
@@ -564,6 +605,188 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
   if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
   return w4a16_gemm(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, scratch,
                     kStaticScratchBytes, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// AWQ scale search (offline): see awq_search.cu for the method and include/w4.h
+// for the contract.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kMaxAlphas = 256;
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct SearchLayout {
+  size_t gemm_ws, packed, scales, zeros, s, m, yref, yq, partial, errs, total;
+};
+
+SearchLayout search_layout(int64_t Mc, int64_t N, int64_t K, int group, int sm) {
+  SearchLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const size_t gws = std::max<size_t>(ws_size_all(Mc, N, K, sm), 256);
+  L.gemm_ws = take(gws);
+  L.packed = take((size_t)N * K / 2);
+  L.scales = take((size_t)N * (K / group) * 2);
+  L.zeros = take((size_t)N * (K / group) * 2);
+  L.s = take((size_t)K * 4);
+  L.m = take((size_t)K * 8);
+  L.yref = take((size_t)Mc * N * 4);
+  L.yq = take((size_t)Mc * N * 4);
+  L.partial = take(256 * 8);
+  L.errs = take(kMaxAlphas * 8);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4_awq_search_workspace_size(int64_t Mc, int64_t N, int64_t K, int group) {
+  if (Mc < 1 || N < 1 || K < 1 || group < 1 || K % group != 0) return 0;
+  int sm = 0;
+  if (current_sm_count(&sm) != cudaSuccess) sm = 148;
+  return search_layout(Mc, N, K, group, sm).total;
+}
+
+w4_status w4_awq_search(const float *W, int64_t N, int64_t K, int group, const void *Xcal, w4_dtype x_dtype,
+                        int64_t Mc, const float *alphas, int n_alpha, float *awq_s, double *errors, int *best,
+                        void *workspace, size_t workspace_bytes, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(Mc, N, K, group);
+  if (st != W4_OK) return st;
+  if (x_dtype != W4_F16 && x_dtype != W4_BF16) return fail(W4_ERR_UNSUPPORTED, "calibration dtype must be F16 or BF16");
+  if (group != w4::kGroup && K % 64 != 0)
+    return fail(W4_ERR_UNSUPPORTED, "group=%d needs K a multiple of 64 (K=%lld)", group, (long long)K);
+  if (n_alpha < 1 || n_alpha > kMaxAlphas || !alphas)
+    return fail(W4_ERR_INVALID_ARG, "need 1..%d exponents (got %d)", kMaxAlphas, n_alpha);
+  for (int i = 0; i < n_alpha; ++i)
+    if (!std::isfinite(alphas[i])) return fail(W4_ERR_INVALID_ARG, "exponent %d is not finite", i);
+  if (!W || !Xcal || !awq_s || !best || !workspace) return fail(W4_ERR_INVALID_ARG, "null W, Xcal, awq_s, best or workspace");
+  if (!aligned16(W) || !aligned16(Xcal) || !aligned16(awq_s) || !aligned16(workspace))
+    return fail(W4_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const SearchLayout L = search_layout(Mc, N, K, group, sm);
+  if (workspace_bytes < L.total)
+    return fail(W4_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", L.total, workspace_bytes);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint8_t *packed = ws + L.packed;
+  uint16_t *scales = reinterpret_cast<uint16_t *>(ws + L.scales);
+  uint16_t *zeros = reinterpret_cast<uint16_t *>(ws + L.zeros);
+  float *s = reinterpret_cast<float *>(ws + L.s);
+  double *m = reinterpret_cast<double *>(ws + L.m);
+  float *yref = reinterpret_cast<float *>(ws + L.yref);
+  float *yq = reinterpret_cast<float *>(ws + L.yq);
+  double *partial = reinterpret_cast<double *>(ws + L.partial);
+  double *errs = reinterpret_cast<double *>(ws + L.errs);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const bool xbf16 = x_dtype == W4_BF16;
+
+  if ((e = w4::launch_mean_abs(Xcal, xbf16, Mc, K, m, cs)) != cudaSuccess) return cuda_fail(e, "activation magnitude");
+  if ((e = w4::launch_dense_ref(Xcal, xbf16, W, Mc, N, K, yref, cs)) != cudaSuccess) return cuda_fail(e, "reference GEMM");
+  for (int i = 0; i < n_alpha; ++i) {
+    if ((e = w4::launch_awq_scale(m, K, (double)alphas[i], s, cs)) != cudaSuccess) return cuda_fail(e, "scale");
+    st = quantize_common(W, W4_F32, s, N, K, group, false, packed, scales, zeros, nullptr, stream);
+    if (st != W4_OK) return st;
+    st = w4a16_gemm(Xcal, x_dtype, Mc, N, K, group, packed, scales, zeros, s, yq, W4_F32, ws + L.gemm_ws,
+                    L.packed - L.gemm_ws, stream);
+    if (st != W4_OK) return st;
+    if ((e = w4::launch_sq_err(yref, yq, Mc * N, partial, errs + i, cs)) != cudaSuccess) return cuda_fail(e, "error sum");
+  }
+  double host_errs[kMaxAlphas];
+  if ((e = cudaMemcpyAsync(host_errs, errs, sizeof(double) * n_alpha, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+    return cuda_fail(e, "copy errors");
+  if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int arg = 0;
+  for (int i = 1; i < n_alpha; ++i)
+    if (host_errs[i] < host_errs[arg]) arg = i;
+  if ((e = w4::launch_awq_scale(m, K, (double)alphas[arg], awq_s, cs)) != cudaSuccess) return cuda_fail(e, "scale");
+  if (errors)
+    for (int i = 0; i < n_alpha; ++i) errors[i] = host_errs[i];
+  *best = arg;
+  return W4_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Dense + sparse split: see outliers.cu for the method, include/w4.h for the contract.
+// ---------------------------------------------------------------------------
+extern "C" {
+
+size_t w4_outliers_workspace_size(int64_t N) {
+  if (N < 1) return 0;
+  return 256 + 2048 * 4 + (size_t)((N * 4 + 255) / 256) * 256;
+}
+
+w4_status w4_quantize_outliers(const float *W, const float *awq_s, int64_t N, int64_t K, int group, int64_t count,
+                               uint8_t *packed, uint16_t *scales, uint16_t *zeros, int32_t *row_ptr, int32_t *col,
+                               uint16_t *val, int64_t capacity, int64_t *nnz, void *workspace,
+                               size_t workspace_bytes, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(1, N, K, group);
+  if (st != W4_OK) return st;
+  if (count < 1 || count > N * K) return fail(W4_ERR_INVALID_ARG, "outlier count %lld not in [1, N*K]", (long long)count);
+  if (N * K > INT32_MAX) return fail(W4_ERR_UNSUPPORTED, "N*K must fit in 31 bits for the CSR indices");
+  if (!W || !packed || !scales || !zeros || !row_ptr || !col || !val || !nnz || !workspace)
+    return fail(W4_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros) || !aligned16(row_ptr) ||
+      !aligned16(col) || !aligned16(val) || !aligned16(workspace) || (awq_s && !aligned16(awq_s)))
+    return fail(W4_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (workspace_bytes < w4_outliers_workspace_size(N))
+    return fail(W4_ERR_INVALID_ARG, "workspace too small: need %zu bytes", w4_outliers_workspace_size(N));
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint32_t *state = reinterpret_cast<uint32_t *>(ws);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(ws + 256);
+  int32_t *counts = reinterpret_cast<int32_t *>(ws + 256 + 2048 * 4);
+  if ((e = w4::launch_outlier_threshold(W, N * K, count, state, hist, sm, cs)) != cudaSuccess)
+    return cuda_fail(e, "outlier threshold");
+  if ((e = w4::launch_quantize(W, 0, awq_s, N, K, group, false, state, packed, scales, zeros, nullptr, sm, cs)) !=
+      cudaSuccess)
+    return cuda_fail(e, "quantize launch");
+  if ((e = w4::launch_outlier_csr(W, N, K, state, counts, row_ptr, capacity, col, val, cs)) != cudaSuccess)
+    return cuda_fail(e, "outlier CSR");
+  int32_t total = 0;
+  if ((e = cudaMemcpyAsync(&total, row_ptr + N, sizeof total, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+    return cuda_fail(e, "copy entry count");
+  if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  *nnz = total;
+  if (total > capacity)
+    return fail(W4_ERR_INVALID_ARG, "outlier capacity %lld below the %d entries found (ties at the threshold)",
+                (long long)capacity, total);
+  return W4_OK;
+}
+
+w4_status w4a16_gemm_outliers(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
+                              const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros,
+                              const float *awq_s, const int32_t *row_ptr, const int32_t *col, const uint16_t *val,
+                              void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                              w4_stream_t stream) {
+  if (!row_ptr || !col || !val) {
+    t_last_error.clear();
+    return fail(W4_ERR_INVALID_ARG, "null CSR pointer");
+  }
+  w4_status st = w4a16_gemm(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, workspace,
+                            workspace_bytes, stream);
+  if (st != W4_OK) return st;
+  cudaError_t e = w4::launch_sparse_add(X, x_dtype == W4_BF16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sparse add");
+  return W4_OK;
 }
 
 }  // extern "C"

@@ -61,6 +61,7 @@ constexpr int kQuantUnroll = 4;  // 128-element chunks in flight per warp
 template <typename TW, bool kAwq, bool kCodes, bool kSym>
 __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W, const float *__restrict__ awq_s,
                                                        int64_t E, int64_t K, int group,
+                                                       const uint32_t *__restrict__ outlier_tau,
                                                        uint8_t *__restrict__ packed, uint16_t *__restrict__ scales,
                                                        uint16_t *__restrict__ zeros, uint8_t *__restrict__ codes) {
   const int lane = threadIdx.x & 31;
@@ -68,6 +69,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int64_t chunks = (E + 127) / 128;
   const int lg = group >> 2;  // lanes per group
+  // dense part of a dense + sparse split: weights with |w| >= tau count as 0 here
+  const uint32_t tau = outlier_tau ? *outlier_tau : 0xFFFFFFFFu;
 
   for (int64_t base = warp * kQuantUnroll; base < chunks; base += nwarps * kQuantUnroll) {
     float v[kQuantUnroll][4];
@@ -76,6 +79,9 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
       const int64_t e = (base + u) * 128 + lane * 4;
       if (e < E) {
         Load4<TW>::run(W + e, v[u]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((__float_as_uint(v[u][j]) & 0x7FFFFFFFu) >= tau) v[u][j] = 0.0f;
         if (kAwq) {
           const int64_t k = e % K;
           const float4 s = __ldg(reinterpret_cast<const float4 *>(awq_s + k));
@@ -173,49 +179,53 @@ int grid_for(int64_t work_items, int items_per_block, int sm_count, int blocks_p
 }
 
 template <typename TW, bool kSym>
-cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, int group, uint8_t *packed,
-                              uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
-                              cudaStream_t stream) {
+cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, int group,
+                              const uint32_t *tau, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
+                              uint8_t *codes, int sm_count, cudaStream_t stream) {
   const int64_t E = N * K;
   const int64_t chunks = (E + 127) / 128;
   const int grid = grid_for(chunks, 8 * kQuantUnroll, sm_count, 8);
   const TW *w = static_cast<const TW *>(W);
   if (awq_s) {
     if (codes)
-      quantize_kernel<TW, true, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
+      quantize_kernel<TW, true, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
     else
-      quantize_kernel<TW, true, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
+      quantize_kernel<TW, true, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
   } else {
     if (codes)
-      quantize_kernel<TW, false, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
+      quantize_kernel<TW, false, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
     else
-      quantize_kernel<TW, false, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, packed, scales, zeros, codes);
+      quantize_kernel<TW, false, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
   }
   return cudaGetLastError();
 }
 
 template <bool kSym>
 cudaError_t launch_quantize_s(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, int group,
-                              uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
-                              cudaStream_t stream) {
+                              const uint32_t *tau, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
+                              uint8_t *codes, int sm_count, cudaStream_t stream) {
   switch (dtype) {
-    case 0: return launch_quantize_t<float, kSym>(W, awq_s, N, K, group, packed, scales, zeros, codes, sm_count, stream);
-    case 1: return launch_quantize_t<__half, kSym>(W, awq_s, N, K, group, packed, scales, zeros, codes, sm_count, stream);
+    case 0:
+      return launch_quantize_t<float, kSym>(W, awq_s, N, K, group, tau, packed, scales, zeros, codes, sm_count, stream);
+    case 1:
+      return launch_quantize_t<__half, kSym>(W, awq_s, N, K, group, tau, packed, scales, zeros, codes, sm_count, stream);
     default:
-      return launch_quantize_t<__nv_bfloat16, kSym>(W, awq_s, N, K, group, packed, scales, zeros, codes, sm_count, stream);
+      return launch_quantize_t<__nv_bfloat16, kSym>(W, awq_s, N, K, group, tau, packed, scales, zeros, codes, sm_count,
+                                                    stream);
   }
 }
 
 }  // namespace quant_impl
 
 // dtype: 0 = fp32, 1 = fp16, 2 = bf16; group 32, 64 or 128; symmetric selects the {-7..7} variant
+// tau: device pointer to the outlier threshold (bits of |w|), or NULL for none.
 cudaError_t launch_quantize(const void *W, int dtype, const float *awq_s, int64_t N, int64_t K, int group,
-                            bool symmetric, uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes,
-                            int sm_count, cudaStream_t stream) {
-  return symmetric ? quant_impl::launch_quantize_s<true>(W, dtype, awq_s, N, K, group, packed, scales, zeros, codes,
-                                                         sm_count, stream)
-                   : quant_impl::launch_quantize_s<false>(W, dtype, awq_s, N, K, group, packed, scales, zeros, codes,
-                                                          sm_count, stream);
+                            bool symmetric, const uint32_t *tau, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
+                            uint8_t *codes, int sm_count, cudaStream_t stream) {
+  return symmetric ? quant_impl::launch_quantize_s<true>(W, dtype, awq_s, N, K, group, tau, packed, scales, zeros,
+                                                         codes, sm_count, stream)
+                   : quant_impl::launch_quantize_s<false>(W, dtype, awq_s, N, K, group, tau, packed, scales, zeros,
+                                                          codes, sm_count, stream);
 }
 
 cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,

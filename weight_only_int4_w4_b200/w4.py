@@ -34,13 +34,17 @@ _lib.w4a16_gemm_decode_static.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ct
                                           ctypes.c_int, _P]
 _lib.w4a16_gemm_decode_static_capacity.argtypes = []
 _lib.w4a16_gemm_decode_static_capacity.restype = _SZ
+_lib.w4_awq_search.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _P, _P,
+                               _P, _SZ, _P]
+_lib.w4_awq_search_workspace_size.argtypes = [_I64, _I64, _I64, ctypes.c_int]
+_lib.w4_awq_search_workspace_size.restype = _SZ
 _lib.w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
 _lib.w4a16_gemm_workspace_size.restype = _SZ
 _lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
 _lib.w4_status_string.argtypes = [ctypes.c_int]
 _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
-for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
+for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_awq_search", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -178,6 +182,27 @@ def w4a16_gemm_decode_static(X: torch.Tensor, packed: torch.Tensor, scales: torc
 
 def w4a16_gemm_decode_static_capacity() -> int:
     return int(_lib.w4a16_gemm_decode_static_capacity())
+
+
+AWQ_EXPONENTS = tuple(round(-1.0 + 0.1 * i, 1) for i in range(21))  # -1.0, -0.9, ..., 1.0
+
+
+def w4_awq_search(W: torch.Tensor, Xcal: torch.Tensor, alphas=AWQ_EXPONENTS, group: int = GROUP, stream=None):
+    """AWQ exponent search on calibration activations.  W [N,K] fp32, Xcal [Mc,K] f16/bf16 (CUDA).
+    Returns (awq_s fp32 [K] on the device, best exponent, errors list)."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    assert Xcal.is_cuda and Xcal.dtype in (torch.float16, torch.bfloat16) and Xcal.is_contiguous()
+    N, K = W.shape
+    Mc = Xcal.shape[0]
+    a = (ctypes.c_float * len(alphas))(*alphas)
+    errs = (ctypes.c_double * len(alphas))()
+    best = ctypes.c_int(-1)
+    s = torch.empty(K, dtype=torch.float32, device=W.device)
+    ws = torch.zeros(int(_lib.w4_awq_search_workspace_size(Mc, N, K, group)), dtype=torch.uint8, device=W.device)
+    _check(_lib.w4_awq_search(_ptr(W), N, K, group, _ptr(Xcal), _DT[Xcal.dtype], Mc, ctypes.cast(a, _P), len(alphas),
+                              _ptr(s), ctypes.cast(errs, _P), ctypes.cast(ctypes.pointer(best), _P), _ptr(ws),
+                              ws.numel(), _stream(stream)), "w4_awq_search")
+    return s, alphas[best.value], list(errs)
 
 
 def w4_device_error() -> int:
