@@ -466,6 +466,40 @@ def stack70b_leg(w4, replays=3):
     return out
 
 
+def outlier_leg(w4, launches=60):
+    """Decode GEMM with the dense + sparse outlier split (0.1% of the weights in fp16 CSR) on the
+    Llama-3-8B gate_up shape at M=1, three weight copies rotated (188 MB > L2), in one CUDA graph."""
+    dev = torch.device("cuda")
+    K, N = synthetic.SHAPES_8B["gate_up"]
+    gen = torch.Generator(device=dev)
+    copies = []
+    for c in range(3):
+        gen.manual_seed(synthetic.seed_of("bench", "outliers", c) % (2 ** 62))
+        W = torch.randn((N, K), generator=gen, device=dev) * 0.02
+        mask = torch.rand((N, K), generator=gen, device=dev) < 0.001
+        W = torch.where(mask, torch.randn((N, K), generator=gen, device=dev) * synthetic.OUTLIER_STD, W)
+        copies.append(w4.w4_quantize_outliers(W))
+        del W, mask
+    X = torch.randn((1, K), generator=gen, device=dev).to(torch.bfloat16)
+    Y = torch.empty((1, N), dtype=torch.float32, device=dev)
+    ws = w4.workspace(1, N, K, dev)
+    stream = torch.cuda.Stream()
+    res = {}
+    for name, fn in (("plain", lambda i: w4.w4a16_gemm(X, *copies[i % 3][:3], out=Y, ws=ws)),
+                     ("with_outliers", lambda i: w4.w4a16_gemm_outliers(X, *copies[i % 3], out=Y, ws=ws))):
+        g = _graph_of(fn, launches, 3, stream)
+        res[name] = _replay_timed(g, stream) / launches * 1e3
+        del g
+    row_ptr, col, val = copies[0][3]
+    nbytes = gemm_bytes(1, N, K) + (N + 1) * 4 + col.numel() * 6
+    out = {"us_per_call": round(res["with_outliers"], 3), "us_per_call_dense_only": round(res["plain"], 3),
+           "GB/s": round(nbytes / (res["with_outliers"] * 1e-6) / 1e9, 1), "nnz": int(col.numel()),
+           "workload": "gate_up 4096->28672, M=1, 0.1% of W in fp16 CSR (N(0,0.02) W with 0.1% N(0,0.4) outliers)"}
+    del copies
+    torch.cuda.empty_cache()
+    return out
+
+
 def awq_search_leg(w4, repeats=3):
     """AWQ exponent search on the Llama-3-8B gate_up weights with a 512-row calibration batch
     (1% of the channels x10), 21 exponents in [-1, 1]: device time per search."""
@@ -539,6 +573,7 @@ def main():
         pf, pf_all, pf_ms = prefill_leg(w4)
         extras["stack70b"] = stack70b_leg(w4)
         extras["awq_search"] = awq_search_leg(w4)
+        extras["outliers"] = outlier_leg(w4)
         extras["prefill"] = {"value": round(pf_all, 1), "unit": "TFLOP/s", "ms_per_step": round(pf_ms, 3),
                              "workload": "Llama-3-70B qkv/o_proj/gate_up/down, M=8192, bf16 X",
                              "per_layer_tflops": pf,

@@ -188,6 +188,50 @@ size_t w4_awq_search_workspace_size(int64_t Mc, int64_t N, int64_t K,
                                     int group);
 
 /*
+ * Dense + sparse split (mhpq.cn practitioner's article, section 2.2: the top
+ * 0.1% of weights by magnitude stay in FP16, the rest go to INT4).  The sparse
+ * part holds every weight with |w| >= tau, tau = the count-th largest |w| of the
+ * matrix (ties at tau are all kept), as fp16.  The dense part is quantized as
+ * by w4_quantize with those weights taken as 0, so their dequantized value is
+ * exactly 0 and  W^ = dequant(dense) + sparse.
+ *   W         device [N][K] fp32 (N*K < 2^31)
+ *   awq_s, group, packed, scales, zeros   as for w4_quantize
+ *   count     1 <= count <= N*K (for 0.1%: ceil(0.001 * N * K))
+ *   row_ptr   device [N+1] int32 out: CSR row offsets by output row
+ *   col, val  device [capacity] int32 / fp16 bit patterns out: the entries of
+ *             each row in increasing k
+ *   nnz       HOST out: entries found (count, more with ties at tau)
+ *   workspace device, w4_outliers_workspace_size(N) bytes, zero-filled before
+ *             its first use (every call leaves it so)
+ * If capacity < nnz, returns W4_ERR_INVALID_ARG with nnz set (col / val then
+ * hold the first `capacity` entries).  Synchronizes `stream`.
+ */
+w4_status w4_quantize_outliers(const float *W, const float *awq_s, int64_t N,
+                               int64_t K, int group, int64_t count,
+                               uint8_t *packed, uint16_t *scales,
+                               uint16_t *zeros, int32_t *row_ptr,
+                               int32_t *col, uint16_t *val, int64_t capacity,
+                               int64_t *nnz, void *workspace,
+                               size_t workspace_bytes, w4_stream_t stream);
+
+/* Bytes of workspace w4_quantize_outliers needs for N rows. */
+size_t w4_outliers_workspace_size(int64_t N);
+
+/*
+ * w4a16_gemm on the dense part, then the sparse part added to Y:
+ * y[m][n] += sum over row n's entries of x[m][col] * val (fp32, entry order).
+ * Arguments as for w4a16_gemm, plus the CSR from w4_quantize_outliers.
+ */
+w4_status w4a16_gemm_outliers(const void *X, w4_dtype x_dtype, int64_t M,
+                              int64_t N, int64_t K, int group,
+                              const uint8_t *packed, const uint16_t *scales,
+                              const uint16_t *zeros, const float *awq_s,
+                              const int32_t *row_ptr, const int32_t *col,
+                              const uint16_t *val, void *Y, w4_dtype y_dtype,
+                              void *workspace, size_t workspace_bytes,
+                              w4_stream_t stream);
+
+/*
  * Decode GEMM with library-owned scratch: the same computation, kernel and
  * result as w4a16_gemm for decode shapes, with no workspace argument.  The
  * source pages have no counterpart to this call; it exists for callers that

@@ -105,6 +105,33 @@ def awq_search(W, X, alphas, group: int = 128):
     return errors, s, best.value
 
 
+def outlier_split(W, count, awq_s=None, group: int = 128):
+    """Dense + sparse split (mhpq.cn article, section 2.2): every weight with |w| >= tau, tau the
+    count-th largest |w| (ties all kept), goes to an fp16 sparse part; the rest is quantized with
+    those weights taken as 0.  Plain numpy selection (full sort) and the C quantizer.
+    Returns (codes, scales, zeros, row_ptr int32 [N+1], col int32 [nnz], val fp16 [nnz])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    mag = np.abs(W)
+    tau = np.sort(mag, axis=None)[::-1][count - 1]
+    mask = mag >= tau
+    codes, scales, zeros = quantize(np.where(mask, np.float32(0.0), W), awq_s, group)
+    rows, cols = np.nonzero(mask)  # row-major: increasing k within each row
+    row_ptr = np.zeros(N + 1, np.int64)
+    np.add.at(row_ptr, rows + 1, 1)
+    row_ptr = np.cumsum(row_ptr).astype(np.int32)
+    return codes, scales, zeros, row_ptr, cols.astype(np.int32), W[rows, cols].astype(np.float16)
+
+
+def outlier_dequant(codes, scales, zeros, row_ptr, col, val, awq_s=None, group: int = 128):
+    """W^ = dequant(dense) + sparse: the fp16 entries added at their positions."""
+    What = dequant(codes, scales, zeros, awq_s, group)
+    N = What.shape[0]
+    rows = np.repeat(np.arange(N), np.diff(row_ptr.astype(np.int64)))
+    What[rows, col] += val.astype(np.float32)
+    return What
+
+
 def pack(codes):
     codes = _c(codes, np.uint8)
     N, K = codes.shape

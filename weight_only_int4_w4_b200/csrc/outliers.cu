@@ -3,7 +3,7 @@
 // the rest are quantized to INT4, W^ = where(mask, fp16(w), int4 dequant)).
 //
 //   * Threshold: tau = the k-th largest |w| over the whole matrix, found by a
-//     three-pass radix select on the bits of |w| (11 + 11 + 10 bits; for
+//     three-pass radix select on the 31 bits of |w| (11 + 11 + 9; for
 //     non-negative floats the bit patterns order like the values).  The mask is
 //     |w| >= tau, so ties at tau are all kept.
 //   * The dense part is quantized with the masked weights replaced by 0 (see
@@ -23,6 +23,14 @@ constexpr int kBins = 2048;  // per radix pass
 // rank still wanted among the elements matching that prefix (1-based),
 // state[2] = how many bits are fixed.
 __device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+__global__ void state_init_kernel(uint32_t *state, uint32_t count) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    state[0] = 0u;
+    state[1] = count;
+    state[2] = 0u;
+  }
+}
 
 // Histogram of the next `width` bits below the fixed prefix, over elements that match it.
 __global__ void __launch_bounds__(256) radix_hist_kernel(const float *__restrict__ W, int64_t E,
@@ -159,13 +167,11 @@ __global__ void __launch_bounds__(256) sparse_add_kernel(const uint16_t *__restr
 }  // namespace outlier_impl
 
 // tau of the `count`-th largest |w| (count >= 1) into state[0] (as |w| bits).
-// state: 3 uint32; hist: 2048 uint32, both zero-filled beforehand (hist is left zeroed).
+// state: 3 uint32, set here; hist: 2048 uint32, zero-filled beforehand and left zeroed.
 cudaError_t launch_outlier_threshold(const float *W, int64_t E, int64_t count, uint32_t *state, uint32_t *hist,
                                      int sm_count, cudaStream_t stream) {
   using namespace outlier_impl;
-  const uint32_t init[3] = {0u, (uint32_t)count, 0u};
-  cudaError_t e = cudaMemcpyAsync(state, init, sizeof init, cudaMemcpyHostToDevice, stream);
-  if (e != cudaSuccess) return e;
+  state_init_kernel<<<1, 32, 0, stream>>>(state, (uint32_t)count);
   const int widths[3] = {11, 11, 9};  // bits 30..0 of |w|
   int64_t blocks = (E + 255) / 256;
   if (blocks > (int64_t)sm_count * 8) blocks = (int64_t)sm_count * 8;

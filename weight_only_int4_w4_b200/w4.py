@@ -38,13 +38,20 @@ _lib.w4_awq_search.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, ctypes.c_int, _
                                _P, _SZ, _P]
 _lib.w4_awq_search_workspace_size.argtypes = [_I64, _I64, _I64, ctypes.c_int]
 _lib.w4_awq_search_workspace_size.restype = _SZ
+_lib.w4_quantize_outliers.argtypes = [_P, _P, _I64, _I64, ctypes.c_int, _I64, _P, _P, _P, _P, _P, _P, _I64, _P, _P,
+                                      _SZ, _P]
+_lib.w4_outliers_workspace_size.argtypes = [_I64]
+_lib.w4_outliers_workspace_size.restype = _SZ
+_lib.w4a16_gemm_outliers.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P,
+                                     _P, ctypes.c_int, _P, _SZ, _P]
 _lib.w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
 _lib.w4a16_gemm_workspace_size.restype = _SZ
 _lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
 _lib.w4_status_string.argtypes = [ctypes.c_int]
 _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
-for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_awq_search", "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
+for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_awq_search", "w4_quantize_outliers", "w4a16_gemm_outliers",
+           "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -182,6 +189,53 @@ def w4a16_gemm_decode_static(X: torch.Tensor, packed: torch.Tensor, scales: torc
 
 def w4a16_gemm_decode_static_capacity() -> int:
     return int(_lib.w4a16_gemm_decode_static_capacity())
+
+
+def w4_quantize_outliers(W: torch.Tensor, count: int | None = None, awq_s: torch.Tensor | None = None,
+                         group: int = GROUP, stream=None):
+    """Dense + sparse split of W [N,K] fp32 (CUDA): the `count` largest |w| (default 0.1%) in fp16 CSR,
+    the rest quantized.  Returns (packed, scales, zeros, (row_ptr, col, val))."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    N, K = W.shape
+    dev = W.device
+    count = max(1, -(-N * K // 1000)) if count is None else int(count)
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    zeros = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    ws = torch.zeros(int(_lib.w4_outliers_workspace_size(N)), dtype=torch.uint8, device=dev)
+    cap = count + 1024
+    while True:
+        col = torch.empty(cap, dtype=torch.int32, device=dev)
+        val = torch.empty(cap, dtype=torch.float16, device=dev)
+        nnz = ctypes.c_int64(0)
+        st = _lib.w4_quantize_outliers(_ptr(W), _ptr(awq_s), N, K, group, count, _ptr(packed), _ptr(scales),
+                                       _ptr(zeros), _ptr(row_ptr), _ptr(col), _ptr(val), cap,
+                                       ctypes.cast(ctypes.pointer(nnz), _P), _ptr(ws), ws.numel(), _stream(stream))
+        if st == W4_ERR_INVALID_ARG and nnz.value > cap:
+            cap = nnz.value
+            continue
+        _check(st, "w4_quantize_outliers")
+        break
+    return packed, scales, zeros, (row_ptr, col[: nnz.value], val[: nnz.value])
+
+
+def w4a16_gemm_outliers(X: torch.Tensor, packed, scales, zeros, csr, awq_s=None, out_dtype=torch.float32,
+                        out: torch.Tensor | None = None, ws: torch.Tensor | None = None, group: int = GROUP,
+                        stream=None) -> torch.Tensor:
+    """Y = X . (dequant(dense) + sparse)^T with the CSR from w4_quantize_outliers."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.dtype in (torch.float16, torch.bfloat16)
+    M, K = X.shape
+    N = packed.shape[0]
+    row_ptr, col, val = csr
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    if ws is None:
+        ws = workspace(M, N, K, X.device, stream)
+    _check(_lib.w4a16_gemm_outliers(_ptr(X), _DT[X.dtype], M, N, K, group, _ptr(packed), _ptr(scales), _ptr(zeros),
+                                    _ptr(awq_s), _ptr(row_ptr), _ptr(col), _ptr(val), _ptr(out), _DT[out.dtype],
+                                    _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)), "w4a16_gemm_outliers")
+    return out
 
 
 AWQ_EXPONENTS = tuple(round(-1.0 + 0.1 * i, 1) for i in range(21))  # -1.0, -0.9, ..., 1.0
