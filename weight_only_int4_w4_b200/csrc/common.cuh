@@ -6,6 +6,7 @@
 // library's device error word and returns false instead of spinning forever.
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -255,6 +256,24 @@ __device__ __forceinline__ float2 lds_f2(uint32_t a) {
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t b) {
   return __half2float(__ushort_as_half(b));
+}
+
+// Dynamic shared memory above 48 KiB needs a per-function attribute on every
+// device; setting it is a driver call, so it is made once per (function, device)
+// and size, tracked in `set` (one slot per device ordinal).
+constexpr int kAttrDevices = 64;
+inline cudaError_t ensure_smem_attr(const void *func, int bytes, std::atomic<int> *set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kAttrDevices && set[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kAttrDevices) {
+    int cur = set[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !set[dev].compare_exchange_weak(cur, bytes)) {
+    }
+  }
+  return e;
 }
 
 }  // namespace w4

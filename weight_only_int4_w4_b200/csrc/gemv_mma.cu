@@ -771,7 +771,8 @@ cudaError_t launch_t(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUten
                      cudaStream_t stream) {
   auto kern = gemv_kernel<T8, kBf16, kAwq, kScTma>;
   const int smem = smem_bytes_for(p.xs_bytes, T8);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<int> smem_set[kAttrDevices];  // largest size already set, per device
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), smem, smem_set);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.grid_x, (unsigned)p.kslices);

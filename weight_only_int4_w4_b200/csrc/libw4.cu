@@ -100,6 +100,50 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// A 2-D tensor map is a pure function of its data type, address, sizes, row
+// stride, box, swizzle and L2 promotion, so an encoded map is reused whenever
+// the same key comes back (repeated calls on the same layer).  A small
+// per-thread cache saves the driver call; entries are replaced round-robin.
+struct MapKey {
+  int dtype, swizzle, l2;
+  const void *addr;
+  uint64_t d0, d1, stride;
+  uint32_t b0, b1;
+  bool operator==(const MapKey &o) const {
+    return dtype == o.dtype && swizzle == o.swizzle && l2 == o.l2 && addr == o.addr && d0 == o.d0 && d1 == o.d1 &&
+           stride == o.stride && b0 == o.b0 && b1 == o.b1;
+  }
+};
+constexpr int kMapCache = 32;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  int n = 0, next = 0;
+};
+thread_local MapCache t_maps;
+
+CUresult encode_2d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *out, CUtensorMapDataType dt, const void *addr,
+                   uint64_t d0, uint64_t d1, uint64_t stride_bytes, uint32_t b0, uint32_t b1,
+                   CUtensorMapSwizzle swz, CUtensorMapL2promotion l2) {
+  const MapKey k{(int)dt, (int)swz, (int)l2, addr, d0, d1, stride_bytes, b0, b1};
+  for (int i = 0; i < t_maps.n; ++i)
+    if (t_maps.key[i] == k) {
+      *out = t_maps.map[i];
+      return CUDA_SUCCESS;
+    }
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(out, dt, 2, const_cast<void *>(addr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return r;
+  const int slot = t_maps.n < kMapCache ? t_maps.n++ : (t_maps.next++ % kMapCache);
+  t_maps.key[slot] = k;
+  t_maps.map[slot] = *out;
+  return CUDA_SUCCESS;
+}
+
 
 enum Path { kPathGemv = 1, kPathTc = 2 };
 
@@ -374,9 +418,18 @@ size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   return ws_size_all(M, N, K, sm);
 }
 
-w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
-                     const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros, const float *awq_s,
-                     void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused dequantize-matmul; with a CSR (row_ptr, col, val) the sparse part of
+// a dense + sparse split is added by a separate kernel right after it.  (Fusing
+// it into the decode kernel's output writes measured slower on B200: the chain
+// of dependent CSR and activation loads lands on every tile's critical path.)
+w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
+                      const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros, const float *awq_s,
+                      void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream,
+                      const int32_t *row_ptr, const int32_t *col, const uint16_t *val) {
   t_last_error.clear();
   w4_status st = check_shape(M, N, K, group);
   if (st != W4_OK) return st;
@@ -415,29 +468,21 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
 
   if (plan.path == kPathGemv) {
     CUtensorMap tmP, tmS, tmZ;
-    const cuuint32_t estr[2] = {1, 1};
     {
-      const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-      const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-      const cuuint32_t box[2] = {128u, 64u};
-      CUresult r = enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      CUresult r = encode_2d(enc, &tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2), (uint64_t)N,
+                             (uint64_t)(K / 2), 128u, 64u, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
       if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
     }
     tmS = tmP;
     tmZ = tmP;
     if (plan.sc_tma) {
-      const cuuint64_t dims[2] = {(cuuint64_t)(K / w4::kGroup), (cuuint64_t)N};
-      const cuuint64_t strides[1] = {(cuuint64_t)(K / w4::kGroup) * 2};
-      const cuuint32_t box[2] = {8u, 64u};
-      CUresult r = enc(&tmS, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(scales), dims, strides, box,
-                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                       CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      const uint64_t kg = (uint64_t)(K / w4::kGroup);
+      CUresult r = encode_2d(enc, &tmS, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, kg, (uint64_t)N, kg * 2, 8u, 64u,
+                             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
       if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for scales failed (CUresult %d)", (int)r);
-      r = enc(&tmZ, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(zeros), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      r = encode_2d(enc, &tmZ, CU_TENSOR_MAP_DATA_TYPE_UINT16, zeros, kg, (uint64_t)N, kg * 2, 8u, 64u,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
       if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for zeros failed (CUresult %d)", (int)r);
     }
     w4::GemvParams p{};
@@ -448,28 +493,23 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
     p.kslices = plan.kslices; p.slots = plan.slots; p.kr = plan.kr; p.grid_x = plan.grid_x; p.xs_bytes = plan.xs_bytes;
     e = w4::launch_gemv(tmP, tmS, tmZ, p, plan.t8, xbf16, plan.sc_tma, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
+    if (row_ptr) {
+      e = w4::launch_sparse_add(X, xbf16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16, s);
+      if (e != cudaSuccess) return cuda_fail(e, "sparse add");
+    }
     return W4_OK;
   }
 
   CUtensorMap tmX, tmP;
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)plan.bn};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&tmX, xbf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                     const_cast<void *>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = encode_2d(enc, &tmX, xbf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X,
+                           (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64u, (uint32_t)plan.bn,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
     if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for X failed (CUresult %d)", (int)r);
   }
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N};
-    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {32, 128};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = encode_2d(enc, &tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2), (uint64_t)N,
+                           (uint64_t)(K / 2), 32u, 128u, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
     if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
   }
   w4::TcParams p{};
@@ -480,7 +520,22 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
   p.group = group;
   e = w4::launch_gemm_tc(tmX, tmP, p, xbf16, plan.bn, s);
   if (e != cudaSuccess) return cuda_fail(e, "tensor-core gemm launch");
+  if (row_ptr) {
+    e = w4::launch_sparse_add(X, xbf16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse add");
+  }
   return W4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
+                     const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros, const float *awq_s,
+                     void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream) {
+  return gemm_common(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, workspace, workspace_bytes,
+                     stream, nullptr, nullptr, nullptr);
 }
 
 w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K,
@@ -780,13 +835,8 @@ w4_status w4a16_gemm_outliers(const void *X, w4_dtype x_dtype, int64_t M, int64_
     t_last_error.clear();
     return fail(W4_ERR_INVALID_ARG, "null CSR pointer");
   }
-  w4_status st = w4a16_gemm(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, workspace,
-                            workspace_bytes, stream);
-  if (st != W4_OK) return st;
-  cudaError_t e = w4::launch_sparse_add(X, x_dtype == W4_BF16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16,
-                                        reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "sparse add");
-  return W4_OK;
+  return gemm_common(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, workspace, workspace_bytes,
+                     stream, row_ptr, col, val);
 }
 
 }  // extern "C"
