@@ -30,17 +30,18 @@ def _u16(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("N,K,awq,frac", [(256, 256, False, 0.001), (4096, 4096, False, 0.001),
-                                          (300, 1024, True, 0.002), (6144, 4096, False, 0.001)])
-def test_outlier_split_bit_exact(w4, N, K, awq, frac):
-    tag = ("outliers", N, K, awq)
+@pytest.mark.parametrize("N,K,awq,frac,group", [(256, 256, False, 0.001, 128), (4096, 4096, False, 0.001, 128),
+                                                (300, 1024, True, 0.002, 128), (6144, 4096, False, 0.001, 128),
+                                                (512, 1024, False, 0.002, 64), (256, 512, True, 0.002, 32)])
+def test_outlier_split_bit_exact(w4, N, K, awq, frac, group):
+    tag = ("outliers", N, K, awq, group)
     W = synthetic.weight(K, N, 0.02, 0.001, tag)
     s = synthetic.awq_scale(K, tag) if awq else None
     count = int(np.ceil(frac * N * K))
     packed, scales, zeros, (row_ptr, col, val) = w4.w4_quantize_outliers(
-        W.cuda(), count, None if s is None else s.cuda())
+        W.cuda(), count, None if s is None else s.cuda(), group=group)
     torch.cuda.synchronize()
-    c, sc, zp, rp, cl, vl = oracle.outlier_split(W.numpy(), count, None if s is None else s.numpy())
+    c, sc, zp, rp, cl, vl = oracle.outlier_split(W.numpy(), count, None if s is None else s.numpy(), group=group)
     assert np.array_equal(row_ptr.cpu().numpy(), rp)
     assert np.array_equal(col.cpu().numpy(), cl)
     assert np.array_equal(_u16(val), vl.view(np.uint16))

@@ -9,6 +9,8 @@
 // step uses IEEE fp32 round-to-nearest intrinsics so the results are bit-exact
 // with the definition in w4.h.  The kernel is HBM-bound: it reads W once and
 // writes 0.5 B of codes + 4 B of scale/zero per 128 weights.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace w4 {
@@ -58,9 +60,9 @@ constexpr int kQuantUnroll = 4;  // 128-element chunks in flight per warp
 // consecutive elements (groups never straddle rows, since G divides K) is held
 // by G/4 consecutive lanes, which reduce its min and max with shuffles.  Group j
 // of the flattened order is scales[j] / zeros[j] of the [N][K/G] arrays.
-template <typename TW, bool kAwq, bool kCodes, bool kSym>
+template <typename TW, bool kAwq, bool kCodes, bool kSym, int kG, bool kMask>
 __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W, const float *__restrict__ awq_s,
-                                                       int64_t E, int64_t K, int group,
+                                                       int64_t E, int64_t K,
                                                        const uint32_t *__restrict__ outlier_tau,
                                                        uint8_t *__restrict__ packed, uint16_t *__restrict__ scales,
                                                        uint16_t *__restrict__ zeros, uint8_t *__restrict__ codes) {
@@ -68,9 +70,9 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int64_t chunks = (E + 127) / 128;
-  const int lg = group >> 2;  // lanes per group
+  constexpr int lg = kG / 4;  // lanes per group
   // dense part of a dense + sparse split: weights with |w| >= tau count as 0 here
-  const uint32_t tau = outlier_tau ? *outlier_tau : 0xFFFFFFFFu;
+  const uint32_t tau = kMask ? *outlier_tau : 0xFFFFFFFFu;
 
   for (int64_t base = warp * kQuantUnroll; base < chunks; base += nwarps * kQuantUnroll) {
     float v[kQuantUnroll][4];
@@ -79,9 +81,11 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
       const int64_t e = (base + u) * 128 + lane * 4;
       if (e < E) {
         Load4<TW>::run(W + e, v[u]);
+        if constexpr (kMask) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if ((__float_as_uint(v[u][j]) & 0x7FFFFFFFu) >= tau) v[u][j] = 0.0f;
+          for (int j = 0; j < 4; ++j)
+            if ((__float_as_uint(v[u][j]) & 0x7FFFFFFFu) >= tau) v[u][j] = 0.0f;
+        }
         if (kAwq) {
           const int64_t k = e % K;
           const float4 s = __ldg(reinterpret_cast<const float4 *>(awq_s + k));
@@ -99,6 +103,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
       const int64_t e = (base + u) * 128 + lane * 4;
       float mn = fminf(fminf(v[u][0], v[u][1]), fminf(v[u][2], v[u][3]));
       float mx = fmaxf(fmaxf(v[u][0], v[u][1]), fmaxf(v[u][2], v[u][3]));
+#pragma unroll
       for (int o = lg >> 1; o > 0; o >>= 1) {  // within each aligned run of lg lanes
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -135,7 +140,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
         reinterpret_cast<uint16_t *>(packed)[e >> 2] = pk;
         if (kCodes) reinterpret_cast<uint32_t *>(codes)[e >> 2] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
         if ((lane & (lg - 1)) == 0) {
-          const int64_t gi = e / group;
+          const int64_t gi = e / kG;
           scales[gi] = __half_as_ushort(sc16);
           zeros[gi] = __half_as_ushort(__float2half_rn(z));
         }
@@ -178,26 +183,58 @@ int grid_for(int64_t work_items, int items_per_block, int sm_count, int blocks_p
   return (int)need;
 }
 
-template <typename TW, bool kSym>
-cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, int group,
-                              const uint32_t *tau, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
-                              uint8_t *codes, int sm_count, cudaStream_t stream) {
+template <typename TW, bool kSym, int kG, bool kMask>
+cudaError_t launch_quantize_g(const void *W, const float *awq_s, int64_t N, int64_t K, const uint32_t *tau,
+                              uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
+                              cudaStream_t stream) {
   const int64_t E = N * K;
   const int64_t chunks = (E + 127) / 128;
   const int grid = grid_for(chunks, 8 * kQuantUnroll, sm_count, 8);
   const TW *w = static_cast<const TW *>(W);
   if (awq_s) {
     if (codes)
-      quantize_kernel<TW, true, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
+      quantize_kernel<TW, true, true, kSym, kG, kMask><<<grid, 256, 0, stream>>>(w, awq_s, E, K, tau, packed, scales,
+                                                                                  zeros, codes);
     else
-      quantize_kernel<TW, true, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
+      quantize_kernel<TW, true, false, kSym, kG, kMask><<<grid, 256, 0, stream>>>(w, awq_s, E, K, tau, packed, scales,
+                                                                                   zeros, codes);
   } else {
     if (codes)
-      quantize_kernel<TW, false, true, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
+      quantize_kernel<TW, false, true, kSym, kG, kMask><<<grid, 256, 0, stream>>>(w, awq_s, E, K, tau, packed, scales,
+                                                                                   zeros, codes);
     else
-      quantize_kernel<TW, false, false, kSym><<<grid, 256, 0, stream>>>(w, awq_s, E, K, group, tau, packed, scales, zeros, codes);
+      quantize_kernel<TW, false, false, kSym, kG, kMask><<<grid, 256, 0, stream>>>(w, awq_s, E, K, tau, packed,
+                                                                                    scales, zeros, codes);
   }
   return cudaGetLastError();
+}
+
+template <typename TW, bool kSym>
+cudaError_t launch_quantize_t(const void *W, const float *awq_s, int64_t N, int64_t K, int group,
+                              const uint32_t *tau, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
+                              uint8_t *codes, int sm_count, cudaStream_t stream) {
+  if (tau) {  // dense part of the outlier split: fp32 weights, asymmetric codes (see libw4.cu)
+    if constexpr (std::is_same<TW, float>::value && !kSym) {
+      switch (group) {
+        case 32: return launch_quantize_g<TW, false, 32, true>(W, awq_s, N, K, tau, packed, scales, zeros, codes,
+                                                              sm_count, stream);
+        case 64: return launch_quantize_g<TW, false, 64, true>(W, awq_s, N, K, tau, packed, scales, zeros, codes,
+                                                              sm_count, stream);
+        default: return launch_quantize_g<TW, false, 128, true>(W, awq_s, N, K, tau, packed, scales, zeros, codes,
+                                                               sm_count, stream);
+      }
+    } else {
+      return cudaErrorInvalidValue;
+    }
+  }
+  switch (group) {
+    case 32: return launch_quantize_g<TW, kSym, 32, false>(W, awq_s, N, K, tau, packed, scales, zeros, codes, sm_count,
+                                                           stream);
+    case 64: return launch_quantize_g<TW, kSym, 64, false>(W, awq_s, N, K, tau, packed, scales, zeros, codes, sm_count,
+                                                           stream);
+    default: return launch_quantize_g<TW, kSym, 128, false>(W, awq_s, N, K, tau, packed, scales, zeros, codes,
+                                                            sm_count, stream);
+  }
 }
 
 template <bool kSym>
