@@ -232,6 +232,45 @@ def time_cpu_oracle(budget_s=12.0, rows_per_layer=512):
                       f"{reps} repetitions in {dt:.1f} s on one host core"}
 
 
+def _oracle_worker(rows, budget_s):
+    """One process of the all-cores oracle timing: its own row slice of every layer, looped
+    for budget_s seconds after a warm-up; returns the algorithmic bytes it covered and its time."""
+    torch.set_num_threads(1)  # one core per process
+    cpu_oracle_step(rows)
+    t0 = time.perf_counter()
+    nbytes = 0
+    while time.perf_counter() - t0 < budget_s:
+        nbytes += cpu_oracle_step(rows)
+    return nbytes, time.perf_counter() - t0
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def time_cpu_oracle_all_cores(budget_s=10.0, rows_per_layer=512):
+    """The oracle on the host cores (up to 32): one spawned process per core, each on its own
+    512-row sample of each layer (independent rows, as the oracle computes them one by one)."""
+    import multiprocessing as mp
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    cores = min(cores, 32)  # bounds the start-up cost (each process imports torch)
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(cores) as pool:
+        res = pool.starmap(_oracle_worker, [(rows_per_layer, budget_s)] * cores)
+    nbytes = sum(r[0] for r in res)
+    dt = max(r[1] for r in res)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{cores} processes, each {rows_per_layer} output rows of each of the 4 Llama-3-8B layers "
+                      f"(dequant + fp64 matmul, M=1) for {budget_s:.0f} s; CPU: {cpu_model()}"}
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -466,6 +505,48 @@ def stack70b_leg(w4, replays=3):
     return out
 
 
+def verify_leg(w4, Ms=(4, 8, 16, 32, 48, 64), steps=20):
+    """Speculative-verification / small-batch decode: the four Llama-3-8B layers with the AWQ
+    scale folded in, at each M; two weight copies per layer rotate (232 MB > L2); each M's
+    steps are captured in one CUDA graph."""
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    layers = []
+    for name in LAYERS:
+        K, N = synthetic.SHAPES_8B[name]
+        s = synthetic.awq_scale(K, ("bench", "verify", name)).to(dev)
+        copies = []
+        for c in range(2):
+            gen.manual_seed(synthetic.seed_of("bench", "verify", name, c) % (2 ** 62))
+            W = torch.randn((N, K), generator=gen, device=dev) * 0.02
+            copies.append(w4.w4_quantize(W, s))
+            del W
+        layers.append((K, N, s, copies))
+    stream = torch.cuda.Stream()
+    out = {}
+    for M in Ms:
+        bufs = []
+        for K, N, s, copies in layers:
+            X = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+            bufs.append((X, torch.empty((M, N), dtype=torch.float32, device=dev), w4.workspace(M, N, K, dev)))
+
+        def step(i):
+            for (K, N, s, copies), (X, Y, ws) in zip(layers, bufs):
+                packed, scales, zeros = copies[i % 2]
+                w4.w4a16_gemm(X, packed, scales, zeros, s, out=Y, ws=ws)
+
+        g = _graph_of(step, steps, 3, stream)
+        ms = _replay_timed(g, stream) / steps
+        del g
+        nbytes = sum(gemm_bytes(M, N, K) + 4 * K for K, N, _, _ in layers)
+        out[f"M{M}"] = {"us_per_step": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    out["workload"] = ("verify_8b: qkv/o_proj/gate_up/down with AWQ s, bf16 X, M = batch x (draft 5 + 1); "
+                       "M <= 8 on the decode kernel, above on the tensor-core kernel")
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
 def outlier_leg(w4, launches=60):
     """Decode GEMM with the dense + sparse outlier split (0.1% of the weights in fp16 CSR) on the
     Llama-3-8B gate_up shape at M=1, three weight copies rotated (188 MB > L2), in one CUDA graph."""
@@ -572,6 +653,7 @@ def main():
                                            "unit": "GB/s", "frac": round(q_gbs / hbm_peak, 4)}}
         pf, pf_all, pf_ms = prefill_leg(w4)
         extras["stack70b"] = stack70b_leg(w4)
+        extras["verify_8b"] = verify_leg(w4)
         extras["awq_search"] = awq_search_leg(w4)
         extras["outliers"] = outlier_leg(w4)
         extras["prefill"] = {"value": round(pf_all, 1), "unit": "TFLOP/s", "ms_per_step": round(pf_ms, 3),
@@ -583,6 +665,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_cpu_oracle()
+        extras["cpu_baseline_all_cores"] = time_cpu_oracle_all_cores()
 
     if rank == 0:
         line = {
