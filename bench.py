@@ -66,12 +66,14 @@ def quant_bytes(N, K):
     return 4 * N * K + N * K // 2 + 4 * N * (K // G)
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {"gemv_mma_gate_up_m1": ("common.cuh", "gemv_mma.cu")}  # files that define the kernel
+
+
+def kernel_source_hash(kernel_key="gemv_mma_gate_up_m1"):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "weight_only_int4_w4_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(d, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel_key]:
+        h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -81,7 +83,7 @@ def committed_traffic(kernel_key):
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
         e = t.get(kernel_key)
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(kernel_key):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -581,6 +583,34 @@ def outlier_leg(w4, launches=60):
     return out
 
 
+def gptq_leg(w4):
+    """GPTQ column sweep of the Llama-3-8B o_proj weights (4096 x 4096) with a 512-row
+    calibration batch (correlated channels): device time per layer (synchronous call)."""
+    dev = torch.device("cuda")
+    K, N = synthetic.SHAPES_8B["o_proj"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synthetic.seed_of("bench", "gptq") % (2 ** 62))
+    W = torch.randn((N, K), generator=gen, device=dev) * 0.02
+    X = torch.randn((512, K), generator=gen, device=dev)
+    X = (X + 0.5 * X[:, :1]).to(torch.bfloat16)
+    w4.w4_quantize_gptq(W, X)  # warm-up
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    packed, scales, zeros = w4.w4_quantize_gptq(W, X)
+    ms = (time.perf_counter() - t0) * 1e3
+    Xf = X.float()
+    y = Xf @ W.t()
+    rtn = w4.w4_quantize(W)
+    err = {}
+    for name, (p, sc, z) in (("gptq", (packed, scales, zeros)), ("rtn", rtn)):
+        err[name] = float(((y - w4.w4a16_gemm(X, p, sc, z)) ** 2).sum())
+    out = {"ms_per_layer": round(ms, 1), "output_error_vs_rtn": round(err["gptq"] / err["rtn"], 4),
+           "workload": "o_proj 4096x4096 fp32 W, 512 x 4096 bf16 calibration (correlated channels), group 128"}
+    del W, X, Xf, y
+    torch.cuda.empty_cache()
+    return out
+
+
 def awq_search_leg(w4, repeats=3):
     """AWQ exponent search on the Llama-3-8B gate_up weights with a 512-row calibration batch
     (1% of the channels x10), 21 exponents in [-1, 1]: device time per search."""
@@ -655,6 +685,7 @@ def main():
         extras["stack70b"] = stack70b_leg(w4)
         extras["verify_8b"] = verify_leg(w4)
         extras["awq_search"] = awq_search_leg(w4)
+        extras["gptq"] = gptq_leg(w4)
         extras["outliers"] = outlier_leg(w4)
         extras["prefill"] = {"value": round(pf_all, 1), "unit": "TFLOP/s", "ms_per_step": round(pf_ms, 3),
                              "workload": "Llama-3-70B qkv/o_proj/gate_up/down, M=8192, bf16 X",

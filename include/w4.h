@@ -232,6 +232,37 @@ w4_status w4a16_gemm_outliers(const void *X, w4_dtype x_dtype, int64_t M,
                               w4_stream_t stream);
 
 /*
+ * GPTQ quantization (ch. 22 "Advanced inference optimisation", section 22.3:
+ * quantize W so as to minimize || W X - W^ X ||_F^2 on calibration inputs,
+ * the Hessian H = 2 X X^T deciding how each weight's quantization error is
+ * compensated on the weights not yet quantized).  The column sweep, in fp64
+ * with a fixed order of operations:
+ *   H = 2 Xcal^T Xcal, plus damp_frac * trace(H) / K on the diagonal;
+ *   U = upper Cholesky factor of H^-1;
+ *   per row, k = 0..K-1: at each group start, scale and zero from the current
+ *   weights by the rule of w4_quantize; q = code of the current weight;
+ *   err = (w - w^) / U[k][k];  w[k'] -= err * U[k][k'] for k' > k.
+ *   W         device [N][K] fp32 (left unchanged)
+ *   Xcal      device [Mc][K] F16 or BF16 calibration activations
+ *   group     32, 64 or 128; K a multiple of 32 and at most 32768
+ *   damp_frac >= 0 (0.01 is usual)
+ *   packed, scales, zeros, codes   as for w4_quantize (codes may be NULL)
+ *   workspace device, w4_gptq_workspace_size(N, K) bytes (3 K^2 + N K doubles)
+ * The outputs are consumed by w4a16_gemm like those of w4_quantize.  Returns
+ * W4_ERR_INVALID_ARG if the damped Hessian is not positive definite.
+ * Synchronizes `stream`.
+ */
+w4_status w4_quantize_gptq(const float *W, int64_t N, int64_t K, int group,
+                           const void *Xcal, w4_dtype x_dtype, int64_t Mc,
+                           double damp_frac, uint8_t *packed,
+                           uint16_t *scales, uint16_t *zeros, uint8_t *codes,
+                           void *workspace, size_t workspace_bytes,
+                           w4_stream_t stream);
+
+/* Bytes of workspace w4_quantize_gptq needs (0 for invalid sizes). */
+size_t w4_gptq_workspace_size(int64_t N, int64_t K);
+
+/*
  * Decode GEMM with library-owned scratch: the same computation, kernel and
  * result as w4a16_gemm for decode shapes, with no workspace argument.  The
  * source pages have no counterpart to this call; it exists for callers that

@@ -40,6 +40,7 @@ def _load():
         _lib.w4o_quantize.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
         _lib.w4o_quantize_sym.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
         _lib.w4o_awq_search.argtypes = [P, I64, I64, ctypes.c_int, P, I64, P, ctypes.c_int, P, P, P]
+        _lib.w4o_gptq.argtypes = [P, I64, I64, ctypes.c_int, P, I64, ctypes.c_double, P, P, P]
         _lib.w4o_pack.argtypes = [P, I64, I64, P]
         _lib.w4o_unpack.argtypes = [P, I64, I64, P]
         _lib.w4o_dequant.argtypes = [P, P, P, P, I64, I64, ctypes.c_int, P]
@@ -130,6 +131,22 @@ def outlier_dequant(codes, scales, zeros, row_ptr, col, val, awq_s=None, group: 
     rows = np.repeat(np.arange(N), np.diff(row_ptr.astype(np.int64)))
     What[rows, col] += val.astype(np.float32)
     return What
+
+
+def gptq(W, X, group: int = 128, damp_frac: float = 0.01):
+    """GPTQ column sweep with Hessian 2 X^T X (plain fp64 loops): W [N,K] fp32, X [Mc,K] floats
+    -> (codes u8 [N,K], scales f16 [N,K/G], zeros f16 [N,K/G])."""
+    W = _c(W, np.float32)
+    X = _c(X, np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K), np.uint8)
+    scales = np.empty((N, K // group), np.uint16)
+    zeros = np.empty((N, K // group), np.uint16)
+    rc = _load().w4o_gptq(_ptr(W), N, K, group, _ptr(X), X.shape[0], float(damp_frac), _ptr(codes), _ptr(scales),
+                          _ptr(zeros))
+    if rc != 0:
+        raise ValueError(f"w4o_gptq failed ({rc})")
+    return codes, scales.view(np.float16), zeros.view(np.float16)
 
 
 def pack(codes):

@@ -303,3 +303,106 @@ done:
     free(m); free(s); free(codes); free(sc); free(zp); free(What); free(Yref); free(Yq);
     return rc;
 }
+
+/*
+ * GPTQ ([Ch22 22.3]: a layer's weights are quantized so as to minimize
+ * || W X - W^ X ||_F^2 on calibration inputs X, using the Hessian H = 2 X X^T to
+ * order the work and to compensate each weight's quantization error on the
+ * weights not yet quantized -- the Optimal Brain Compression idea).  The page
+ * gives no algorithm beyond that; the reading taken is the standard column
+ * sweep, in plain fp64 loops (no fused multiply-add):
+ *   H[a][b] = 2 sum_m x[m][a] x[m][b]  (m increasing);  H[a][a] += damp,
+ *   damp = damp_frac * (sum_a H[a][a]) / K  (a increasing);
+ *   U = the upper Cholesky factor of H^-1, computed as P inv(L') P with
+ *   L' the lower Cholesky factor of P H P (P reverses the order of k);
+ *   for each row, for k = 0..K-1 in order: at the start of each group, its
+ *   scale and zero point come from the current (updated) weights by the rule of
+ *   w4o_quantize (in fp32); q = the rounded code of the current weight,
+ *   err = (w - w^) / U[k][k], and every later weight of the row moves by
+ *   w[k'] -= err * U[k][k'].
+ * X [Mc][K] floats (the calibration activations), W [N][K] fp32.
+ * Outputs as for w4o_quantize.  Returns 0, -1 on bad arguments, -2 if H is not
+ * positive definite.
+ */
+int w4o_gptq(const float *W, int64_t N, int64_t K, int group, const float *X,
+             int64_t Mc, double damp_frac, uint8_t *codes, uint16_t *scales,
+             uint16_t *zeros) {
+    if (N < 1 || K < 1 || Mc < 1 || group <= 0 || K % group != 0 || group > 1024) return -1;
+    fesetround(FE_TONEAREST);
+    const int64_t Kg = K / group;
+    double *H = (double *)malloc(sizeof(double) * (size_t)(K * K));
+    double *L = (double *)calloc((size_t)(K * K), sizeof(double));
+    double *Li = (double *)calloc((size_t)(K * K), sizeof(double));
+    double *w = (double *)malloc(sizeof(double) * (size_t)K);
+    int rc = -1;
+    if (!H || !L || !Li || !w) goto out;
+    /* H = 2 X^T X, then damping */
+    for (int64_t a = 0; a < K; ++a)
+        for (int64_t b = 0; b < K; ++b) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < Mc; ++m) acc = acc + (double)X[m * K + a] * (double)X[m * K + b];
+            H[a * K + b] = 2.0 * acc;
+        }
+    {
+        double tr = 0.0;
+        for (int64_t a = 0; a < K; ++a) tr = tr + H[a * K + a];
+        const double damp = damp_frac * (tr / (double)K);
+        for (int64_t a = 0; a < K; ++a) H[a * K + a] = H[a * K + a] + damp;
+    }
+    /* L = lower Cholesky factor of R = P H P, R[i][j] = H[K-1-i][K-1-j] (left-looking) */
+    for (int64_t j = 0; j < K; ++j) {
+        double d = H[(K - 1 - j) * K + (K - 1 - j)];
+        for (int64_t k = 0; k < j; ++k) d = d - L[j * K + k] * L[j * K + k];
+        if (!(d > 0.0)) { rc = -2; goto out; }
+        const double ljj = sqrt(d);
+        L[j * K + j] = ljj;
+        for (int64_t i = j + 1; i < K; ++i) {
+            double acc = H[(K - 1 - i) * K + (K - 1 - j)];
+            for (int64_t k = 0; k < j; ++k) acc = acc - L[i * K + k] * L[j * K + k];
+            L[i * K + j] = acc / ljj;
+        }
+    }
+    /* Li = inverse of L (lower), column by column */
+    for (int64_t c = 0; c < K; ++c) {
+        Li[c * K + c] = 1.0 / L[c * K + c];
+        for (int64_t i = c + 1; i < K; ++i) {
+            double acc = 0.0;
+            for (int64_t k = c; k < i; ++k) acc = acc + L[i * K + k] * Li[k * K + c];
+            Li[i * K + c] = -acc / L[i * K + i];
+        }
+    }
+    /* U[j][k] = Li[K-1-j][K-1-k]; sweep each row */
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) w[k] = (double)W[n * K + k];
+        float sc = 1.0f, z = 0.0f;
+        for (int64_t j = 0; j < K; ++j) {
+            if (j % group == 0) {
+                float mn = (float)w[j], mx = (float)w[j];
+                for (int64_t i = 1; i < group; ++i) {
+                    const float v = (float)w[j + i];
+                    if (v < mn) mn = v;
+                    if (v > mx) mx = v;
+                }
+                uint16_t sc_bits = f32_to_f16_bits((mx - mn) / 15.0f);
+                sc = f16_bits_to_f32(sc_bits);
+                if (sc == 0.0f) {
+                    sc = 1.0f;
+                    sc_bits = f32_to_f16_bits(1.0f);
+                }
+                z = clamp_0_15(rintf(-mn / sc));
+                scales[n * Kg + j / group] = sc_bits;
+                zeros[n * Kg + j / group] = f32_to_f16_bits(z);
+            }
+            const float q = clamp_0_15(rintf((float)w[j] / sc) + z);
+            codes[n * K + j] = (uint8_t)q;
+            const float wq = (q - z) * sc;
+            const double ujj = Li[(K - 1 - j) * K + (K - 1 - j)];
+            const double err = (w[j] - (double)wq) / ujj;
+            for (int64_t k = j + 1; k < K; ++k) w[k] = w[k] - err * Li[(K - 1 - j) * K + (K - 1 - k)];
+        }
+    }
+    rc = 0;
+out:
+    free(H); free(L); free(Li); free(w);
+    return rc;
+}

@@ -440,3 +440,60 @@ def test_outlier_ties_at_threshold_are_all_kept():
     W[0, 3] = W[1, 7] = W[1, 9] = 0.5  # three tied largest magnitudes, count = 2
     codes, sc, zp, row_ptr, col, val = oracle.outlier_split(W, 2)
     assert list(row_ptr) == [0, 1, 3] and list(col) == [3, 7, 9]
+
+
+# ---------------------------------------------------------------- GPTQ column sweep
+
+def _gptq_numpy(W, X, group=G, damp_frac=0.01):
+    """Independent route: numpy/LAPACK inverse and Cholesky for U, the same sweep rule."""
+    W = W.astype(np.float64)
+    H = 2.0 * (X.astype(np.float64).T @ X.astype(np.float64))
+    H[np.diag_indices_from(H)] += damp_frac * np.trace(H) / H.shape[0]
+    U = np.linalg.cholesky(np.linalg.inv(H)).T  # upper factor: H^-1 = U^T U
+    N, K = W.shape
+    codes = np.zeros((N, K), np.uint8)
+    for n in range(N):
+        w = W[n].copy()
+        for j in range(K):
+            if j % group == 0:
+                c, s, z = oracle.quantize(w[j:j + group].astype(np.float32)[None, :], group=group)
+                sc, zp = np.float32(s[0, 0]), np.float32(z[0, 0])
+            q = min(max(np.rint(np.float32(w[j]) / sc) + zp, 0), 15)
+            codes[n, j] = q
+            err = (w[j] - np.float64((np.float32(q) - zp) * sc)) / U[j, j]
+            w[j + 1:] -= err * U[j, j + 1:]
+    return codes
+
+
+def test_gptq_matches_independent_linear_algebra_route():
+    """The oracle's own Cholesky/inverse loops against numpy's LAPACK route: same codes."""
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((12, 64)) * 0.02).astype(np.float32)
+    X = rng.standard_normal((48, 64)).astype(np.float32)
+    X += 0.7 * X[:, [3]]  # correlated channels, a non-trivial Hessian
+    c, s, z = oracle.gptq(W, X, group=32)
+    assert np.array_equal(c, _gptq_numpy(W, X, group=32))
+
+
+def test_gptq_with_diagonal_hessian_is_plain_rtn():
+    """X = 2 I (orthogonal channels): H is diagonal, no error is fed forward, so the
+    sweep reduces to round-to-nearest with the same per-group rule."""
+    K = 256
+    W = _weights(N=16, K=K, tag="gptq-diag")
+    X = (2.0 * np.eye(K)).astype(np.float32)
+    c, s, z = oracle.gptq(W, X)
+    c2, s2, z2 = oracle.quantize(W)
+    assert np.array_equal(c, c2)
+    assert np.array_equal(s.view(np.uint16), s2.view(np.uint16))
+    assert np.array_equal(z.view(np.uint16), z2.view(np.uint16))
+
+
+def test_gptq_lowers_the_layer_output_error():
+    """The objective ||X W^T - X W^^T||^2 is lower than plain RTN's on correlated data."""
+    rng = np.random.default_rng(3)
+    W = _weights(N=32, K=256, tag="gptq-obj")
+    X = rng.standard_normal((128, 256)).astype(np.float32)
+    X += 0.5 * X[:, [0]]
+    def err(c, s, z):
+        return float(np.sum((X @ W.T - X @ oracle.dequant(c, s, z).T) ** 2))
+    assert err(*oracle.gptq(W, X)) < 0.5 * err(*oracle.quantize(W))

@@ -1,0 +1,190 @@
+// gptq.cu -- GPTQ quantization of one weight matrix (ch. 22 "Advanced inference
+// optimisation", section 22.3: minimize || W X - W^ X ||_F^2 on calibration
+// inputs X, with the Hessian H = 2 X X^T deciding how each weight's quantization
+// error is compensated on the weights not yet quantized).
+//
+// Every step is fp64 with explicit round-to-nearest operations (no fused
+// multiply-add) and a fixed summation order, so the result is reproducible and
+// equals a plain-loop evaluation of the same definition:
+//   * H[a][b] = 2 sum_m x[m][a] x[m][b]  (m increasing); the diagonal gets
+//     damp = damp_frac * trace(H) / K added (trace summed in index order);
+//   * U, the upper Cholesky factor of H^-1, is P inv(L') P with L' the lower
+//     Cholesky factor of P H P (P reverses k): one Cholesky (one launch per
+//     column, parallel over rows, L' stored column-major) and one triangular
+//     inverse (one launch per row, parallel over columns);
+//   * the column sweep: one warp per weight row, k = 0..K-1 in order; at each
+//     group start the scale and zero come from the current weights by the RTN
+//     rule (fp32, as in quantize.cu); err = (w - w^) / U[k][k] and every later
+//     weight moves by w[k'] -= err * U[k][k'].
+#include "common.cuh"
+
+namespace w4 {
+namespace gptq_impl {
+
+constexpr int kHT = 16;  // Hessian tile (16 x 16 outputs per block)
+constexpr int kHM = 32;  // calibration rows per shared-memory chunk
+
+template <bool kBf16>
+__device__ __forceinline__ double x_val(uint16_t b) {
+  return (double)(kBf16 ? __uint_as_float((uint32_t)b << 16) : __half2float(__ushort_as_half(b)));
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256) hessian_kernel(const uint16_t *__restrict__ X, int64_t Mc, int64_t K,
+                                                      double *__restrict__ H) {
+  __shared__ double xa[kHM][kHT], xb[kHM][kHT];
+  const int ta = threadIdx.x / kHT, tb = threadIdx.x % kHT;
+  const int64_t a0 = (int64_t)blockIdx.y * kHT, b0 = (int64_t)blockIdx.x * kHT;
+  double acc = 0.0;
+  for (int64_t m0 = 0; m0 < Mc; m0 += kHM) {
+    for (int i = threadIdx.x; i < kHM * kHT; i += blockDim.x) {
+      const int mm = i / kHT, c = i % kHT;
+      const int64_t m = m0 + mm;
+      xa[mm][c] = (m < Mc && a0 + c < K) ? x_val<kBf16>(X[m * K + a0 + c]) : 0.0;
+      xb[mm][c] = (m < Mc && b0 + c < K) ? x_val<kBf16>(X[m * K + b0 + c]) : 0.0;
+    }
+    __syncthreads();
+    const int lim = (int)min((int64_t)kHM, Mc - m0);
+    for (int mm = 0; mm < lim; ++mm) acc = __dadd_rn(acc, __dmul_rn(xa[mm][ta], xb[mm][tb]));
+    __syncthreads();
+  }
+  const int64_t a = a0 + ta, b = b0 + tb;
+  if (a < K && b < K) H[a * K + b] = __dmul_rn(2.0, acc);
+}
+
+__global__ void damp_kernel(double *__restrict__ H, int64_t K, double damp_frac) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  double tr = 0.0;
+  for (int64_t a = 0; a < K; ++a) tr = __dadd_rn(tr, H[a * K + a]);
+  const double damp = __dmul_rn(damp_frac, __ddiv_rn(tr, (double)K));
+  for (int64_t a = 0; a < K; ++a) H[a * K + a] = __dadd_rn(H[a * K + a], damp);
+}
+
+// Column j of L' (lower Cholesky factor of R = P H P, R[i][j] = H[K-1-i][K-1-j]).
+// Lc is column-major: Lc[k * K + i] = L'[i][k].  Every thread recomputes the
+// pivot with the same operations, so all of them agree on it bit for bit.
+__global__ void __launch_bounds__(256) chol_col_kernel(const double *__restrict__ H, int64_t K, int64_t j,
+                                                       double *__restrict__ Lc, int *__restrict__ bad) {
+  const int64_t i = j + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= K) return;
+  double d = H[(K - 1 - j) * K + (K - 1 - j)];
+  for (int64_t k = 0; k < j; ++k) {
+    const double l = Lc[k * K + j];
+    d = __dsub_rn(d, __dmul_rn(l, l));
+  }
+  if (!(d > 0.0)) {
+    if (i == j) *bad = 1;
+    d = 1.0;  // keeps the values finite; the call reports the failure
+  }
+  const double ljj = __dsqrt_rn(d);
+  if (i == j) {
+    Lc[j * K + j] = ljj;
+    return;
+  }
+  double acc = H[(K - 1 - i) * K + (K - 1 - j)];
+  for (int64_t k = 0; k < j; ++k) acc = __dsub_rn(acc, __dmul_rn(Lc[k * K + i], Lc[k * K + j]));
+  Lc[j * K + i] = __ddiv_rn(acc, ljj);
+}
+
+// Row i of Li = inv(L') (row-major), for columns c <= i:
+// Li[i][i] = 1 / L'[i][i];  Li[i][c] = -(sum_{k=c}^{i-1} L'[i][k] Li[k][c]) / L'[i][i].
+__global__ void __launch_bounds__(256) inv_row_kernel(const double *__restrict__ Lc, int64_t K, int64_t i,
+                                                      double *__restrict__ Li) {
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (c > i) return;
+  const double lii = Lc[i * K + i];
+  if (c == i) {
+    Li[i * K + i] = __ddiv_rn(1.0, lii);
+    return;
+  }
+  double acc = 0.0;
+  for (int64_t k = c; k < i; ++k) acc = __dadd_rn(acc, __dmul_rn(Lc[k * K + i], Li[k * K + c]));
+  Li[i * K + c] = __ddiv_rn(-acc, lii);
+}
+
+__device__ __forceinline__ float clamp15f(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
+
+// One warp per weight row; U[j][k] = Li[K-1-j][K-1-k].
+template <int kG>
+__global__ void __launch_bounds__(256) sweep_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                    const double *__restrict__ Li, double *__restrict__ Wd,
+                                                    uint8_t *__restrict__ codes, uint16_t *__restrict__ scales,
+                                                    uint16_t *__restrict__ zeros) {
+  constexpr int kPer = kG / 32;  // group elements per lane
+  const int lane = threadIdx.x & 31;
+  const int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (n >= N) return;
+  double *w = Wd + n * K;
+  for (int64_t k = lane; k < K; k += 32) w[k] = (double)W[n * K + k];
+  __syncwarp();
+  const int64_t Kg = K / kG;
+  float sc = 1.0f, z = 0.0f;
+  for (int64_t j = 0; j < K; ++j) {
+    if (j % kG == 0) {
+      float mn, mx;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const float v = __double2float_rn(w[j + lane * kPer + e]);
+        mn = e == 0 ? v : fminf(mn, v);
+        mx = e == 0 ? v : fmaxf(mx, v);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      __half sc16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+      sc = __half2float(sc16);
+      if (sc == 0.0f) {
+        sc = 1.0f;
+        sc16 = __float2half_rn(1.0f);
+      }
+      z = clamp15f(rintf(__fdiv_rn(-mn, sc)));
+      if (lane == 0) {
+        scales[n * Kg + j / kG] = __half_as_ushort(sc16);
+        zeros[n * Kg + j / kG] = __half_as_ushort(__float2half_rn(z));
+      }
+    }
+    const double wj = w[j];
+    const float q = clamp15f(__fadd_rn(rintf(__fdiv_rn(__double2float_rn(wj), sc)), z));
+    if (lane == 0) codes[n * K + j] = (uint8_t)q;
+    const float wq = __fmul_rn(__fsub_rn(q, z), sc);
+    const double *urow = Li + (K - 1 - j) * K + (K - 1);  // urow[-k] = U[j][k]
+    const double err = __ddiv_rn(__dsub_rn(wj, (double)wq), urow[-j]);
+    for (int64_t k = j + 1 + lane; k < K; k += 32) w[k] = __dsub_rn(w[k], __dmul_rn(err, urow[-k]));
+    __syncwarp();
+  }
+}
+
+}  // namespace gptq_impl
+
+// Hessian, damping, Cholesky and inverse: Li (row-major K x K) holds inv(L').
+// H, Lc, Li: K*K doubles each (Lc need not be zeroed: only its lower part is read);
+// bad: one int, zero on entry, set when H is not positive definite.
+cudaError_t launch_gptq_hinv(const void *X, bool x_bf16, int64_t Mc, int64_t K, double damp_frac, double *H,
+                             double *Lc, double *Li, int *bad, cudaStream_t stream) {
+  using namespace gptq_impl;
+  const dim3 hg((unsigned)((K + kHT - 1) / kHT), (unsigned)((K + kHT - 1) / kHT));
+  const uint16_t *x = static_cast<const uint16_t *>(X);
+  if (x_bf16) hessian_kernel<true><<<hg, kHT * kHT, 0, stream>>>(x, Mc, K, H);
+  else hessian_kernel<false><<<hg, kHT * kHT, 0, stream>>>(x, Mc, K, H);
+  damp_kernel<<<1, 32, 0, stream>>>(H, K, damp_frac);
+  for (int64_t j = 0; j < K; ++j)
+    chol_col_kernel<<<(unsigned)((K - j + 255) / 256), 256, 0, stream>>>(H, K, j, Lc, bad);
+  for (int64_t i = 0; i < K; ++i) inv_row_kernel<<<(unsigned)((i + 1 + 255) / 256), 256, 0, stream>>>(Lc, K, i, Li);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gptq_sweep(const float *W, int64_t N, int64_t K, int group, const double *Li, double *Wd,
+                              uint8_t *codes, uint16_t *scales, uint16_t *zeros, cudaStream_t stream) {
+  using namespace gptq_impl;
+  const unsigned blocks = (unsigned)((N * 32 + 255) / 256);
+  switch (group) {
+    case 32: sweep_kernel<32><<<blocks, 256, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
+    case 64: sweep_kernel<64><<<blocks, 256, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
+    default: sweep_kernel<128><<<blocks, 256, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace w4

@@ -21,6 +21,7 @@
 #include "quantize.cu"
 #include "awq_search.cu"
 #include "outliers.cu"
+#include "gptq.cu"
 #include "w4.h"
 
 namespace w4 {
@@ -37,6 +38,10 @@ cudaError_t launch_outlier_threshold(const float *W, int64_t E, int64_t count, u
                                      int sm_count, cudaStream_t stream);
 cudaError_t launch_outlier_csr(const float *W, int64_t N, int64_t K, const uint32_t *state, int32_t *counts,
                                int32_t *row_ptr, int64_t cap, int32_t *col, uint16_t *val, cudaStream_t stream);
+cudaError_t launch_gptq_hinv(const void *X, bool x_bf16, int64_t Mc, int64_t K, double damp_frac, double *H,
+                             double *Lc, double *Li, int *bad, cudaStream_t stream);
+cudaError_t launch_gptq_sweep(const float *W, int64_t N, int64_t K, int group, const double *Li, double *Wd,
+                              uint8_t *codes, uint16_t *scales, uint16_t *zeros, cudaStream_t stream);
 cudaError_t launch_sparse_add(const void *X, bool x_bf16, int64_t M, int64_t N, int64_t K, const int32_t *row_ptr,
                               const int32_t *col, const uint16_t *val, void *Y, bool y_bf16, cudaStream_t stream);
 cudaError_t launch_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed, int sm_count,
@@ -837,6 +842,87 @@ w4_status w4a16_gemm_outliers(const void *X, w4_dtype x_dtype, int64_t M, int64_
   }
   return gemm_common(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, workspace, workspace_bytes,
                      stream, row_ptr, col, val);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// GPTQ: see gptq.cu for the method, include/w4.h for the contract.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct GptqLayout {
+  size_t h, lc, li, wd, codes, bad, total;
+};
+
+GptqLayout gptq_layout(int64_t N, int64_t K) {
+  GptqLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.h = take((size_t)K * K * 8);
+  L.lc = take((size_t)K * K * 8);
+  L.li = take((size_t)K * K * 8);
+  L.wd = take((size_t)N * K * 8);
+  L.codes = take((size_t)N * K);
+  L.bad = take(256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4_gptq_workspace_size(int64_t N, int64_t K) {
+  if (N < 1 || K < 1) return 0;
+  return gptq_layout(N, K).total;
+}
+
+w4_status w4_quantize_gptq(const float *W, int64_t N, int64_t K, int group, const void *Xcal, w4_dtype x_dtype,
+                           int64_t Mc, double damp_frac, uint8_t *packed, uint16_t *scales, uint16_t *zeros,
+                           uint8_t *codes, void *workspace, size_t workspace_bytes, w4_stream_t stream) {
+  t_last_error.clear();
+  w4_status st = check_shape(Mc, N, K, group);
+  if (st != W4_OK) return st;
+  if (x_dtype != W4_F16 && x_dtype != W4_BF16) return fail(W4_ERR_UNSUPPORTED, "calibration dtype must be F16 or BF16");
+  if (K % 32 != 0) return fail(W4_ERR_INVALID_ARG, "K=%lld must be a multiple of 32", (long long)K);
+  if (K > 32768) return fail(W4_ERR_UNSUPPORTED, "K=%lld: the K x K Hessian factors are limited to K <= 32768",
+                             (long long)K);
+  if (!(damp_frac >= 0.0) || !std::isfinite(damp_frac)) return fail(W4_ERR_INVALID_ARG, "damp_frac must be >= 0");
+  if (!W || !Xcal || !packed || !scales || !zeros || !workspace) return fail(W4_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(W) || !aligned16(Xcal) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros) ||
+      !aligned16(workspace) || (codes && !aligned16(codes)))
+    return fail(W4_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  const GptqLayout L = gptq_layout(N, K);
+  if (workspace_bytes < L.total)
+    return fail(W4_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", L.total, workspace_bytes);
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  double *H = reinterpret_cast<double *>(ws + L.h);
+  double *Lc = reinterpret_cast<double *>(ws + L.lc);
+  double *Li = reinterpret_cast<double *>(ws + L.li);
+  double *Wd = reinterpret_cast<double *>(ws + L.wd);
+  uint8_t *cbuf = codes ? codes : ws + L.codes;
+  int *bad = reinterpret_cast<int *>(ws + L.bad);
+  if ((e = cudaMemsetAsync(bad, 0, sizeof(int), cs)) != cudaSuccess) return cuda_fail(e, "clear flag");
+  if ((e = w4::launch_gptq_hinv(Xcal, x_dtype == W4_BF16, Mc, K, damp_frac, H, Lc, Li, bad, cs)) != cudaSuccess)
+    return cuda_fail(e, "Hessian factors");
+  if ((e = w4::launch_gptq_sweep(W, N, K, group, Li, Wd, cbuf, scales, zeros, cs)) != cudaSuccess)
+    return cuda_fail(e, "column sweep");
+  if ((e = w4::launch_pack(cbuf, N, K, packed, sm, cs)) != cudaSuccess) return cuda_fail(e, "pack");
+  int host_bad = 0;
+  if ((e = cudaMemcpyAsync(&host_bad, bad, sizeof host_bad, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+    return cuda_fail(e, "read flag");
+  if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  if (host_bad) return fail(W4_ERR_INVALID_ARG, "the damped Hessian 2 X^T X is not positive definite");
+  return W4_OK;
 }
 
 }  // extern "C"

@@ -44,6 +44,10 @@ _lib.w4_outliers_workspace_size.argtypes = [_I64]
 _lib.w4_outliers_workspace_size.restype = _SZ
 _lib.w4a16_gemm_outliers.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P,
                                      _P, ctypes.c_int, _P, _SZ, _P]
+_lib.w4_quantize_gptq.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, ctypes.c_int, _I64, ctypes.c_double, _P, _P, _P,
+                                  _P, _P, _SZ, _P]
+_lib.w4_gptq_workspace_size.argtypes = [_I64, _I64]
+_lib.w4_gptq_workspace_size.restype = _SZ
 _lib.w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
 _lib.w4a16_gemm_workspace_size.restype = _SZ
 _lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -51,6 +55,7 @@ _lib.w4_status_string.argtypes = [ctypes.c_int]
 _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
 for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_awq_search", "w4_quantize_outliers", "w4a16_gemm_outliers",
+           "w4_quantize_gptq",
            "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -236,6 +241,25 @@ def w4a16_gemm_outliers(X: torch.Tensor, packed, scales, zeros, csr, awq_s=None,
                                     _ptr(awq_s), _ptr(row_ptr), _ptr(col), _ptr(val), _ptr(out), _DT[out.dtype],
                                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)), "w4a16_gemm_outliers")
     return out
+
+
+def w4_quantize_gptq(W: torch.Tensor, Xcal: torch.Tensor, group: int = GROUP, damp_frac: float = 0.01,
+                     return_codes: bool = False, stream=None):
+    """GPTQ column sweep of W [N,K] fp32 with calibration Xcal [Mc,K] f16/bf16 (CUDA).
+    Returns (packed, scales, zeros) and, with return_codes, codes u8 [N,K]."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    assert Xcal.is_cuda and Xcal.dtype in (torch.float16, torch.bfloat16) and Xcal.is_contiguous()
+    N, K = W.shape
+    dev = W.device
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    zeros = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    codes = torch.empty((N, K), dtype=torch.uint8, device=dev) if return_codes else None
+    ws = torch.empty(int(_lib.w4_gptq_workspace_size(N, K)), dtype=torch.uint8, device=dev)
+    _check(_lib.w4_quantize_gptq(_ptr(W), N, K, group, _ptr(Xcal), _DT[Xcal.dtype], Xcal.shape[0], float(damp_frac),
+                                 _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(codes), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "w4_quantize_gptq")
+    return (packed, scales, zeros, codes) if return_codes else (packed, scales, zeros)
 
 
 AWQ_EXPONENTS = tuple(round(-1.0 + 0.1 * i, 1) for i in range(21))  # -1.0, -0.9, ..., 1.0
