@@ -128,7 +128,8 @@ w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed,
  *             again.  Calls that share a workspace must not overlap in time.
  * Accuracy: |Y - Y_exact| <= 2e-3 * sum_k |X[m][k] * W^[n][k]| per element on
  * the library's test distributions (fp32 accumulation; the prefill path rounds
- * W^ to 16 bits once, the decode path keeps (q - z) exact).
+ * W^ to 16 bits once, the decode path keeps (q - z) exact and, with AWQ,
+ * rounds x * s to fp16 once).
  */
 w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N,
                      int64_t K, int group, const uint8_t *packed,
@@ -268,8 +269,7 @@ size_t w4_gptq_workspace_size(int64_t N, int64_t K);
  * source pages have no counterpart to this call; it exists for callers that
  * cannot allocate device memory where they run the layer (an engine plugin
  * with no allocator of its own, a loop that must not take cudaMalloc).
- *   Arguments as for w4a16_gemm.  M <= 64 (M <= 32 with awq_s), else
- *   W4_ERR_UNSUPPORTED.
+ *   Arguments as for w4a16_gemm.  M <= 64, else W4_ERR_UNSUPPORTED.
  *   Scratch: a fixed array of w4a16_gemm_decode_static_capacity() bytes
  *   (8 MiB) per device, part of the library's own module.  A shape whose plan
  *   needs more returns W4_ERR_UNSUPPORTED with the sizes in w4_last_error()

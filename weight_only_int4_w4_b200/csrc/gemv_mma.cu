@@ -34,7 +34,8 @@
 //     power of two e per token and k-slice chosen so max|x'| lies in
 //     [2^13, 2^14): bf16 and fp16 inputs both convert exactly to fp16 (bar
 //     values 2^27 times below the token's maximum), and the result is scaled
-//     back by 2^-e exactly.  With AWQ, x' is split into fp16 high + low parts.
+//     back by 2^-e exactly.  With AWQ, x * s is rounded to fp16 (at most 2^-11
+//     relative per product), and P and S are summed from the rounded values.
 //   * Split-K (k-slices > 1): the row block's fp32 partials are stored, then
 //     one lane announces them with a release atomic on the 16-row block's
 //     counter; the ticket is read one tile later (hiding the round trip) and
@@ -85,7 +86,7 @@ constexpr int kComputeThreads = kComputeWarps * 32;
 
 // Staged activations for KR groups and M tokens: B fragments [g][tok][part][t][16 u32],
 // then (P, S) float pairs [g][tok], then the per-token exponents.
-__host__ __device__ constexpr int xs_frag_bytes(int kr, int m, bool awq) { return kr * m * (awq ? 2 : 1) * 4 * 64; }
+__host__ __device__ constexpr int xs_frag_bytes(int kr, int m, bool) { return kr * m * 4 * 64; }
 __host__ __device__ constexpr int xs_bytes_for(int kr, int m, bool awq) {
   return xs_frag_bytes(kr, m, awq) + kr * m * 8 + kMaxTok * 4;
 }
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
                                                    const __grid_constant__ CUtensorMap tmS,
                                                    const __grid_constant__ CUtensorMap tmZ, const GemvParams p) {
   constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
-  constexpr int kParts = kAwq ? 2 : 1;      // high / low fp16 parts of x'
+  constexpr int kParts = 1;  // x' (x * s with AWQ) staged as one fp16 value per channel
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -275,7 +276,10 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         mbar_arrive(&full[s]);
         mbar_arrive(&full[s]);
       }
-      grid_launch_dependents();  // all of this CTA's loads are issued
+      // All of this CTA's loads are issued: let the next kernel in the stream start
+      // launching.  (Triggering at CTA start measured slower on B200: consecutive
+      // kernels then pile their CTAs onto the same SMs and compete for issue slots.)
+      grid_launch_dependents();
     }
     return;
   }
@@ -341,17 +345,13 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
           }
           f.x *= se;  // exact power-of-two scaling
           f.y *= so;
+          // With AWQ, x * s is rounded to fp16 here (at most 2^-11 relative per
+          // product, well inside the accuracy bound); P and S below are summed from
+          // the same rounded values the tensor core multiplies.
           const uint32_t hi = f16x2_bits(f.x, f.y);
           const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
           hw[0][j] = hi;
-          float be = hv.x, bo = hv.y;
-          if constexpr (kAwq) {
-            const uint32_t lo = f16x2_bits(f.x - hv.x, f.y - hv.y);
-            const float2 lv = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
-            hw[kParts - 1][j] = lo;
-            be += lv.x;
-            bo += lv.y;
-          }
+          const float be = hv.x, bo = hv.y;
           sumB += be + bo;
           sumX += fmaf(16.0f, bo, be);
         }
@@ -806,7 +806,7 @@ cudaError_t launch_s(const CUtensorMap &tmP, const CUtensorMap &tmS, const CUten
 
 }  // namespace gemv_impl
 
-bool gemv_supports(int64_t M, bool awq) { return M <= 64 && !(awq && M > 32); }
+bool gemv_supports(int64_t M, bool) { return M <= 64; }
 
 // Shared-memory bytes of the staged activations for a k-slice of kr groups.
 int gemv_xs_bytes(int kr, int64_t M, bool awq) { return gemv_impl::xs_bytes_for(kr, (int)M, awq); }

@@ -15,7 +15,8 @@
 //   * the column sweep: one warp per weight row, k = 0..K-1 in order; at each
 //     group start the scale and zero come from the current weights by the RTN
 //     rule (fp32, as in quantize.cu); err = (w - w^) / U[k][k] and every later
-//     weight moves by w[k'] -= err * U[k][k'].
+//     weight moves by w[k'] -= err * U[k][k'] (a CTA of 8 row-warps stages each
+//     row of U in shared memory once for all of them).
 #include "common.cuh"
 
 namespace w4 {
@@ -104,55 +105,77 @@ __global__ void __launch_bounds__(256) inv_row_kernel(const double *__restrict__
 
 __device__ __forceinline__ float clamp15f(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
 
-// One warp per weight row; U[j][k] = Li[K-1-j][K-1-k].
+// One warp per weight row, kSweepRows rows per CTA; U[j][k] = Li[K-1-j][K-1-k].
+// At every step j the CTA stages the row U[j][j..K) in shared memory once for
+// all its warps (the same values in the same order as reading them directly).
+constexpr int kSweepRows = 8;
+constexpr int kUChunk = 2048;  // U entries staged per round (16 KiB)
+
 template <int kG>
-__global__ void __launch_bounds__(256) sweep_kernel(const float *__restrict__ W, int64_t N, int64_t K,
-                                                    const double *__restrict__ Li, double *__restrict__ Wd,
-                                                    uint8_t *__restrict__ codes, uint16_t *__restrict__ scales,
-                                                    uint16_t *__restrict__ zeros) {
+__global__ void __launch_bounds__(32 * kSweepRows) sweep_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                                 const double *__restrict__ Li,
+                                                                 double *__restrict__ Wd, uint8_t *__restrict__ codes,
+                                                                 uint16_t *__restrict__ scales,
+                                                                 uint16_t *__restrict__ zeros) {
   constexpr int kPer = kG / 32;  // group elements per lane
+  __shared__ double us[kUChunk];
+  __shared__ double errs[kSweepRows];
   const int lane = threadIdx.x & 31;
-  const int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (n >= N) return;
-  double *w = Wd + n * K;
-  for (int64_t k = lane; k < K; k += 32) w[k] = (double)W[n * K + k];
+  const int wid = threadIdx.x >> 5;
+  const int64_t n = (int64_t)blockIdx.x * kSweepRows + wid;
+  const bool row_ok = n < N;
+  double *w = Wd + (row_ok ? n : 0) * K;
+  if (row_ok)
+    for (int64_t k = lane; k < K; k += 32) w[k] = (double)W[n * K + k];
   __syncwarp();
   const int64_t Kg = K / kG;
   float sc = 1.0f, z = 0.0f;
   for (int64_t j = 0; j < K; ++j) {
-    if (j % kG == 0) {
-      float mn, mx;
+    const double *urow = Li + (K - 1 - j) * K + (K - 1);  // urow[-k] = U[j][k]
+    if (row_ok) {
+      if (j % kG == 0) {
+        float mn, mx;
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) {
-        const float v = __double2float_rn(w[j + lane * kPer + e]);
-        mn = e == 0 ? v : fminf(mn, v);
-        mx = e == 0 ? v : fmaxf(mx, v);
-      }
+        for (int e = 0; e < kPer; ++e) {
+          const float v = __double2float_rn(w[j + lane * kPer + e]);
+          mn = e == 0 ? v : fminf(mn, v);
+          mx = e == 0 ? v : fmaxf(mx, v);
+        }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        for (int o = 16; o > 0; o >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        __half sc16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+        sc = __half2float(sc16);
+        if (sc == 0.0f) {
+          sc = 1.0f;
+          sc16 = __float2half_rn(1.0f);
+        }
+        z = clamp15f(rintf(__fdiv_rn(-mn, sc)));
+        if (lane == 0) {
+          scales[n * Kg + j / kG] = __half_as_ushort(sc16);
+          zeros[n * Kg + j / kG] = __half_as_ushort(__float2half_rn(z));
+        }
       }
-      __half sc16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
-      sc = __half2float(sc16);
-      if (sc == 0.0f) {
-        sc = 1.0f;
-        sc16 = __float2half_rn(1.0f);
-      }
-      z = clamp15f(rintf(__fdiv_rn(-mn, sc)));
-      if (lane == 0) {
-        scales[n * Kg + j / kG] = __half_as_ushort(sc16);
-        zeros[n * Kg + j / kG] = __half_as_ushort(__float2half_rn(z));
+      const double wj = w[j];
+      const float q = clamp15f(__fadd_rn(rintf(__fdiv_rn(__double2float_rn(wj), sc)), z));
+      if (lane == 0) codes[n * K + j] = (uint8_t)q;
+      const float wq = __fmul_rn(__fsub_rn(q, z), sc);
+      if (lane == 0) errs[wid] = __ddiv_rn(__dsub_rn(wj, (double)wq), urow[-j]);
+    }
+    // every later weight of every row: w[k] -= err * U[j][k], U staged chunk by chunk
+    for (int64_t c0 = j + 1; c0 < K; c0 += kUChunk) {
+      const int64_t cn = min((int64_t)kUChunk, K - c0);
+      __syncthreads();  // errs written; the previous chunk fully used
+      for (int64_t t = threadIdx.x; t < cn; t += blockDim.x) us[t] = urow[-(c0 + t)];
+      __syncthreads();
+      if (row_ok) {
+        const double err = errs[wid];
+        for (int64_t t = lane; t < cn; t += 32) w[c0 + t] = __dsub_rn(w[c0 + t], __dmul_rn(err, us[t]));
       }
     }
-    const double wj = w[j];
-    const float q = clamp15f(__fadd_rn(rintf(__fdiv_rn(__double2float_rn(wj), sc)), z));
-    if (lane == 0) codes[n * K + j] = (uint8_t)q;
-    const float wq = __fmul_rn(__fsub_rn(q, z), sc);
-    const double *urow = Li + (K - 1 - j) * K + (K - 1);  // urow[-k] = U[j][k]
-    const double err = __ddiv_rn(__dsub_rn(wj, (double)wq), urow[-j]);
-    for (int64_t k = j + 1 + lane; k < K; k += 32) w[k] = __dsub_rn(w[k], __dmul_rn(err, urow[-k]));
-    __syncwarp();
+    __syncthreads();  // this step's updates are visible before the next step reads them
   }
 }
 
@@ -178,11 +201,12 @@ cudaError_t launch_gptq_hinv(const void *X, bool x_bf16, int64_t Mc, int64_t K, 
 cudaError_t launch_gptq_sweep(const float *W, int64_t N, int64_t K, int group, const double *Li, double *Wd,
                               uint8_t *codes, uint16_t *scales, uint16_t *zeros, cudaStream_t stream) {
   using namespace gptq_impl;
-  const unsigned blocks = (unsigned)((N * 32 + 255) / 256);
+  const unsigned blocks = (unsigned)((N + kSweepRows - 1) / kSweepRows);
+  const int threads = 32 * kSweepRows;
   switch (group) {
-    case 32: sweep_kernel<32><<<blocks, 256, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
-    case 64: sweep_kernel<64><<<blocks, 256, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
-    default: sweep_kernel<128><<<blocks, 256, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
+    case 32: sweep_kernel<32><<<blocks, threads, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
+    case 64: sweep_kernel<64><<<blocks, threads, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
+    default: sweep_kernel<128><<<blocks, threads, 0, stream>>>(W, N, K, Li, Wd, codes, scales, zeros); break;
   }
   return cudaGetLastError();
 }

@@ -649,8 +649,7 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
   const bool awq = awq_s != nullptr;
   if (group != w4::kGroup) return fail(W4_ERR_UNSUPPORTED, "the static-scratch decode GEMM serves group 128 only");
   if (!w4::gemv_supports(M, awq))
-    return fail(W4_ERR_UNSUPPORTED, "the static-scratch decode GEMM serves M <= 64 (M <= 32 with AWQ), got M=%lld%s",
-                (long long)M, awq ? " with AWQ" : "");
+    return fail(W4_ERR_UNSUPPORTED, "the static-scratch decode GEMM serves M <= 64, got M=%lld", (long long)M);
   int sm = 0;
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
