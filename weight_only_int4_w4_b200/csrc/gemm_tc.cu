@@ -14,10 +14,13 @@
 //               into 16-bit (q - z) * scale (* s[k] for AWQ), rounded once,
 //               and stores them with tcgen05.st straight into TMEM, where they
 //               are the A operand (TMEM lane = weight row, 2 values per column).
+//               With AWQ, warps 4..11: two warps per row, 32 codes each
+//               (measured: 8 warps speed up the AWQ kernel at M = 16..64 by
+//               6-22% and slow plain weights by 9-15%, so plain keeps 4).
 //   warp 1      one thread issues tcgen05.mma (A from TMEM, B = X from shared
 //               memory, fp32 accumulator in TMEM) and tcgen05.commit.
 //   warps 4..7  epilogue: tcgen05.ld of the accumulator, fp32 or bf16 stores
-//               (each warp store covers 32 consecutive output channels).
+//   (..11)      (each warp store covers 32 consecutive output channels).
 // TMEM columns: [0, BN) accumulator, then NS stages of 32 columns of A.
 // All waits are bounded (see common.cuh).  No TMA multicast anywhere.
 #include "common.cuh"
@@ -40,15 +43,40 @@ struct TcParams {
 
 namespace tc_impl {
 
+// Untiled bulk copy, global -> this CTA's shared memory (no multicast).  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// tcgen05.st of 16 consecutive 32-bit columns into each thread's own TMEM lane.
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 constexpr int kBK = 64;   // k per pipeline stage
-constexpr int kNS = 4;    // pipeline stages (measured: 6 stages ran 10-15% slower at M = 512..8192)
 constexpr int kPStage = 128 * 32;
 
 template <int BN>
 struct TcCfg {
+  // Pipeline stages.  Measured: 6 ran 10-15% slower than 4 at M = 512..8192;
+  // with BN = 64, 12 stages (148 KB) ran up to 50% slower than 4 on plain
+  // weights, where 4 stages (50 KB, 256 TMEM columns) let two CTAs share an SM,
+  // and 8 or 12 stages changed the AWQ kernel (one CTA per SM) by under 2%.
+  static constexpr int kNS = 4;
   static constexpr int kXStage = BN * 128;
+  static_assert(BN + 32 * kNS <= 512, "accumulator + A stages exceed TMEM");
   static constexpr uint32_t kTmemCols = (BN + 32 * kNS <= 256) ? 256u : 512u;
-  static constexpr int kSmem = 1024 /*align slack*/ + kNS * (kXStage + kPStage) + 256;
+  static constexpr int kSStage = kBK * 4;  // AWQ s of the stage's 64 channels (fp32)
+  static constexpr int kSmem = 1024 /*align slack*/ + kNS * (kXStage + kPStage + kSStage) + (3 * kNS + 2) * 8;
 };
 
 // 64 codes of one row (32 bytes) -> 32 columns of 16-bit pairs (k even in the low half).
@@ -95,30 +123,77 @@ __device__ __forceinline__ void dequant_row64(const uint4 &w0, const uint4 &w1, 
   }
 }
 
-// AND of a predicate over the 128 dequant/epilogue threads (named barrier 1).
+// Half of a row's k-block: 32 codes (16 bytes) -> 16 columns of 16-bit pairs, one (sc, z).
+template <bool kBf16, bool kAwq>
+__device__ __forceinline__ void dequant_row32(const uint4 &w4v, float sc, float z, const float *__restrict__ sk,
+                                              uint32_t (&out)[16]) {
+  const uint32_t words[4] = {w4v.x, w4v.y, w4v.z, w4v.w};
+  const float off_lo = -(256.0f + z) * sc;
+  const float sc16 = sc * 0.0625f;
+  const float off_hi = -(16.0f + z) * sc;
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    const uint32_t w = words[wi];
+    const uint32_t tb[4] = {w << 15, w << 7, w >> 1, w >> 9};  // byte b at bits 15..22
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float flo = __uint_as_float(lop3_and_or(tb[b], 0x00078000u, 0x43800000u));
+      const float fhi = __uint_as_float(lop3_and_or(tb[b], 0x00780000u, 0x43800000u));
+      float vlo = fmaf(flo, sc, off_lo);
+      float vhi = fmaf(fhi, sc16, off_hi);
+      const int col = wi * 4 + b;
+      if constexpr (kAwq) {
+        const float2 s2 = *reinterpret_cast<const float2 *>(sk + 2 * col);
+        vlo *= s2.x;
+        vhi *= s2.y;
+      }
+      if constexpr (kBf16) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(vlo, vhi);
+        out[col] = *reinterpret_cast<const uint32_t *>(&v);
+      } else {
+        const __half2 v = __floats2half2_rn(vlo, vhi);
+        out[col] = *reinterpret_cast<const uint32_t *>(&v);
+      }
+    }
+  }
+}
+
+// Dequant / epilogue warps: 4 (warps 4..7) for plain weights; 8 (warps 4..11) with
+// AWQ scales, whose extra multiply per weight makes the dequant the longer stage.
+template <bool kAwq>
+struct TcWarps {
+  static constexpr int kHalves = kAwq ? 2 : 1;      // warps per TMEM lane quadrant
+  static constexpr int kEpi = 128 * kHalves;        // dequant / epilogue threads
+  static constexpr int kThreads = 128 + kEpi;
+};
+
+// AND of a predicate over the kEpi dequant/epilogue threads (named barrier 1).
+template <int kEpi>
 __device__ __forceinline__ bool epilogue_vote(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.cta.red.and.pred q, 1, 128, p;\n\t"
+      "barrier.cta.red.and.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "n"(kEpi)
       : "memory");
   return r != 0;
 }
 
 template <int BN, bool kBf16, bool kAwq>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
+  constexpr int kNS = Cfg::kNS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sX = smem;
   uint8_t *sP = sX + kNS * Cfg::kXStage;
-  uint64_t *full = reinterpret_cast<uint64_t *>(sP + kNS * kPStage);
+  float *sS = reinterpret_cast<float *>(sP + kNS * kPStage);
+  uint64_t *full = reinterpret_cast<uint64_t *>(sS + kNS * kBK);
   uint64_t *empty = full + kNS;
   uint64_t *afull = empty + kNS;
   uint64_t *accfull = afull + kNS;
@@ -140,7 +215,7 @@ __global__ void __launch_bounds__(256, 1)
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], 128);
+      mbar_init(&afull[s], TcWarps<kAwq>::kEpi);
     }
     mbar_init(accfull, 1);
     fence_barrier_init();
@@ -162,10 +237,11 @@ __global__ void __launch_bounds__(256, 1)
         const int s = i % kNS;
         const uint32_t ph = (uint32_t)(i / kNS) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) break;
-        mbar_arrive_expect_tx(&full[s], Cfg::kXStage + kPStage);
+        mbar_arrive_expect_tx(&full[s], Cfg::kXStage + kPStage + (kAwq ? Cfg::kSStage : 0));
         const int kb = kb0 + i;
         tma_load_2d(sX + s * Cfg::kXStage, &tmX, &full[s], kb * kBK, (int32_t)m0);
         tma_load_2d(sP + s * kPStage, &tmP, &full[s], kb * (kBK / 2), (int32_t)n0);
+        if constexpr (kAwq) bulk_load(sS + s * kBK, p.awq_s + (int64_t)kb * kBK, Cfg::kSStage, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -187,13 +263,60 @@ __global__ void __launch_bounds__(256, 1)
       tc_commit(accfull);
     }
   } else if (warp >= 4) {
-    const int q = warp - 4;
+    constexpr int kHalves = TcWarps<kAwq>::kHalves;
+    constexpr int kEpi = TcWarps<kAwq>::kEpi;
+    // Warp w serves TMEM lane quadrant w % 4 (rows 32 (w % 4) ..+32).  With two
+    // warps per quadrant (w and w + 4), the first takes channels 0..31 of every
+    // k-block and the second 32..63.
+    const int q = warp & 3;
+    const int h = kHalves == 2 ? (warp - 4) >> 2 : 0;
     const int r = q * 32 + lane;
     const int64_t n = n0 + r;
     const bool row_ok = n < N;
     const int G = p.group;
     const int64_t Kg = K / G;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    // This row's scales and zeros.  When rows start on 16-byte boundaries
+    // (Kg % 8 == 0) they are read 8 groups at a time, one 16-byte chunk ahead of
+    // use, so the load latency overlaps the dequantization of earlier groups
+    // instead of stalling the stage that needs them.
+    const uint16_t *sc_row = p.scales + (row_ok ? n : 0) * Kg;
+    const uint16_t *z_row = p.zeros + (row_ok ? n : 0) * Kg;
+    const bool vec = (Kg & 7) == 0;
+    const int64_t nch = Kg >> 3;
+    uint4 scv = make_uint4(0, 0, 0, 0), zv = scv, scn = scv, zn = scv;
+    auto fetch = [&](int64_t c, uint4 &a, uint4 &b) {
+      if (row_ok && c < nch) {
+        a = __ldg(reinterpret_cast<const uint4 *>(sc_row) + c);
+        b = __ldg(reinterpret_cast<const uint4 *>(z_row) + c);
+      } else {
+        a = make_uint4(0, 0, 0, 0);
+        b = a;
+      }
+    };
+    // first group of this thread's k-range; its chunk is fetched before the loop
+    const int64_t g_first = G == 32 ? 2 * (int64_t)kb0 + h : (int64_t)kb0 / (G / 64);
+    int64_t cur = (g_first >> 3) - 1;  // chunk held in (scv, zv); the next one is in (scn, zn)
+    if (vec) fetch(cur + 1, scn, zn);
+    auto group_params = [&](int64_t g, float &gs, float &gz) {
+      if (vec) {
+        const int64_t c = g >> 3;  // groups advance by at most one chunk at a time
+        if (c != cur) {
+          scv = scn;
+          zv = zn;
+          cur = c;
+          fetch(c + 1, scn, zn);
+        }
+        const int e = (int)(g & 7), wsel = e >> 1, sh = 16 * (e & 1);
+        const uint32_t a = wsel == 0 ? scv.x : wsel == 1 ? scv.y : wsel == 2 ? scv.z : scv.w;
+        const uint32_t b = wsel == 0 ? zv.x : wsel == 1 ? zv.y : wsel == 2 ? zv.z : zv.w;
+        gs = half_bits_to_float((uint16_t)(a >> sh));
+        gz = half_bits_to_float((uint16_t)(b >> sh));
+      } else {
+        gs = row_ok ? half_bits_to_float(__ldg(sc_row + g)) : 0.0f;
+        gz = row_ok ? half_bits_to_float(__ldg(z_row + g)) : 0.0f;
+      }
+    };
     float sc = 0.0f, z = 0.0f, sc1 = 0.0f, z1 = 0.0f;
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
@@ -201,38 +324,39 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t ph = (uint32_t)(i / kNS) & 1u;
       const int kb = kb0 + i;
       if (G == 32) {  // two groups per 64-channel k-block
-        const int64_t grp = 2 * (int64_t)kb;
-        sc = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp)) : 0.0f;
-        z = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp)) : 0.0f;
-        sc1 = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp + 1)) : 0.0f;
-        z1 = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp + 1)) : 0.0f;
+        group_params(2 * (int64_t)kb + h, sc, z);
+        if (kHalves == 1) group_params(2 * (int64_t)kb + 1, sc1, z1);
       } else if (i == 0 || (kb & (G / 64 - 1)) == 0) {  // a group spans G / 64 k-blocks
-        const int64_t grp = kb / (G / 64);
-        sc = row_ok ? half_bits_to_float(__ldg(p.scales + n * Kg + grp)) : 0.0f;
-        z = row_ok ? half_bits_to_float(__ldg(p.zeros + n * Kg + grp)) : 0.0f;
+        group_params((int64_t)kb / (G / 64), sc, z);
         sc1 = sc;
         z1 = z;
       }
       if (!mbar_wait(&full[s], ph, kErrTimeoutDequant)) { ok = false; break; }
       const uint4 *src = reinterpret_cast<const uint4 *>(sP + s * kPStage + r * 32);
-      const uint4 w0 = src[0], w1 = src[1];
-      uint32_t out[32];
-      dequant_row64<kBf16, kAwq>(w0, w1, sc, z, sc1, z1, kAwq ? p.awq_s + (int64_t)kb * kBK : nullptr, out);
-      tmem_st_32x32b_x32(lane_base + (uint32_t)(BN + s * 32), out);
+      if constexpr (kHalves == 2) {
+        uint32_t out[16];
+        dequant_row32<kBf16, kAwq>(src[h], sc, z, sS + s * kBK + 32 * h, out);
+        tmem_st_32x32b_x16(lane_base + (uint32_t)(BN + s * 32 + 16 * h), out);
+      } else {
+        uint32_t out[32];
+        dequant_row64<kBf16, kAwq>(src[0], src[1], sc, z, sc1, z1, sS + s * kBK, out);
+        tmem_st_32x32b_x32(lane_base + (uint32_t)(BN + s * 32), out);
+      }
+      // (Deferring this wait until the next stage is dequantized measured 5-10% slower.)
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&afull[s]);
     }
 
-    // ---- epilogue (the decision to run it is made uniform over the 128 threads,
+    // ---- epilogue (the decision to run it is made uniform over the kEpi threads,
     // so the named barriers below are reached by all of them or by none)
     bool go = ok && nkb > 0 && mbar_wait(accfull, 0, kErrTimeoutEpilogue);
-    go = epilogue_vote(go);
+    go = epilogue_vote<kEpi>(go);
     if (go) {
       tc_fence_after();
       const bool direct = p.splits == 1;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = h * (BN / 32 / kHalves); c < (h + 1) * (BN / 32 / kHalves); ++c) {  // this warp's columns
         uint32_t v[32];
         tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), v);
         tc_wait_ld();
@@ -254,17 +378,17 @@ __global__ void __launch_bounds__(256, 1)
       if (!direct) {
         // last CTA of this output tile to arrive sums the split-K partials
         __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpi) : "memory");
         const int64_t tile = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
-        if (r == 0) {
+        if (r == 0 && h == 0) {
           const uint32_t prev = atomicAdd(&p.counters[tile], 1u);
           *s_last = prev == (uint32_t)(p.splits - 1);
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpi) : "memory");
         if (*s_last) {
           __threadfence();
           if (row_ok) {
-            for (int j = 0; j < BN; ++j) {
+            for (int j = h * (BN / kHalves); j < (h + 1) * (BN / kHalves); ++j) {
               const int64_t m = m0 + j;
               if (m >= M) break;
               float acc = 0.0f;
@@ -273,7 +397,7 @@ __global__ void __launch_bounds__(256, 1)
               else static_cast<float *>(p.Y)[m * N + n] = acc;
             }
           }
-          if (r == 0) atomicExch(&p.counters[tile], 0u);
+          if (r == 0 && h == 0) atomicExch(&p.counters[tile], 0u);
         }
       }
     }
@@ -295,7 +419,7 @@ cudaError_t launch_t(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcPar
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), Cfg::kSmem, smem_set);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN), (unsigned)p.splits);
-  kern<<<grid, 256, Cfg::kSmem, stream>>>(tmX, tmP, p);
+  kern<<<grid, TcWarps<kAwq>::kThreads, Cfg::kSmem, stream>>>(tmX, tmP, p);
   return cudaGetLastError();
 }
 

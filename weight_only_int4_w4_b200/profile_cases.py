@@ -7,6 +7,8 @@ Cases (seeded synthetic inputs drawn on the device, bf16 activations):
                     gate_up 4096->28672, down 14336->4096 at M=1 -- 4 times
   gemv_gate_up      gate_up 4096->28672 at M=1, 4 launches
   tc_o_proj         Llama-3-70B o_proj 8192->8192 at M=2048, 3 launches
+  tc_awq_gate_up    gate_up 4096->28672 with AWQ scales at M=48 (speculative
+                    verification of 8 drafts x 6 tokens), 3 launches
   quantize_gate_up  quantize+pack of gate_up's fp32 weights, 3 launches
 
 Each case launches eagerly (no CUDA graph), checks the device error word and
@@ -20,7 +22,7 @@ import torch
 
 from . import synthetic, w4
 
-CASES = ("decode_step", "gemv_gate_up", "tc_o_proj", "quantize_gate_up")
+CASES = ("decode_step", "gemv_gate_up", "tc_o_proj", "tc_awq_gate_up", "quantize_gate_up")
 
 
 def _weights(K, N, std, gen):
@@ -61,6 +63,16 @@ def run(case: str) -> None:
         Y = torch.empty((2048, N), device="cuda")
         for _ in range(3):
             w4.w4a16_gemm(X, packed, scales, zeros, out=Y)
+    elif case == "tc_awq_gate_up":
+        K, N = synthetic.SHAPES_8B["gate_up"]
+        s = synthetic.awq_scale(K, ("profile", case)).cuda()
+        W = torch.randn((N, K), generator=gen, device="cuda") * 0.02
+        packed, scales, zeros = w4.w4_quantize(W, awq_s=s)
+        del W
+        X = torch.randn((48, K), generator=gen, device="cuda").to(torch.bfloat16)
+        Y = torch.empty((48, N), device="cuda")
+        for _ in range(3):
+            w4.w4a16_gemm(X, packed, scales, zeros, awq_s=s, out=Y)
     else:
         K, N = synthetic.SHAPES_8B["gate_up"]
         W = torch.randn((N, K), generator=gen, device="cuda") * 0.02
