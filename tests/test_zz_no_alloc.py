@@ -30,6 +30,7 @@ def w4():
     (4, 4096, 14336, True),
     (3, 1000, 4096, False),
     (16, 4096, 14336, False),
+    (64, 4096, 14336, False),  # tensor-core plan with fewer K splits so its partials fit the scratch
 ])
 def test_static_scratch_matches_workspace_entry(w4, M, N, K, awq):
     tag = ("noalloc", M, N, K, awq)

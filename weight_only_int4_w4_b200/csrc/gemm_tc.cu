@@ -388,13 +388,44 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
         if (*s_last) {
           __threadfence();
           if (row_ok) {
-            for (int j = h * (BN / kHalves); j < (h + 1) * (BN / kHalves); ++j) {
-              const int64_t m = m0 + j;
-              if (m >= M) break;
-              float acc = 0.0f;
-              for (int s = 0; s < p.splits; ++s) acc += __ldcg(p.ws + ((int64_t)s * M + m) * N + n);
-              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[m * N + n] = __float2bfloat16_rn(acc);
-              else static_cast<float *>(p.Y)[m * N + n] = acc;
+            // 8 tokens x 4 splits of partials are loaded before they are added, so
+            // 32 independent loads are in flight (one token and one split at a
+            // time left every step waiting on L2).  The splits are summed in
+            // increasing order for every token.
+            const int j_begin = h * (BN / kHalves);
+            const int64_t rem = M - m0;
+            const int j_end = rem < j_begin + BN / kHalves ? (int)rem : j_begin + BN / kHalves;
+            for (int j0 = j_begin; j0 < j_end; j0 += 8) {
+              float acc[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+              int s = 0;
+              for (; s + 4 <= p.splits; s += 4) {
+                float v[4][8];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                  const float *part = p.ws + ((int64_t)(s + c) * M + m0 + j0) * N + n;
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) v[c][u] = j0 + u < j_end ? __ldcg(part + (int64_t)u * N) : 0.0f;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) acc[u] += v[c][u];
+              }
+              for (; s < p.splits; ++s) {
+                const float *part = p.ws + ((int64_t)s * M + m0 + j0) * N + n;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  if (j0 + u < j_end) acc[u] += __ldcg(part + (int64_t)u * N);
+              }
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                if (j0 + u >= j_end) break;
+                const int64_t m = m0 + j0 + u;
+                if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[m * N + n] = __float2bfloat16_rn(acc[u]);
+                else static_cast<float *>(p.Y)[m * N + n] = acc[u];
+              }
             }
           }
           if (r == 0 && h == 0) atomicExch(&p.counters[tile], 0u);

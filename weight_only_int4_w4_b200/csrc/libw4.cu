@@ -272,14 +272,31 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   return p;
 }
 
-GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, int sm) {
+// CTAs of the tensor-core kernel resident per SM.  Plain weights with BN <= 128
+// fit two (256 threads x at most 128 registers, <= 83 KB of shared memory, 256
+// TMEM columns each); the AWQ kernel (384 threads x 128 registers) and BN = 256
+// (150 KB of shared memory) fit one.
+int tc_ctas_per_sm(int bn, bool awq) { return (awq || bn == 256) ? 1 : 2; }
+
+// ws_cap: the partials must fit this many workspace bytes (fewer K splits otherwise).
+GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_cap = SIZE_MAX) {
   GemmPlan p;
   p.path = kPathTc;
   p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
   const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
   const int64_t total_kb = K / 64;
+  // Split K when the output tiles do not fill the SMs (each split keeps >= 8
+  // k-blocks), and further toward the second resident CTA per SM where that
+  // fits only while each split keeps >= 32 k-blocks.  Measured on B200: the
+  // second slot made 70B layers at M = 16..128 up to 30 % faster, while the
+  // 4096-deep 8B layers, cut into 8 to 11 k-blocks per split, ran slower.
   int64_t splits = 1;
-  if (tiles < sm && tiles <= kMaxSplitCounters) splits = std::max<int64_t>(1, std::min<int64_t>(sm / tiles, total_kb / 8));
+  if (tiles < sm && tiles <= kMaxSplitCounters)
+    splits = std::max<int64_t>(1, std::min<int64_t>(sm / tiles, total_kb / 8));
+  const int64_t slots = (int64_t)sm * tc_ctas_per_sm(p.bn, awq);
+  if (tiles < slots && tiles <= kMaxSplitCounters)
+    splits = std::max<int64_t>(splits, std::min<int64_t>(slots / tiles, total_kb / 32));
+  while (splits > 1 && kCounterBytes + (size_t)splits * M * N * 4 > ws_cap) --splits;
   int64_t kbps = cdiv(total_kb, splits);
   splits = cdiv(total_kb, kbps);
   p.splits = (int)splits;
@@ -295,19 +312,19 @@ bool gemv_fits(int64_t M, int64_t N, bool awq) {
   return M <= 8 && w4::gemv_supports(M, awq);
 }
 
-GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
+GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_cap) {
   int f = forced_path();
-  if (f == kPathTc) return plan_tc(M, N, K, sm);
+  if (f == kPathTc) return plan_tc(M, N, K, awq, sm, ws_cap);
   if (f == kPathGemv || gemv_fits(M, N, awq)) {
     const GemmPlan p = plan_gemv(M, N, K, awq, sm);
     if (p.path == kPathGemv || f == kPathGemv) return p;
   }
-  return plan_tc(M, N, K, sm);
+  return plan_tc(M, N, K, awq, sm, ws_cap);
 }
 
 // W4_DEBUG_PLAN=1 prints every launch plan to stderr (tuning aid).
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
-  GemmPlan p = plan_gemm_raw(M, N, K, awq, sm);
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_cap = SIZE_MAX) {
+  GemmPlan p = plan_gemm_raw(M, N, K, awq, sm, ws_cap);
   if (getenv("W4_DEBUG_PLAN")) {
     if (p.path == kPathGemv)
       fprintf(stderr,
@@ -322,7 +339,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
 }
 
 size_t ws_size_all(int64_t M, int64_t N, int64_t K, int sm) {
-  size_t ws = plan_tc(M, N, K, sm).ws_bytes;
+  size_t ws = std::max(plan_tc(M, N, K, false, sm).ws_bytes, plan_tc(M, N, K, true, sm).ws_bytes);
   if (M <= 64) {
     ws = std::max(ws, plan_gemv(M, N, K, false, sm).ws_bytes);
     if (M <= 32) ws = std::max(ws, plan_gemv(M, N, K, true, sm).ws_bytes);
@@ -434,7 +451,8 @@ namespace {
 w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K, int group,
                       const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros, const float *awq_s,
                       void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream,
-                      const int32_t *row_ptr, const int32_t *col, const uint16_t *val) {
+                      const int32_t *row_ptr, const int32_t *col, const uint16_t *val,
+                      size_t plan_ws_cap = SIZE_MAX) {
   t_last_error.clear();
   w4_status st = check_shape(M, N, K, group);
   if (st != W4_OK) return st;
@@ -454,7 +472,8 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const bool awq = awq_s != nullptr;
-  const GemmPlan plan = group == w4::kGroup ? plan_gemm(M, N, K, awq, sm) : plan_tc(M, N, K, sm);
+  const GemmPlan plan =
+      group == w4::kGroup ? plan_gemm(M, N, K, awq, sm, plan_ws_cap) : plan_tc(M, N, K, awq, sm, plan_ws_cap);
   if (plan.path == 0)
     return fail(W4_ERR_UNSUPPORTED, "W4_FORCE_PATH=gemv cannot serve N=%lld with K split into k-slices",
                 (long long)N);
@@ -653,7 +672,8 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
   int sm = 0;
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
-  const size_t need = plan_gemm(M, N, K, awq, sm).ws_bytes;
+  // The tensor-core plan takes fewer K splits where its partials would not fit.
+  const size_t need = plan_gemm(M, N, K, awq, sm, kStaticScratchBytes).ws_bytes;
   if (need > kStaticScratchBytes)
     return fail(W4_ERR_UNSUPPORTED,
                 "M=%lld N=%lld K=%lld needs %zu bytes of scratch; the static scratch holds %zu "
@@ -662,8 +682,8 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
   void *scratch = nullptr;
   e = static_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
-  return w4a16_gemm(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, scratch,
-                    kStaticScratchBytes, stream);
+  return gemm_common(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, scratch,
+                     kStaticScratchBytes, stream, nullptr, nullptr, nullptr, kStaticScratchBytes);
 }
 
 }  // extern "C"
