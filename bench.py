@@ -246,6 +246,33 @@ def _oracle_worker(rows, budget_s):
     return nbytes, time.perf_counter() - t0
 
 
+def _oracle_70b_worker(part, parts):
+    """One process of the whole-stack oracle estimate: rows [part/parts] of each Llama-3-70B
+    layer shape and of lm_head, dequant + fp64 matmul at M=1.  The codes, scales and zeros
+    are drawn uniformly (the oracle's time does not depend on their values).  Returns the
+    algorithmic bytes and seconds of its slice of one layer set, and of lm_head."""
+    import numpy as np
+    import oracle  # test/bench-only: the CPU baseline leg
+    torch.set_num_threads(1)
+    rng = np.random.default_rng(synthetic.seed_of("oracle70b", part, parts) % (2 ** 62))
+
+    def one(K, N):
+        n = N * (part + 1) // parts - N * part // parts
+        if n == 0:
+            return 0, 0.0
+        codes = rng.integers(0, 16, size=(n, K), dtype=np.uint8)
+        sc = (0.001 + 0.003 * rng.random((n, K // G), dtype=np.float32)).astype(np.float16)
+        zp = rng.integers(0, 16, size=(n, K // G)).astype(np.float16)
+        X = rng.standard_normal((1, K), dtype=np.float32)
+        t0 = time.perf_counter()
+        oracle.gemm(X, oracle.dequant(codes, sc, zp))
+        return gemm_bytes(1, n, K), time.perf_counter() - t0
+
+    layer = [one(K, N) for K, N in synthetic.SHAPES_70B.values()]
+    head = one(*synthetic.LM_HEAD_70B)
+    return sum(b for b, _ in layer), sum(t for _, t in layer), head[0], head[1]
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -266,11 +293,22 @@ def time_cpu_oracle_all_cores(budget_s=10.0, rows_per_layer=512):
     ctx = mp.get_context("spawn")
     with ctx.Pool(cores) as pool:
         res = pool.starmap(_oracle_worker, [(rows_per_layer, budget_s)] * cores)
+        res70 = pool.starmap(_oracle_70b_worker, [(i, cores) for i in range(cores)])
     nbytes = sum(r[0] for r in res)
     dt = max(r[1] for r in res)
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{cores} processes, each {rows_per_layer} output rows of each of the 4 Llama-3-8B layers "
-                      f"(dequant + fp64 matmul, M=1) for {budget_s:.0f} s; CPU: {cpu_model()}"}
+    eight_b = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{cores} processes, each {rows_per_layer} output rows of each of the 4 Llama-3-8B layers "
+                         f"(dequant + fp64 matmul, M=1) for {budget_s:.0f} s; CPU: {cpu_model()}"}
+    # Whole 70B stack at M=1: one full layer set and lm_head measured, the layers extrapolated x80.
+    n_layers = synthetic.N_LAYERS_70B
+    step_bytes = n_layers * sum(r[0] for r in res70) + sum(r[2] for r in res70)
+    step_s = max(n_layers * r[1] + r[3] for r in res70)
+    stack = {"value": step_bytes / step_s / 1e9, "unit": "GB/s", "ms_per_step": step_s * 1e3, "cores": cores,
+             "kind": "oracle",
+             "sample": f"one full Llama-3-70B layer set (qkv, o_proj, gate_up, down) and lm_head at M=1, rows split "
+                       f"over {cores} processes, dequant + fp64 matmul; the step time extrapolates the layer set "
+                       f"x{n_layers} plus lm_head"}
+    return eight_b, stack
 
 
 def run_reference(args):
@@ -696,7 +734,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_cpu_oracle()
-        extras["cpu_baseline_all_cores"] = time_cpu_oracle_all_cores()
+        extras["cpu_baseline_all_cores"], extras["cpu_baseline_stack70b"] = time_cpu_oracle_all_cores()
 
     if rank == 0:
         line = {
