@@ -271,9 +271,11 @@ size_t w4_gptq_workspace_size(int64_t N, int64_t K);
  * with no allocator of its own, a loop that must not take cudaMalloc).
  *   Arguments as for w4a16_gemm.  M <= 64, else W4_ERR_UNSUPPORTED.
  *   Scratch: a fixed array of w4a16_gemm_decode_static_capacity() bytes
- *   (8 MiB) per device, part of the library's own module.  A shape whose plan
- *   needs more returns W4_ERR_UNSUPPORTED with the sizes in w4_last_error()
- *   and launches nothing; use w4a16_gemm with a workspace for it.
+ *   (8 MiB) per device, part of the library's own module.  A tensor-core plan
+ *   takes fewer K splits where its fp32 partials would not fit it.  A decode
+ *   plan that needs more (its k-slices' partials) returns W4_ERR_UNSUPPORTED
+ *   with the sizes in w4_last_error() and launches nothing; use w4a16_gemm
+ *   with a workspace for it.
  *   The first call on a device looks up the scratch address on that device
  *   (the device must be current); make it before any stream capture.
  *   The scratch starts zero-filled and every completed call leaves its

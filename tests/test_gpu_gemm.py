@@ -141,6 +141,22 @@ def test_bf16_output(w4, path):
     _run_case(w4, 4, 512, 1024, path=path, out_dtype=torch.bfloat16, tag=("bf16out",))
 
 
+@pytest.mark.parametrize("M,N,K,awq,splits", [
+    (21, 256, 2688, True, 5),    # AWQ kernel (8 dequant warps): one batch of 4 splits and 1 more
+    (45, 384, 8192, False, 16),  # plain weights: four batches of 4 splits
+    (13, 130, 3200, False, 6),   # one batch and 2 more, ragged weight rows
+    (13, 130, 1536, False, 3),   # fewer splits than one batch
+])
+def test_split_k_reduction_ragged(w4, monkeypatch, capfd, M, N, K, awq, splits):
+    """Tensor-core split-K: the last CTA of each tile sums the fp32 partials in
+    batches of 4 splits plus a remainder, for token counts that are not multiples
+    of 8.  The plan printed with W4_DEBUG_PLAN confirms the split count."""
+    monkeypatch.setenv("W4_DEBUG_PLAN", "1")
+    _run_case(w4, M, N, K, awq=awq, tag=("splitk", M, N, K, awq))
+    err = capfd.readouterr().err
+    assert f"tensor-core: bn=64 splits={splits} " in err, err
+
+
 def test_long_k_split_both_paths(w4):
     """K = 28672 (70B down_proj depth) at small M: split-K on both paths."""
     for path in ("gemv", "tc"):
