@@ -399,8 +399,14 @@ def decode_leg(w4, layers, steps, warmup, world):
     with ClockSampler(torch.cuda.current_device()) as clk:
         ms = _replay_timed(g, stream)
     barrier(world)
+    # 20 more replays of the same graph, each timed alone, for the spread of the
+    # step time (the value is the single timed region of exactly `steps` steps).
+    reps = sorted(_replay_timed(g, stream) / steps for _ in range(20))
     del g
-    return ms, clk.summary()
+    repeats = {"n": 20, "steps_each": steps,
+               "median_ms_per_step": round(max_over_ranks(statistics.median(reps), world), 5),
+               "min_ms_per_step": round(reps[0], 5), "max_ms_per_step": round(reps[-1], 5)}
+    return ms, clk.summary(), repeats
 
 
 def dominant_leg(w4, layers, launches, warmup):
@@ -698,7 +704,7 @@ def main():
     layers = build_decode_state(w4, torch.device("cuda"))
     step_bytes = sum(gemm_bytes(1, layers[n]["N"], layers[n]["K"]) for n in LAYERS)
 
-    ms, clocks = decode_leg(w4, layers, args.steps, args.warmup, world)
+    ms, clocks, repeats = decode_leg(w4, layers, args.steps, args.warmup, world)
     value, ms = job_throughput(step_bytes * args.steps, ms, world)
 
     K, N = synthetic.SHAPES_8B[DOMINANT]
@@ -754,6 +760,7 @@ def main():
                     "api": "w4a16_gemm_host (pinned host X/Y, copies + sync inside the call)"},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
+            "repeats": repeats,
             "cpu_baseline": cpu,
         }
         line.update(extras)
