@@ -497,3 +497,130 @@ def test_gptq_lowers_the_layer_output_error():
     def err(c, s, z):
         return float(np.sum((X @ W.T - X @ oracle.dequant(c, s, z).T) ** 2))
     assert err(*oracle.gptq(W, X)) < 0.5 * err(*oracle.quantize(W))
+
+
+# ---------------------------------------------------------------- AWQ exponent search
+# The search (aiwing.uk ch. 22, section 22.3: s from calibration activation
+# magnitudes, W^ = quant(W / s) * s, a layer judged by ||X W^T - X W^^T||^2) is
+# pinned step by step against numpy routes that share nothing with the C loops:
+# the channel magnitude m_k, the exponent s = m^a, each exponent's output error
+# (quantization by the pinned quantizer, the products by BLAS), the argmin with
+# the first index on ties, and a constructed layer whose best exponent is known
+# by hand.
+
+def _search_numpy(W, X, alphas, group=G):
+    """Independent route: numpy magnitudes and powers, BLAS products in fp64."""
+    X64 = X.astype(np.float64)
+    m = np.abs(X64).mean(axis=0)  # one magnitude per input channel k
+    Yref = X64 @ W.astype(np.float64).T
+    errs, ss = [], []
+    for a in alphas:
+        s = np.where(m > 0, np.power(m, a), 1.0).astype(np.float32)
+        c, sc, zp = oracle.quantize(W, awq_s=s, group=group)
+        # W^ = (q - z) * scale * s, fp32 left to right, from the stored values
+        What = ((c.astype(np.float32) - np.repeat(zp.astype(np.float32), group, axis=1))
+                * np.repeat(sc.astype(np.float32), group, axis=1)) * s[None, :]
+        d = Yref - X64 @ What.astype(np.float64).T
+        errs.append(float(np.sum(d * d)))
+        ss.append(s)
+    return np.array(errs), ss, m
+
+
+def test_awq_search_magnitude_is_channel_mean_of_abs():
+    """With a = 1, s is m_k = mean over the calibration ROWS of |x_k| (fp64,
+    rounded to fp32).  Dyadic inputs make every sum exact, so the comparison
+    is bit for bit; a non-square X tells rows from channels apart."""
+    rng = np.random.default_rng(21)
+    Mc, K = 24, 256
+    X = (rng.integers(-64, 65, (Mc, K)) / 8.0).astype(np.float32)
+    X[:, 7] = 0.0  # a silent channel: m = 0, s must be 1
+    W = _weights(N=8, K=K, tag="awq-m")
+    _, s, best = oracle.awq_search(W, X, [1.0])
+    m = np.abs(X.astype(np.float64)).mean(axis=0)
+    want = np.where(m > 0, m, 1.0).astype(np.float32)
+    assert best == 0
+    assert np.array_equal(s, want)
+    assert s[7] == 1.0
+
+
+@pytest.mark.parametrize("a", [0.5, -0.3, 0.0, 1.0])
+def test_awq_search_scale_is_power_of_magnitude(a):
+    """s = m^a for the exponent returned, against numpy's power (1 fp32 ulp)."""
+    rng = np.random.default_rng(22)
+    X = rng.standard_normal((40, 128)).astype(np.float32) * np.exp(rng.uniform(-3, 3, 128)).astype(np.float32)
+    W = _weights(N=4, K=128, tag="awq-pow")
+    _, s, best = oracle.awq_search(W, X, [a])
+    m = np.abs(X.astype(np.float64)).mean(axis=0)
+    want = np.power(m, a).astype(np.float32)
+    assert best == 0
+    assert np.all(np.abs(s - want) <= np.spacing(np.abs(want)))
+    if a == 0.0:
+        assert np.all(s == 1.0)
+
+
+@pytest.mark.parametrize("group", [128, 64])
+def test_awq_search_errors_match_blas_route(group):
+    """Every exponent's error ||X W^T - X W^^T||_F^2 equals the numpy/BLAS route
+    (quantizer pinned above, products in fp64 by BLAS) to 1e-9 relative, and the
+    returned index is the argmin of those errors."""
+    rng = np.random.default_rng(23)
+    Mc, K, N = 48, 256, 24
+    X = rng.standard_normal((Mc, K)).astype(np.float32)
+    X[:, rng.choice(K, 3, replace=False)] *= 10.0  # heavy channels
+    W = _weights(N=N, K=K, outliers=0.0, tag=("awq-blas", group))
+    alphas = [-1.0, -0.5, -0.25, 0.0, 0.25, 0.5, 1.0]
+    errs, s, best = oracle.awq_search(W, X, alphas, group=group)
+    e_np, s_np, _ = _search_numpy(W, X, alphas, group=group)
+    assert np.allclose(errs, e_np, rtol=1e-9, atol=0.0), (errs, e_np)
+    assert best == int(np.argmin(e_np))
+    assert np.array_equal(s, s_np[best])
+    assert len(set(errs.tolist())) == len(alphas)  # the exponents really differ
+
+
+def test_awq_search_first_index_on_ties():
+    """Equal errors keep the first exponent: repeated exponents give bit-equal
+    errors, and channels of equal magnitude make every exponent's s the same."""
+    rng = np.random.default_rng(24)
+    X = rng.standard_normal((16, 128)).astype(np.float32)
+    X[:, 0] *= 10.0
+    W = _weights(N=6, K=128, tag="awq-tie")
+    errs, _, best = oracle.awq_search(W, X, [0.5, 0.0, 0.5, -0.5])
+    assert errs[0] == errs[2]
+    assert best == (0 if errs[0] <= min(errs[1], errs[3]) else int(np.argmin(errs)))
+    # |x| = 1 everywhere: m = 1, s = 1 for every exponent -> all errors equal -> index 0
+    Xs = np.where(rng.standard_normal((16, 128)) > 0, 1.0, -1.0).astype(np.float32)
+    errs, s, best = oracle.awq_search(W, Xs, [0.7, -0.2, 0.0])
+    assert errs[0] == errs[1] == errs[2]
+    assert best == 0 and np.all(s == 1.0)
+
+
+def test_awq_search_constructed_layer_prefers_positive_exponent():
+    """A layer built so that only a = 0.5 quantizes exactly.  Channels 0..3 are
+    heavy (|x| = 4, so m = 4 and s = 4^a), the rest have |x| = 1 (s = 1).  The
+    weights are W = g * s(0.5) with g on a power-of-two grid (scale 2^-6, zero 8,
+    codes 0 and 15 present, heavy values inside the range).  At a = 0.5, W / s = g
+    exactly, so W^ = W and the error is exactly 0; at a = 0 the heavy weights
+    leave the range, at a = 1 they fall halfway between grid points, at a < 0
+    they grow further: every other exponent has a positive error."""
+    K, N, Mc = 128, 3, 8
+    sc = 2.0 ** -6
+    rng = np.random.default_rng(25)
+    q = rng.integers(1, 15, (N, K))
+    q[:, 4] = 0
+    q[:, 5] = 15  # min and max codes present in every row: scale = sc, zero = 8
+    q[:, 0:4] = [13, 3, 11, 9]  # heavy channels: (q - 8) = 5, -5, 3, 1 (odd: halving leaves the grid)
+    g = (q - 8) * sc
+    s_true = np.ones(K)
+    s_true[0:4] = 2.0  # 4 ** 0.5
+    W = (g * s_true[None, :]).astype(np.float32)
+    signs = np.where(rng.standard_normal((Mc, K)) > 0, 1.0, -1.0)
+    X = (signs * np.where(np.arange(K) < 4, 4.0, 1.0)[None, :]).astype(np.float32)
+    alphas = [-1.0, -0.5, 0.0, 0.5, 1.0]
+    errs, s, best = oracle.awq_search(W, X, alphas)
+    assert alphas[best] == 0.5
+    assert errs[best] == 0.0
+    assert all(e > 0.0 for i, e in enumerate(errs) if i != best)
+    assert np.array_equal(s, s_true.astype(np.float32))
+    # the same ordering from the independent route
+    e_np, _, _ = _search_numpy(W, X, alphas)
+    assert int(np.argmin(e_np)) == best and e_np[best] == 0.0
