@@ -107,8 +107,9 @@ w4_status w4_quantize_symmetric(const void *W, w4_dtype w_dtype,
 
 /*
  * Pack one-code-per-byte codes [N][K] (device) into packed [N][K/2]
- * (device): low nibble = even k.  Values above 15 are masked to 4 bits.
- * K must be a positive multiple of 32.
+ * (device): two 4-bit codes per byte, 0.5 byte per parameter (ch. 22,
+ * section 22.3 table); low nibble = even k.  Values above 15 are masked to
+ * 4 bits.  K must be a positive multiple of 32.
  */
 w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed,
                   w4_stream_t stream);
@@ -138,7 +139,12 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N,
                      void *workspace, size_t workspace_bytes,
                      w4_stream_t stream);
 
-/* Bytes of workspace w4a16_gemm needs for this shape (0 if none). */
+/*
+ * Bytes of workspace w4a16_gemm needs for this shape (0 if none): split-K
+ * counters and fp32 partials of the fused dequantize-matmul (ch. 22, section
+ * 22.3).  Covers every plan the call may take for (M, N, K), with or without
+ * AWQ, for groups of 32, 64 or 128; 0 also for invalid sizes.
+ */
 size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -146,6 +152,8 @@ size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * (pinned host memory, [M][K]) into X_dev, runs w4a16_gemm, copies Y_dev
  * back into Y_host (pinned host memory, [M][N]) and waits for `stream`.
  * X_dev and Y_dev are caller-owned device staging buffers of the same sizes.
+ * The computation is w4a16_gemm's (ch. 22, section 22.3); the stream wait
+ * inside every call makes Y_host valid on return.
  */
 w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype,
                           int64_t M, int64_t N, int64_t K, int group,
@@ -197,7 +205,7 @@ size_t w4_awq_search_workspace_size(int64_t Mc, int64_t N, int64_t K,
  * exactly 0 and  W^ = dequant(dense) + sparse.
  *   W         device [N][K] fp32 (N*K < 2^31)
  *   awq_s, group, packed, scales, zeros   as for w4_quantize
- *   count     1 <= count <= N*K (for 0.1%: ceil(0.001 * N * K))
+ *   count     1 <= count <= N*K, or 0 for w4_outliers_default_count(N, K)
  *   row_ptr   device [N+1] int32 out: CSR row offsets by output row
  *   col, val  device [capacity] int32 / fp16 bit patterns out: the entries of
  *             each row in increasing k
@@ -215,8 +223,17 @@ w4_status w4_quantize_outliers(const float *W, const float *awq_s, int64_t N,
                                int64_t *nnz, void *workspace,
                                size_t workspace_bytes, w4_stream_t stream);
 
-/* Bytes of workspace w4_quantize_outliers needs for N rows. */
+/* Bytes of workspace w4_quantize_outliers needs for N rows (radix-select
+ * histograms and per-row counts of the split of the mhpq.cn article, 2.2). */
 size_t w4_outliers_workspace_size(int64_t N);
+
+/*
+ * Default outlier count of the dense + sparse split: the top 0.1 % of the
+ * weights (mhpq.cn practitioner's article, section 2.2), ceil(N * K / 1000),
+ * at least 1 (0 for invalid sizes).  w4_quantize_outliers uses it when given
+ * count = 0.
+ */
+int64_t w4_outliers_default_count(int64_t N, int64_t K);
 
 /*
  * w4a16_gemm on the dense part, then the sparse part added to Y:
@@ -264,20 +281,22 @@ w4_status w4_quantize_gptq(const float *W, int64_t N, int64_t K, int group,
 size_t w4_gptq_workspace_size(int64_t N, int64_t K);
 
 /*
- * Decode GEMM with library-owned scratch: the same computation, kernel and
- * result as w4a16_gemm for decode shapes, with no workspace argument.  The
- * source pages have no counterpart to this call; it exists for callers that
- * cannot allocate device memory where they run the layer (an engine plugin
- * with no allocator of its own, a loop that must not take cudaMalloc).
+ * Decode GEMM with library-owned scratch: the same computation and result as
+ * w4a16_gemm for decode shapes, with no workspace argument.  The source pages
+ * have no counterpart to this call; it exists for callers that cannot allocate
+ * device memory where they run the layer (an engine plugin with no allocator of
+ * its own, a loop that must not take cudaMalloc).
  *   Arguments as for w4a16_gemm.  M <= 64, else W4_ERR_UNSUPPORTED.
  *   Scratch: a fixed array of w4a16_gemm_decode_static_capacity() bytes
  *   (8 MiB) per device, part of the library's own module.  A tensor-core plan
- *   takes fewer K splits where its fp32 partials would not fit it.  A decode
- *   plan that needs more (its k-slices' partials) returns W4_ERR_UNSUPPORTED
- *   with the sizes in w4_last_error() and launches nothing; use w4a16_gemm
- *   with a workspace for it.
- *   The first call on a device looks up the scratch address on that device
- *   (the device must be current); make it before any stream capture.
+ *   takes fewer K splits where its fp32 partials would not fit it, and a
+ *   decode-kernel plan whose k-slice partials would not fit is replaced by that
+ *   tensor-core plan, so every M <= 64 shape is served.  (With the decode
+ *   kernel forced through W4_FORCE_PATH=gemv, such a plan returns
+ *   W4_ERR_UNSUPPORTED with the sizes in w4_last_error() and launches nothing.)
+ *   The first call in a CUDA context looks up the scratch address there (the
+ *   device must be current); make it before any stream capture.  A context that
+ *   is destroyed and created again (cudaDeviceReset) gets a fresh lookup.
  *   The scratch starts zero-filled and every completed call leaves its
  *   counters at zero.  Calls on one device share it: calls that overlap in
  *   time (other streams or threads) race on it and give wrong results.
@@ -296,14 +315,18 @@ size_t w4a16_gemm_decode_static_capacity(void);
 /*
  * Device-side error word: kernels whose bounded waits run out set it instead
  * of hanging.  Copies its value to *flag (0 = no error) and clears it; this
- * call synchronizes the current device.
+ * call synchronizes the current device.  Library error reporting: the pages
+ * define no counterpart.
  */
 w4_status w4_device_error(int *flag);
 
-/* Human-readable name of a status code (static string). */
+/* Human-readable name of a status code (static string).  Library error
+ * reporting: the pages define no counterpart. */
 const char *w4_status_string(w4_status status);
 
-/* Message of the last failed call on this thread ("" if none). */
+/* Message of the last failed call on this thread ("" if none), naming the
+ * argument or CUDA call that failed.  Library error reporting: the pages define
+ * no counterpart. */
 const char *w4_last_error(void);
 
 #ifdef __cplusplus

@@ -115,3 +115,16 @@ def test_workspace_size_plan(lib):
     # invalid shapes need none
     assert lib.w4a16_gemm_workspace_size(0, 16, 128) == 0
     assert lib.w4a16_gemm_workspace_size(1, 16, 100) == 0
+
+
+def test_outlier_default_count_is_top_tenth_percent(lib):
+    """The default count of the dense + sparse split is the top 0.1 % of the
+    weights (mhpq.cn practitioner's article, section 2.2): ceil(N K / 1000), at
+    least 1; a host-only helper, so it runs without a GPU."""
+    lib.w4_outliers_default_count.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    lib.w4_outliers_default_count.restype = ctypes.c_int64
+    f = lib.w4_outliers_default_count
+    assert f(4096, 4096) == 16778          # 16777216 / 1000 rounded up
+    assert f(28672, 4096) == 117441        # Llama-3-8B gate_up
+    assert f(1000, 1) == 1 and f(1001, 1) == 2 and f(1, 1) == 1
+    assert f(0, 128) == 0 and f(4, -1) == 0

