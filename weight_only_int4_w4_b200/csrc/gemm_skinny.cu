@@ -151,56 +151,62 @@ __device__ __forceinline__ uint32_t dq2(uint32_t w, uint32_t mask, uint32_t zc) 
 }
 
 // ------------------------------------------------------------------ main kernel
-// Warp roles (160 + 256 + 8 BN threads):
-//   warp 0        TMA producer (lanes 0..7 issue the boxes of every stage)
-//   warps 1..4    MMA issuers: issuer j = w - 1 owns TMEM A buffer j and
-//                 accumulator j, i.e. every 4th group (warp 1 also owns TMEM).
+// Warp roles (512 threads for BN <= 32, 640 above):
+//   warps 0..3    TMA producers: warp k issues the boxes of the stages
+//                 i = k (mod 4), lanes 0..5 one box each.  On B200 the boxes a
+//                 thread issues are in flight roughly one after another, so
+//                 stages issued by different warps are what overlaps.
+//   warps 4..7    MMA issuers: issuer j = w - 4 owns TMEM A buffer j and
+//                 accumulator j, i.e. every 4th group (warp 4 also owns TMEM).
 //                 A tcgen05.mma costs its issuing thread about 0.1 us on B200
 //                 whatever N is, so one issuer caps a 128-row x 16-channel MMA
 //                 stream far below the HBM rate; four issuers overlap.
-//   warps 5..12   dequantization: warp w serves TMEM lane quadrant w % 4 and
-//                 channels 64 h .. 64 h + 63 of every group, h = (w - 5) / 4
-//   warps 13..    promotion and epilogue, BN / 16 warps per quadrant: warp w
-//                 serves quadrant w % 4 and tokens 16 hp .. 16 hp + 15,
-//                 hp = (w - 13) / 4
+//   warps 8..11   dequantization: warp w serves TMEM lane quadrant w % 4, one
+//                 weight row per thread, all 128 channels of every group
+//   warps 12..    promotion and epilogue, one warp per quadrant (two for BN > 32):
+//                 warp w serves quadrant w % 4, one weight row and tokens
+//                 hp kTB .. hp kTB + kTB - 1 per thread, hp = (w - 12) / 4
 // The two sets run decoupled: dequantization runs up to kNA groups ahead of the
 // tensor core, promotion up to kNR groups behind it, and each set pays its TMEM
 // store (or load) wait once per two groups.
 constexpr int kNR = 4;                        // per-group accumulators in TMEM
-constexpr int kMmaWarps = 4;                  // warps 1..4
-constexpr int kDq0 = 32 * (1 + kMmaWarps);    // first dequantization thread (warp 5)
-constexpr int kDqThreads = 256;               // warps 5..12
-constexpr int kPr0 = kDq0 + kDqThreads;       // first promotion thread (warp 13)
-constexpr int kSZBox = kRows * 8 * 2;         // 8 groups x 128 rows of fp16 scales (or zeros)
+constexpr int kProdWarps = 4;                 // warps 0..3
+constexpr int kMmaWarps = 4;                  // warps 4..7
+constexpr int kMma0 = kProdWarps;             // first MMA warp
+constexpr int kDq0 = 32 * (kProdWarps + kMmaWarps);  // first dequantization thread (warp 8)
+constexpr int kDqThreads = 128;               // warps 8..11
+constexpr int kPr0 = kDq0 + kDqThreads;       // first promotion thread (warp 12)
 
 template <int BN>
 struct Cfg {
   static constexpr int kXStage = 4 * BN * 128;  // 4 boxes [BN tokens x 64 channels] fp16
-  static constexpr int kStage = kWStage + kXStage + 2 * kSZBox;
-  static constexpr int kNS = (229376 / kStage) > 8 ? 8 : (229376 / kStage);
+  static constexpr int kStage = kWStage + kXStage;
+  // ring depth: a multiple of the producer warps (each owns the stages i = k mod 4)
+  static constexpr int kNS = (229376 / kStage) >= 8 ? 8 : 4;
   static constexpr int kSmem = 1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + 64;
-  static constexpr int kTB = 16;                   // tokens promoted by each promotion thread
-  static constexpr int kPrThreads = 8 * BN;        // BN / 16 warps per lane quadrant
+  static constexpr int kPW = BN > 32 ? 2 : 1;  // promotion warps per lane quadrant
+  static constexpr int kTB = BN / kPW;         // tokens promoted by each promotion thread
+  static constexpr int kPrThreads = 128 * kPW;
   static constexpr int kThreads = kPr0 + kPrThreads;
   static_assert(kAccCol + kNR * BN <= 512, "TMEM columns");
   static_assert(kSmem <= 232448, "shared memory");
 };
 
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-      "%13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t &a, uint32_t &b, uint32_t &c,
-                                                  uint32_t &d) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "r"(taddr)
                : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
 }
 
 template <int kCount>
@@ -210,10 +216,9 @@ __device__ __forceinline__ void named_bar_pr() { asm volatile("bar.sync 1, %0;" 
 __device__ __forceinline__ int64_t sk_begin(int64_t c, int64_t T, int64_t C) { return (c * T) / C; }
 __device__ __forceinline__ int64_t sk_owner(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
 
-template <int BN, bool kScTma>
+template <int BN>
 __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                  const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
                   const SkinnyParams p) {
   using C_ = Cfg<BN>;
   constexpr int kNS = C_::kNS;
@@ -222,8 +227,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sW = smem;
   uint8_t *sX = smem + kNS * kWStage;
-  uint8_t *sSZ = sX + kNS * C_::kXStage;  // per stage: scales box, then zeros box
-  uint64_t *full = reinterpret_cast<uint64_t *>(sSZ + kNS * 2 * kSZBox);
+  uint64_t *full = reinterpret_cast<uint64_t *>(sX + kNS * C_::kXStage);
   uint64_t *empty = full + kNS;
   uint64_t *afull = empty + kNS;
   uint64_t *aempty = afull + kNA;
@@ -259,7 +263,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     }
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMma0) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -268,67 +272,58 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    // ---------------- TMA producer.  Lanes 0..7 each issue one box of every stage
-    // in the same instruction (the two 64-row halves of the codes, the four x'
-    // boxes, scales, zeros): boxes issued by one thread stream at well under the
-    // HBM rate on B200, boxes issued by separate lanes are in flight together.
-    if (lane < 8) {
-      if (lane == 0) {
+  if (warp < kProdWarps) {
+    // ---------------- TMA producers: warp k issues the stages i = k (mod 4) of the
+    // range; lanes 0, 1 the two 64-row halves of the codes, lanes 2..5 the four x'
+    // boxes.  Scales and zeros are not staged: read as 4-byte pairs by the warps
+    // that use them.
+    if (lane < 6) {
+      const int k = warp;
+      if (lane == 0 && k == 0) {
         prefetch_tensormap(&tmW);
         prefetch_tensormap(&tmX);
-        if (kScTma) {
-          prefetch_tensormap(&tmS);
-          prefetch_tensormap(&tmZ);
-        }
       }
-      // lane 0, 1: codes rows 64 lane ..; 2..5: x' box lane - 2; 6, 7: scales, zeros
       auto load_lane = [&](int i) {
         const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
         const int s = i % kNS;
         if (lane < 2) {
           tma_load_2d(sW + s * kWStage + lane * (kWStage / 2), &tmW, &full[s], (int32_t)(st * 128),
                       (int32_t)(rt * kRows + 64 * lane));
-        } else if (lane < 6) {
+        } else {
           const int b = lane - 2;
           tma_load_2d(sX + s * C_::kXStage + b * BN * 128, &tmX, &full[s], (int32_t)(st * 256 + 64 * b), 0);
-        } else if (kScTma) {
-          // the 8-group boxes that hold this stage's two groups (x = 2 st rounded down to 8)
-          const int32_t gx = (int32_t)((2 * st) & ~(int64_t)7);
-          tma_load_2d(sSZ + s * 2 * kSZBox + (lane - 6) * kSZBox, lane == 6 ? &tmS : &tmZ, &full[s], gx,
-                      (int32_t)(rt * kRows));
         }
       };
-      const bool x_lane = lane >= 2 && lane < 6;
-      // Weights and their scales never come from a preceding kernel: the first
-      // stages' boxes are requested before waiting for the staged activations.
+      const bool x_lane = lane >= 2;
+      // Weights never come from a preceding kernel: the first ring's codes are
+      // requested before waiting for the staged activations.
       const int pre = n_it < kNS ? n_it : kNS;
-      for (int i = 0; i < pre; ++i) {
-        if (lane == 0) mbar_arrive_expect_tx(&full[i % kNS], kScTma ? C_::kStage : C_::kStage - 2 * kSZBox);
-        __syncwarp(0xFFu);
+      for (int i = k; i < pre; i += kProdWarps) {
+        if (lane == 0) mbar_arrive_expect_tx(&full[i % kNS], C_::kStage);
+        __syncwarp(0x3Fu);
         if (!x_lane) load_lane(i);
       }
       grid_dependency_wait();
-      for (int i = 0; i < pre; ++i)
+      for (int i = k; i < pre; i += kProdWarps)
         if (x_lane) load_lane(i);
-      for (int i = pre; i < n_it; ++i) {
+      for (int i = pre + ((k - pre % kProdWarps + kProdWarps) % kProdWarps); i < n_it; i += kProdWarps) {
         const int s = i % kNS;
         // every issuing lane waits for the free slot itself; the vote keeps the
         // lanes on one path if a wait ever gives up
         const bool w_ok = mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, kErrTimeoutTma);
-        if (!__all_sync(0xFFu, w_ok)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], kScTma ? C_::kStage : C_::kStage - 2 * kSZBox);
-        __syncwarp(0xFFu);
+        if (!__all_sync(0x3Fu, w_ok)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], C_::kStage);
+        __syncwarp(0x3Fu);
         load_lane(i);
       }
       // every load of this CTA is issued: the next kernel in the stream may launch
       if (lane == 0) grid_launch_dependents();
     }
-  } else if (warp >= 1 && warp <= kMmaWarps) {
+  } else if (warp >= kMma0 && warp < kMma0 + kMmaWarps) {
     // ---------------- MMA issuers: issuer j issues the groups g = j (mod 4) of the
     // range (CTA-local group index g = 2 * stage + gi), into A buffer j and
     // accumulator j.
-    const int j = warp - 1;
+    const int j = warp - kMma0;
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(false, BN);
       const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * j);
@@ -353,30 +348,39 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         tc_commit(&empty[s]);
       }
     }
-  } else if (warp > kMmaWarps && warp < kPr0 / 32) {
+  } else if (warp >= kDq0 / 32 && warp < kPr0 / 32) {
     // ---------------- dequantization: 64 channels of every group for one weight row
     const int q = warp & 3;
-    const int h = (warp - kDq0 / 32) >> 2;
     const int rr = q * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    // the zero points of both groups of stage i (adjacent fp16, one 4-byte load),
+    // requested two stages ahead of use
+    auto pair_of = [&](const uint16_t *base, int i) -> uint32_t {
+      if (i >= n_it) return 0u;
+      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
+      const int64_t n = rt * kRows + rr;
+      if (n >= N) return 0u;
+      const int64_t kg = 2 * st;
+      const uint16_t *row = base + n * Kg;
+      if (kg + 1 < Kg && ((n * Kg + kg) & 1) == 0) return __ldg(reinterpret_cast<const uint32_t *>(row + kg));
+      const uint32_t lo = __ldg(row + kg);
+      const uint32_t hi = kg + 1 < Kg ? (uint32_t)__ldg(row + kg + 1) : 0u;
+      return lo | (hi << 16);
+    };
+    uint32_t zq0 = pair_of(p.zeros, 0), zq1 = pair_of(p.zeros, 1);
     int g = 0;
     for (int i = 0; i < n_it; ++i) {
-      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
-      const bool row_ok = rt * kRows + rr < N;
+      const uint32_t zpair = zq0;
+      zq0 = zq1;
+      zq1 = pair_of(p.zeros, i + 2);
       const int s = i % kNS;
       // A wait that gives up raises the device error word (later waits then give up
       // quickly); the loop runs to the end all the same.
       mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutDequant);
       const uint32_t wrow = smem_u32(sW + s * kWStage + rr * 128);
-      const uint32_t szrow = smem_u32(sSZ + s * 2 * kSZBox + rr * 16);
 #pragma unroll
       for (int gi = 0; gi < 2; ++gi) {
-        const int64_t kg = 2 * st + gi;
-        uint32_t z_bits = 0u;
-        if (kg < Kg && row_ok) {
-          if constexpr (kScTma) z_bits = lds_u16(szrow + kSZBox + (uint32_t)(kg & 7) * 2);
-          else z_bits = __ldg(p.zeros + (rt * kRows + rr) * Kg + kg);
-        }
+        const uint32_t z_bits = gi ? (zpair >> 16) : (zpair & 0xFFFFu);
         const int a = (g + gi) % kNA;
         mbar_wait(&aempty[a], ((uint32_t)((g + gi) / kNA) & 1u) ^ 1u, kErrTimeoutDequant);
         // zero-point constants 1024 + z (low nibbles) and 1024 + 16 z (high), both halves
@@ -386,22 +390,23 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         const __half2 hi2 = __hfma2(z2, __float2half2_rn(16.0f), __float2half2_rn(1024.0f));
         const uint32_t zlo = *reinterpret_cast<const uint32_t *>(&lo2);
         const uint32_t zhi = *reinterpret_cast<const uint32_t *>(&hi2);
-        // 32 bytes of this group's codes: logical chunks 4 gi + 2 h, + 1 (128-byte
-        // swizzle), 16 bytes (32 channels, 16 TMEM columns) at a time
+        // the group's 64 bytes of codes: logical chunks 4 gi .. 4 gi + 3 (128-byte
+        // swizzle), 32 bytes (64 channels, 32 TMEM columns) per store
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 u = lds128(wrow + (uint32_t)(((4 * gi + 2 * h + c) ^ (rr & 7)) << 4));
-          const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-          uint32_t out[16];
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint4 u0 = lds128(wrow + (uint32_t)(((4 * gi + 2 * hh) ^ (rr & 7)) << 4));
+          const uint4 u1 = lds128(wrow + (uint32_t)(((4 * gi + 2 * hh + 1) ^ (rr & 7)) << 4));
+          const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          uint32_t out[32];
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
+          for (int wi = 0; wi < 8; ++wi) {
             const uint32_t w = wv[wi], w8 = w >> 8;
             out[4 * wi + 0] = dq2(w, 0x000F000Fu, zlo);
             out[4 * wi + 1] = dq2(w, 0x00F000F0u, zhi);
             out[4 * wi + 2] = dq2(w8, 0x000F000Fu, zlo);
             out[4 * wi + 3] = dq2(w8, 0x00F000F0u, zhi);
           }
-          tmem_st_32x32b_x16(lane_base + (uint32_t)(64 * a + 32 * h + 16 * c), out);
+          tmem_st_32x32b_x32(lane_base + (uint32_t)(64 * a + 32 * hh), out);
         }
       }
       // one store wait for both groups of the stage
@@ -510,18 +515,13 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       const bool ok0 = mbar_wait(&accfull[r0], (uint32_t)(g / kNR) & 1u, kErrTimeoutEpilogue);
       const bool ok1 = mbar_wait(&accfull[r1], (uint32_t)((g + 1) / kNR) & 1u, kErrTimeoutEpilogue);
       tc_fence_after();
-      // 8 tokens at a time (registers): both groups' columns, one load wait
+      // 8 tokens at a time: both groups' columns (one 8-column load each), one wait
 #pragma unroll
       for (int c0 = 0; c0 < kTB; c0 += 8) {
+        const uint32_t col = (uint32_t)(kAccCol + tok0 + c0);
         uint32_t v0[8], v1[8];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t col = (uint32_t)(kAccCol + tok0 + c0 + 4 * c);
-          tmem_ld_32x32b_x4(lane_base + col + (uint32_t)(BN * r0), v0[4 * c], v0[4 * c + 1], v0[4 * c + 2],
-                            v0[4 * c + 3]);
-          tmem_ld_32x32b_x4(lane_base + col + (uint32_t)(BN * r1), v1[4 * c], v1[4 * c + 1], v1[4 * c + 2],
-                            v1[4 * c + 3]);
-        }
+        tmem_ld_32x32b_x8(lane_base + col + (uint32_t)(BN * r0), v0);
+        tmem_ld_32x32b_x8(lane_base + col + (uint32_t)(BN * r1), v1);
         tc_wait_ld();
         if (ok0 && ok1) {
 #pragma unroll
@@ -545,25 +545,30 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       __threadfence();
       const int64_t n = rt * kRows + rr;
       if (n < N) {
-        // slot by slot, every token's load of a slot in flight at once; the
-        // slots are summed in increasing order for every token
-        float acc[kTB];
+        // 8 tokens at a time, slot by slot, with every token's load of a slot in
+        // flight at once; the slots are summed in increasing order for every token
 #pragma unroll
-        for (int jj = 0; jj < kTB; ++jj) acc[jj] = 0.0f;
-        for (int sl = 0; sl < cnt; ++sl) {
-          float v[kTB];
+        for (int c0 = 0; c0 < kTB; c0 += 8) {
+          float acc[8];
 #pragma unroll
-          for (int jj = 0; jj < kTB; ++jj)
-            v[jj] = tok0 + jj < M ? __ldcg(p.ws + ((int64_t)sl * M + tok0 + jj) * N + n) : 0.0f;
+          for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
+          for (int sl = 0; sl < cnt; ++sl) {
+            float v[8];
 #pragma unroll
-          for (int jj = 0; jj < kTB; ++jj) acc[jj] += v[jj];
-        }
+            for (int jj = 0; jj < 8; ++jj) {
+              const int t = tok0 + c0 + jj;
+              v[jj] = t < M ? __ldcg(p.ws + ((int64_t)sl * M + t) * N + n) : 0.0f;
+            }
 #pragma unroll
-        for (int jj = 0; jj < kTB; ++jj) {
-          const int t = tok0 + jj;
-          if (t < M) {
-            if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[(int64_t)t * N + n] = __float2bfloat16_rn(acc[jj]);
-            else static_cast<float *>(p.Y)[(int64_t)t * N + n] = acc[jj];
+            for (int jj = 0; jj < 8; ++jj) acc[jj] += v[jj];
+          }
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int t = tok0 + c0 + jj;
+            if (t < M) {
+              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[(int64_t)t * N + n] = __float2bfloat16_rn(acc[jj]);
+              else static_cast<float *>(p.Y)[(int64_t)t * N + n] = acc[jj];
+            }
           }
         }
       }
@@ -573,7 +578,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMma0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -596,25 +601,18 @@ inline cudaError_t launch_pdl(const void *func, dim3 grid, dim3 block, size_t sm
   return cudaLaunchKernelExC(&cfg, func, args);
 }
 
-template <int BN, bool kScTma>
-cudaError_t launch_main(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
-                        const CUtensorMap &tmZ, const SkinnyParams &p, int grid, cudaStream_t stream) {
-  auto kern = skinny_kernel<BN, kScTma>;
+template <int BN>
+cudaError_t launch_main(const CUtensorMap &tmW, const CUtensorMap &tmX, const SkinnyParams &p, int grid,
+                        cudaStream_t stream) {
+  auto kern = skinny_kernel<BN>;
   static std::atomic<int> smem_set[kAttrDevices];
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), Cfg<BN>::kSmem, smem_set);
   if (e != cudaSuccess) return e;
-  CUtensorMap w = tmW, x = tmX, sc = tmS, z = tmZ;
+  CUtensorMap w = tmW, x = tmX;
   SkinnyParams pp = p;
-  void *args[] = {&w, &x, &sc, &z, &pp};
-  return launch_pdl(reinterpret_cast<const void *>(kern), dim3((unsigned)grid), dim3(Cfg<BN>::kThreads), Cfg<BN>::kSmem,
-                    stream, args);
-}
-
-template <int BN>
-cudaError_t launch_bn(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
-                      const CUtensorMap &tmZ, const SkinnyParams &p, int grid, bool sc_tma, cudaStream_t stream) {
-  return sc_tma ? launch_main<BN, true>(tmW, tmX, tmS, tmZ, p, grid, stream)
-                : launch_main<BN, false>(tmW, tmX, tmS, tmZ, p, grid, stream);
+  void *args[] = {&w, &x, &pp};
+  return launch_pdl(reinterpret_cast<const void *>(kern), dim3((unsigned)grid), dim3(Cfg<BN>::kThreads),
+                    Cfg<BN>::kSmem, stream, args);
 }
 
 }  // namespace sk_impl
@@ -636,13 +634,13 @@ cudaError_t launch_stage_x(const void *X, bool x_bf16, const float *awq_s, int64
   return launch_pdl(func, dim3((unsigned)M), dim3(256), 0, stream, args);
 }
 
-cudaError_t launch_skinny(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
-                          const CUtensorMap &tmZ, const SkinnyParams &p, int grid, bool sc_tma, cudaStream_t stream) {
+cudaError_t launch_skinny(const CUtensorMap &tmW, const CUtensorMap &tmX, const SkinnyParams &p, int grid,
+                          cudaStream_t stream) {
   switch (skinny_bn(p.M)) {
-    case 16: return sk_impl::launch_bn<16>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
-    case 32: return sk_impl::launch_bn<32>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
-    case 48: return sk_impl::launch_bn<48>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
-    default: return sk_impl::launch_bn<64>(tmW, tmX, tmS, tmZ, p, grid, sc_tma, stream);
+    case 16: return sk_impl::launch_main<16>(tmW, tmX, p, grid, stream);
+    case 32: return sk_impl::launch_main<32>(tmW, tmX, p, grid, stream);
+    case 48: return sk_impl::launch_main<48>(tmW, tmX, p, grid, stream);
+    default: return sk_impl::launch_main<64>(tmW, tmX, p, grid, stream);
   }
 }
 

@@ -573,25 +573,13 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
     if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for staged activations failed (CUresult %d)", (int)r);
     e = w4::launch_stage_x(X, xbf16, awq_s, M, K, xp, xexp, s);
     if (e != cudaSuccess) return cuda_fail(e, "activation staging launch");
-    // scales and zeros by TMA (8-group boxes of 128 rows) when rows start on 16-byte boundaries
-    const bool sc_tma = ((K / w4::kGroup) % 8) == 0;
-    CUtensorMap tmS = tmW, tmZ = tmW;
-    if (sc_tma) {
-      const uint64_t kg = (uint64_t)(K / w4::kGroup);
-      r = encode_2d(enc, &tmS, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, kg, (uint64_t)N, kg * 2, 8u, 128u,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
-      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for scales failed (CUresult %d)", (int)r);
-      r = encode_2d(enc, &tmZ, CU_TENSOR_MAP_DATA_TYPE_UINT16, zeros, kg, (uint64_t)N, kg * 2, 8u, 128u,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
-      if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for zeros failed (CUresult %d)", (int)r);
-    }
     w4::SkinnyParams p{};
     p.M = M; p.N = N; p.K = K;
     p.scales = scales; p.zeros = zeros;
     p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
     p.xexp = xexp; p.ws = reinterpret_cast<float *>(wsb + plan.part_off); p.counters = counters;
     p.slots = plan.slots;
-    e = w4::launch_skinny(tmW, tmXp, tmS, tmZ, p, plan.grid_x, sc_tma, s);
+    e = w4::launch_skinny(tmW, tmXp, p, plan.grid_x, s);
     if (e != cudaSuccess) return cuda_fail(e, "skinny gemm launch");
     if (row_ptr) {
       e = w4::launch_sparse_add(X, xbf16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16, s);
