@@ -9,9 +9,14 @@
 //   * H[a][b] = 2 sum_m x[m][a] x[m][b]  (m increasing); the diagonal gets
 //     damp = damp_frac * trace(H) / K added (trace summed in index order);
 //   * U, the upper Cholesky factor of H^-1, is P inv(L') P with L' the lower
-//     Cholesky factor of P H P (P reverses k): one Cholesky (one launch per
-//     column, parallel over rows, L' stored column-major) and one triangular
-//     inverse (one launch per row, parallel over columns);
+//     Cholesky factor of P H P (P reverses k).  Both factorizations are
+//     right-looking and blocked by panels of kPanel columns (rows): a one-CTA
+//     kernel finalizes the panel in order, then one launch applies the panel's
+//     updates to every trailing element.  Each element still receives its
+//     updates one at a time in increasing k -- exactly the sequential
+//     subtraction (Cholesky) and summation (inverse) of the plain loops:
+//       L'[i][j] = (R[i][j] - L'[i][0] L'[j][0] - ... - L'[i][j-1] L'[j][j-1]) / L'[j][j],
+//       inv[i][c] = -(0 + L'[i][c] inv[c][c] + ... + L'[i][i-1] inv[i-1][c]) / L'[i][i];
 //   * the column sweep: one warp per weight row, k = 0..K-1 in order; at each
 //     group start the scale and zero come from the current weights by the RTN
 //     rule (fp32, as in quantize.cu); err = (w - w^) / U[k][k] and every later
@@ -61,46 +66,115 @@ __global__ void damp_kernel(double *__restrict__ H, int64_t K, double damp_frac)
   for (int64_t a = 0; a < K; ++a) H[a * K + a] = __dadd_rn(H[a * K + a], damp);
 }
 
-// Column j of L' (lower Cholesky factor of R = P H P, R[i][j] = H[K-1-i][K-1-j]).
-// Lc is column-major: Lc[k * K + i] = L'[i][k].  Every thread recomputes the
-// pivot with the same operations, so all of them agree on it bit for bit.
-__global__ void __launch_bounds__(256) chol_col_kernel(const double *__restrict__ H, int64_t K, int64_t j,
-                                                       double *__restrict__ Lc, int *__restrict__ bad) {
-  const int64_t i = j + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= K) return;
-  double d = H[(K - 1 - j) * K + (K - 1 - j)];
-  for (int64_t k = 0; k < j; ++k) {
-    const double l = Lc[k * K + j];
-    d = __dsub_rn(d, __dmul_rn(l, l));
-  }
-  if (!(d > 0.0)) {
-    if (i == j) *bad = 1;
-    d = 1.0;  // keeps the values finite; the call reports the failure
-  }
-  const double ljj = __dsqrt_rn(d);
-  if (i == j) {
-    Lc[j * K + j] = ljj;
-    return;
-  }
-  double acc = H[(K - 1 - i) * K + (K - 1 - j)];
-  for (int64_t k = 0; k < j; ++k) acc = __dsub_rn(acc, __dmul_rn(Lc[k * K + i], Lc[k * K + j]));
-  Lc[j * K + i] = __ddiv_rn(acc, ljj);
+constexpr int kPanel = 8;     // columns (rows) per panel
+constexpr int kPanelThreads = 1024;
+
+// R = P H P into the lower triangle of A (row-major): A[i][j] = H[K-1-i][K-1-j], j <= i.
+__global__ void __launch_bounds__(256) reverse_kernel(const double *__restrict__ H, int64_t K, double *__restrict__ A) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= K * K) return;
+  const int64_t i = e / K, j = e - i * K;
+  if (j <= i) A[e] = H[(K - 1 - i) * K + (K - 1 - j)];
 }
 
-// Row i of Li = inv(L') (row-major), for columns c <= i:
-// Li[i][i] = 1 / L'[i][i];  Li[i][c] = -(sum_{k=c}^{i-1} L'[i][k] Li[k][c]) / L'[i][i].
-__global__ void __launch_bounds__(256) inv_row_kernel(const double *__restrict__ Lc, int64_t K, int64_t i,
-                                                      double *__restrict__ Li) {
-  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (c > i) return;
-  const double lii = Lc[i * K + i];
-  if (c == i) {
-    Li[i * K + i] = __ddiv_rn(1.0, lii);
-    return;
+__global__ void __launch_bounds__(256) zero_lower_kernel(double *__restrict__ A, int64_t K) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= K * K) return;
+  const int64_t i = e / K, j = e - i * K;
+  if (j <= i) A[e] = 0.0;
+}
+
+// Cholesky panel: columns j0 .. j0 + nb - 1 of A (updated through column j0 - 1)
+// become columns of L' in order; PT[jj][i] = L'[i][j0 + jj] is a transposed copy
+// for the trailing update's coalesced reads.  One CTA.
+__global__ void __launch_bounds__(kPanelThreads) chol_panel_kernel(double *__restrict__ A, int64_t K, int64_t j0,
+                                                                   int nb, double *__restrict__ PT,
+                                                                   int *__restrict__ bad) {
+  __shared__ double s_piv;
+  for (int jj = 0; jj < nb; ++jj) {
+    const int64_t c = j0 + jj;
+    if (threadIdx.x == 0) {
+      double d = A[c * K + c];
+      if (!(d > 0.0)) {
+        *bad = 1;
+        d = 1.0;  // keeps the values finite; the call reports the failure
+      }
+      const double l = __dsqrt_rn(d);
+      A[c * K + c] = l;
+      s_piv = l;
+    }
+    __syncthreads();
+    const double l = s_piv;
+    for (int64_t i = c + 1 + threadIdx.x; i < K; i += blockDim.x) {
+      const double v = __ddiv_rn(A[i * K + c], l);
+      A[i * K + c] = v;
+      PT[jj * K + i] = v;
+    }
+    __syncthreads();
+    // the rest of the panel: A[i][c'] -= L'[i][c] L'[c'][c], c < c' <= i
+    for (int cc = jj + 1; cc < nb; ++cc) {
+      const int64_t c2 = j0 + cc;
+      const double lc2 = A[c2 * K + c];
+      for (int64_t i = c2 + threadIdx.x; i < K; i += blockDim.x)
+        A[i * K + c2] = __dsub_rn(A[i * K + c2], __dmul_rn(A[i * K + c], lc2));
+    }
+    __syncthreads();
   }
-  double acc = 0.0;
-  for (int64_t k = c; k < i; ++k) acc = __dadd_rn(acc, __dmul_rn(Lc[k * K + i], Li[k * K + c]));
-  Li[i * K + c] = __ddiv_rn(-acc, lii);
+}
+
+// Cholesky trailing update: every A[i][c], c >= j1 = j0 + nb, i >= c, minus
+// L'[i][k] L'[c][k] for k = j0 .. j1 - 1 in increasing k.  blockIdx.x is the row
+// i - j1, blockIdx.y a tile of 256 columns; tiles right of the diagonal exit.
+__global__ void __launch_bounds__(256) chol_trail_kernel(double *__restrict__ A, const double *__restrict__ PT,
+                                                         int64_t K, int64_t j0, int nb) {
+  const int64_t j1 = j0 + nb;
+  const int64_t i = j1 + blockIdx.x, c = j1 + (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
+  if (c > i) return;
+  double a = A[i * K + c];
+  const double *li = A + i * K + j0;  // the same row for the whole CTA
+#pragma unroll
+  for (int k = 0; k < kPanel; ++k)
+    if (k < nb) a = __dsub_rn(a, __dmul_rn(li[k], PT[k * K + c]));
+  A[i * K + c] = a;
+}
+
+// Inverse panel: rows r0 .. r0 + nb - 1 of Li = inv(L') from their sums S (updated
+// through row r0 - 1): Li[r][c] = -S[r][c] / L'[r][r] for c < r, Li[r][r] = 1 / L'[r][r];
+// then the later rows of the panel add L'[r'][r] Li[r][c] to S[r'][c].  One CTA.
+__global__ void __launch_bounds__(kPanelThreads) inv_panel_kernel(const double *__restrict__ L, double *__restrict__ S,
+                                                                  int64_t K, int64_t r0, int nb,
+                                                                  double *__restrict__ Li) {
+  for (int rr = 0; rr < nb; ++rr) {
+    const int64_t r = r0 + rr;
+    const double lrr = L[r * K + r];
+    for (int64_t c = threadIdx.x; c <= r; c += blockDim.x)
+      Li[r * K + c] = c == r ? __ddiv_rn(1.0, lrr) : __ddiv_rn(-S[r * K + c], lrr);
+    __syncthreads();
+    for (int q = rr + 1; q < nb; ++q) {
+      const int64_t r2 = r0 + q;
+      const double l = L[r2 * K + r];
+      for (int64_t c = threadIdx.x; c <= r; c += blockDim.x)
+        S[r2 * K + c] = __dadd_rn(S[r2 * K + c], __dmul_rn(l, Li[r * K + c]));
+    }
+    __syncthreads();
+  }
+}
+
+// Inverse trailing update: every S[i][c], i >= r1 = r0 + nb, c < r1, plus
+// L'[i][k] Li[k][c] for k = max(c, r0) .. r1 - 1 in increasing k.  blockIdx.x is
+// the row i - r1, blockIdx.y a tile of 256 columns.
+__global__ void __launch_bounds__(256) inv_trail_kernel(const double *__restrict__ L, double *__restrict__ S,
+                                                        const double *__restrict__ Li, int64_t K, int64_t r0, int nb) {
+  const int64_t r1 = r0 + nb;
+  const int64_t i = r1 + blockIdx.x, c = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= r1) return;
+  double a = S[i * K + c];
+#pragma unroll
+  for (int k = 0; k < kPanel; ++k) {
+    const int64_t kk = r0 + k;
+    if (k < nb && kk >= c) a = __dadd_rn(a, __dmul_rn(L[i * K + kk], Li[kk * K + c]));
+  }
+  S[i * K + c] = a;
 }
 
 __device__ __forceinline__ float clamp15f(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
@@ -182,7 +256,8 @@ __global__ void __launch_bounds__(32 * kSweepRows) sweep_kernel(const float *__r
 }  // namespace gptq_impl
 
 // Hessian, damping, Cholesky and inverse: Li (row-major K x K) holds inv(L').
-// H, Lc, Li: K*K doubles each (Lc need not be zeroed: only its lower part is read);
+// H, Lc, Li: K*K doubles each (Lc need not be zeroed: only its lower part is
+// read; H is reused for the inverse's running sums once L' is formed);
 // bad: one int, zero on entry, set when H is not positive definite.
 cudaError_t launch_gptq_hinv(const void *X, bool x_bf16, int64_t Mc, int64_t K, double damp_frac, double *H,
                              double *Lc, double *Li, int *bad, cudaStream_t stream) {
@@ -192,9 +267,23 @@ cudaError_t launch_gptq_hinv(const void *X, bool x_bf16, int64_t Mc, int64_t K, 
   if (x_bf16) hessian_kernel<true><<<hg, kHT * kHT, 0, stream>>>(x, Mc, K, H);
   else hessian_kernel<false><<<hg, kHT * kHT, 0, stream>>>(x, Mc, K, H);
   damp_kernel<<<1, 32, 0, stream>>>(H, K, damp_frac);
-  for (int64_t j = 0; j < K; ++j)
-    chol_col_kernel<<<(unsigned)((K - j + 255) / 256), 256, 0, stream>>>(H, K, j, Lc, bad);
-  for (int64_t i = 0; i < K; ++i) inv_row_kernel<<<(unsigned)((i + 1 + 255) / 256), 256, 0, stream>>>(Lc, K, i, Li);
+  const unsigned sq = (unsigned)((K * K + 255) / 256);
+  reverse_kernel<<<sq, 256, 0, stream>>>(H, K, Lc);  // Lc: row-major, becomes L'
+  double *PT = Li;  // kPanel x K transposed panel; Li is written only after the Cholesky
+  for (int64_t j0 = 0; j0 < K; j0 += kPanel) {
+    const int nb = (int)std::min<int64_t>(kPanel, K - j0);
+    chol_panel_kernel<<<1, kPanelThreads, 0, stream>>>(Lc, K, j0, nb, PT, bad);
+    const int64_t T = K - j0 - nb;
+    if (T > 0) chol_trail_kernel<<<dim3((unsigned)T, (unsigned)((T + 255) / 256)), 256, 0, stream>>>(Lc, PT, K, j0, nb);
+  }
+  zero_lower_kernel<<<sq, 256, 0, stream>>>(H, K);  // H becomes the inverse's running sums
+  for (int64_t r0 = 0; r0 < K; r0 += kPanel) {
+    const int nb = (int)std::min<int64_t>(kPanel, K - r0);
+    inv_panel_kernel<<<1, kPanelThreads, 0, stream>>>(Lc, H, K, r0, nb, Li);
+    const int64_t rows = K - r0 - nb, r1 = r0 + nb;
+    if (rows > 0)
+      inv_trail_kernel<<<dim3((unsigned)rows, (unsigned)((r1 + 255) / 256)), 256, 0, stream>>>(Lc, H, Li, K, r0, nb);
+  }
   return cudaGetLastError();
 }
 
