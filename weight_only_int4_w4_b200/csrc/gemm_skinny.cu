@@ -60,25 +60,33 @@ namespace sk_impl {
 
 constexpr int kRows = 128;             // weight rows per tile = TMEM lanes
 constexpr int kWStage = kRows * 128;   // 16 KiB of codes per stage (2 groups)
-constexpr int kNA = 4;                 // TMEM A buffers, one group (64 columns) each
-constexpr int kAccCol = kNA * 64;      // first accumulator column
 
 
 // ------------------------------------------------------------------ staging of x'
-// One CTA of 256 threads per token.  Pass 1: max |x * s| over K; pass 2: x' in
-// the permuted order (see the file head).  Channels k = 8j + c (c = 0..7).
+// One CTA of 256 threads per token of the BN-token tile.  Pass 1: max |x * s|
+// over K; pass 2: x' in the permuted order (see the file head).  Channels
+// k = 8j + c (c = 0..7).  Layout: x'[k / 64][token][k % 64] (64-channel blocks,
+// BN tokens each), so one stage's 4 blocks x BN tokens are consecutive rows of
+// 128 bytes and arrive in one TMA box.  Tokens M..BN-1 are zeros.
 template <bool kBf16, bool kAwq>
 __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict__ X, const float *__restrict__ s,
-                                                      int64_t K, uint16_t *__restrict__ Xp, int *__restrict__ xexp) {
+                                                      int64_t M, int64_t K, int bn, uint16_t *__restrict__ Xp,
+                                                      int *__restrict__ xexp) {
   __shared__ float red[8];
   // The activations may be written by the preceding kernel, and x' may still be
   // read by the preceding matmul: wait for it, then let the matmul launch.
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
   const int64_t m = blockIdx.x;
-  const uint16_t *xr = X + m * K;
-  uint16_t *outr = Xp + m * K;
   const int64_t nb = K / 8;
+  // chunk j (channels 8j .. 8j + 7) of this token in the blocked layout
+  auto out_at = [&](int64_t j) { return Xp + ((j >> 3) * bn + m) * 64 + (j & 7) * 8; };
+  if (m >= M) {  // padding token of the tile
+    if (threadIdx.x == 0) xexp[m] = 0;
+    for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) *reinterpret_cast<uint4 *>(out_at(j)) = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const uint16_t *xr = X + m * K;
   auto load8 = [&](int64_t j, float (&v)[8]) {
     const uint4 u = __ldg(reinterpret_cast<const uint4 *>(xr + 8 * j));
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -134,7 +142,7 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict
     o.y = *reinterpret_cast<const uint32_t *>(&h1);
     o.z = *reinterpret_cast<const uint32_t *>(&h2);
     o.w = *reinterpret_cast<const uint32_t *>(&h3);
-    *reinterpret_cast<uint4 *>(outr + 8 * j) = o;
+    *reinterpret_cast<uint4 *>(out_at(j)) = o;
   }
 }
 
@@ -145,6 +153,15 @@ __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
   return r;
 }
 
+// 4-byte asynchronous copy global -> shared (both 4-byte aligned); completion is
+// tracked per thread with commit / wait groups.
+__device__ __forceinline__ void cp_async4(uint32_t saddr, const void *gaddr) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(saddr), "l"(gaddr) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+
 // Exact fp16 pair: (w & mask) | 1024.0 minus zc (1024 + z, or 1024 + 16 z for the high nibbles).
 __device__ __forceinline__ uint32_t dq2(uint32_t w, uint32_t mask, uint32_t zc) {
   return hsub2_u32(lop3_and_or(w, mask, 0x64006400u), zc);
@@ -152,10 +169,10 @@ __device__ __forceinline__ uint32_t dq2(uint32_t w, uint32_t mask, uint32_t zc) 
 
 // ------------------------------------------------------------------ main kernel
 // Warp roles (512 threads for BN <= 32, 640 above):
-//   warps 0..3    TMA producers: warp k issues the boxes of the stages
-//                 i = k (mod 4), lanes 0..5 one box each.  On B200 the boxes a
-//                 thread issues are in flight roughly one after another, so
-//                 stages issued by different warps are what overlaps.
+//   warps 0..3    TMA producers: warp k issues the stages i = k (mod 4), lane 0
+//                 the codes box, lane 1 the x' box.  The boxes one thread issues
+//                 are in flight roughly one after another, so stages issued by
+//                 different warps are what overlaps.
 //   warps 4..7    MMA issuers: issuer j = w - 4 owns TMEM A buffer j and
 //                 accumulator j, i.e. every 4th group (warp 4 also owns TMEM).
 //                 A tcgen05.mma costs its issuing thread about 0.1 us on B200
@@ -166,27 +183,89 @@ __device__ __forceinline__ uint32_t dq2(uint32_t w, uint32_t mask, uint32_t zc) 
 //   warps 12..    promotion and epilogue, one warp per quadrant (two for BN > 32):
 //                 warp w serves quadrant w % 4, one weight row and tokens
 //                 hp kTB .. hp kTB + kTB - 1 per thread, hp = (w - 12) / 4
+// TMEM holds kNA A buffers (64 columns, one group, each) then kNR accumulators of
+// BN columns; kNA is as many as fit (7 at BN = 16 down to 4 at BN = 64).  A buffer
+// goes round dequantization, hand-off, eight MMA issues and their completion
+// (about 1.2 us), so the buffer count sets how many groups are in flight.  Groups
+// take buffers g mod kNA; dequantization fills them in group order and each issuer
+// takes its groups in order, so no waiter runs two barrier phases ahead.
 // The two sets run decoupled: dequantization runs up to kNA groups ahead of the
 // tensor core, promotion up to kNR groups behind it, and each set pays its TMEM
 // store (or load) wait once per two groups.
 constexpr int kNR = 4;                        // per-group accumulators in TMEM
+// Scales and zeros are copied kPf stages ahead of use into a per-thread ring in
+// shared memory (cp.async): under a full HBM stream a global load takes about a
+// microsecond, several stages.  (A register queue does not work: rotating it
+// copies the register of the most recent load and waits for that load.)
+constexpr int kPf = 8;
 constexpr int kProdWarps = 4;                 // warps 0..3
+constexpr int kMma0 = kProdWarps;             // first MMA warp (TMEM owner)
 constexpr int kMmaWarps = 4;                  // warps 4..7
-constexpr int kMma0 = kProdWarps;             // first MMA warp
 constexpr int kDq0 = 32 * (kProdWarps + kMmaWarps);  // first dequantization thread (warp 8)
 constexpr int kDqThreads = 128;               // warps 8..11
 constexpr int kPr0 = kDq0 + kDqThreads;       // first promotion thread (warp 12)
 
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+
+// Walks the stages of a CTA's range in order and copies, for weight row rr of
+// each stage's tile, the adjacent fp16 pair of the stage's two groups (scales or
+// zero points) into ring slot (stage mod kPf) at `slot0 + slot * slot_stride`
+// bytes.  One cp.async group is committed per stage, so cp.async.wait_group
+// kPf - 1 makes the oldest stage's copy visible.  Rows past N, stages past the
+// range and a group past Kg give 0; a pair that is not 4-byte aligned (Kg odd)
+// is read with plain loads.
+struct PairFetcher {
+  const uint16_t *base;
+  int N, Kg, S, n_it, i, rr;  // N < 2^31 and Kg < 2^31 (the planner's limits)
+  int rt, st;                 // tile and stage of fetch i
+  uint32_t slot0, stride;
+  __device__ PairFetcher(const uint16_t *b, int64_t it0, int n, int64_t S_, int64_t N_, int64_t Kg_, int r,
+                         uint32_t s0, uint32_t str)
+      : base(b), N((int)N_), Kg((int)Kg_), S((int)S_), n_it(n), i(0), rr(r), slot0(s0), stride(str) {
+    rt = (int)(it0 / S_);
+    st = (int)(it0 - (int64_t)rt * S_);
+  }
+  __device__ __forceinline__ void next() {
+    const uint32_t dst = slot0 + (uint32_t)(i % kPf) * stride;
+    if (i < n_it) {
+      const int n = rt * kRows + rr, kg = 2 * st;
+      const int64_t off = (int64_t)n * Kg + kg;
+      if (n < N && kg + 1 < Kg && (off & 1) == 0) {
+        cp_async4(dst, base + off);
+      } else {
+        uint32_t v = 0u;
+        if (n < N) v = (uint32_t)__ldg(base + off) | (kg + 1 < Kg ? (uint32_t)__ldg(base + off + 1) << 16 : 0u);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(v) : "memory");
+      }
+      if (++st == S) {
+        st = 0;
+        ++rt;
+      }
+    }
+    cp_async_commit();  // one group per stage, empty past the range
+    ++i;
+  }
+};
+
 template <int BN>
 struct Cfg {
-  static constexpr int kXStage = 4 * BN * 128;  // 4 boxes [BN tokens x 64 channels] fp16
+  static constexpr int kXStage = 4 * BN * 128;  // 4 blocks [BN tokens x 64 channels] fp16, one box
   static constexpr int kStage = kWStage + kXStage;
   // ring depth: a multiple of the producer warps (each owns the stages i = k mod 4)
   static constexpr int kNS = (229376 / kStage) >= 8 ? 8 : 4;
-  static constexpr int kSmem = 1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + 64;
   static constexpr int kPW = BN > 32 ? 2 : 1;  // promotion warps per lane quadrant
   static constexpr int kTB = BN / kPW;         // tokens promoted by each promotion thread
   static constexpr int kPrThreads = 128 * kPW;
+  // rings of zero-point pairs [kPf][dequantization threads] and scale pairs [kPf][promotion threads]
+  static constexpr int kRingBytes = kPf * kDqThreads * 4 + kPf * kPrThreads * 4;
+  static constexpr int kNA = (512 - kNR * BN) / 64;  // TMEM A buffers
+  static constexpr int kAccCol = 64 * kNA;          // first accumulator column
+  static constexpr int kSmem =
+      1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + kRingBytes + 64;
   static constexpr int kThreads = kPr0 + kPrThreads;
   static_assert(kAccCol + kNR * BN <= 512, "TMEM columns");
   static_assert(kSmem <= 232448, "shared memory");
@@ -221,6 +300,8 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                   const SkinnyParams p) {
   using C_ = Cfg<BN>;
+  constexpr int kNA = C_::kNA;
+  constexpr int kAccCol = C_::kAccCol;
   constexpr int kNS = C_::kNS;
   constexpr int kTB = C_::kTB;
   extern __shared__ uint8_t smem_raw[];
@@ -236,6 +317,8 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accempty + kNR);
   int *s_ticket = reinterpret_cast<int *>(tmem_holder + 1);       // [2]
   float *s_escale = reinterpret_cast<float *>(tmem_holder + 4);  // [64] 2^-e per token
+  uint32_t *zring = reinterpret_cast<uint32_t *>(s_escale + 64);  // [kPf][kDqThreads]
+  uint32_t *sring = zring + kPf * kDqThreads;                     // [kPf][kPrThreads]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -254,12 +337,12 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       mbar_init(&empty[s], 2);  // one commit per group, from that group's issuer
     }
     for (int a = 0; a < kNA; ++a) {
-      mbar_init(&afull[a], kDqThreads);
+      mbar_init(&afull[a], kDqThreads / 32);  // one arrival per dequantization warp
       mbar_init(&aempty[a], 1);
     }
     for (int r = 0; r < kNR; ++r) {
       mbar_init(&accfull[r], 1);
-      mbar_init(&accempty[r], C_::kPrThreads);
+      mbar_init(&accempty[r], C_::kPrThreads / 32);  // one arrival per promotion warp
     }
     fence_barrier_init();
   }
@@ -272,107 +355,93 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp < kProdWarps) {
-    // ---------------- TMA producers: warp k issues the stages i = k (mod 4) of the
-    // range; lanes 0, 1 the two 64-row halves of the codes, lanes 2..5 the four x'
-    // boxes.  Scales and zeros are not staged: read as 4-byte pairs by the warps
-    // that use them.
-    if (lane < 6) {
-      const int k = warp;
-      if (lane == 0 && k == 0) {
-        prefetch_tensormap(&tmW);
-        prefetch_tensormap(&tmX);
-      }
-      auto load_lane = [&](int i) {
-        const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
-        const int s = i % kNS;
-        if (lane < 2) {
-          tma_load_2d(sW + s * kWStage + lane * (kWStage / 2), &tmW, &full[s], (int32_t)(st * 128),
-                      (int32_t)(rt * kRows + 64 * lane));
-        } else {
-          const int b = lane - 2;
-          tma_load_2d(sX + s * C_::kXStage + b * BN * 128, &tmX, &full[s], (int32_t)(st * 256 + 64 * b), 0);
-        }
-      };
-      const bool x_lane = lane >= 2;
-      // Weights never come from a preceding kernel: the first ring's codes are
-      // requested before waiting for the staged activations.
-      const int pre = n_it < kNS ? n_it : kNS;
-      for (int i = k; i < pre; i += kProdWarps) {
-        if (lane == 0) mbar_arrive_expect_tx(&full[i % kNS], C_::kStage);
-        __syncwarp(0x3Fu);
-        if (!x_lane) load_lane(i);
-      }
-      grid_dependency_wait();
-      for (int i = k; i < pre; i += kProdWarps)
-        if (x_lane) load_lane(i);
-      for (int i = pre + ((k - pre % kProdWarps + kProdWarps) % kProdWarps); i < n_it; i += kProdWarps) {
-        const int s = i % kNS;
-        // every issuing lane waits for the free slot itself; the vote keeps the
-        // lanes on one path if a wait ever gives up
-        const bool w_ok = mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, kErrTimeoutTma);
-        if (!__all_sync(0x3Fu, w_ok)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], C_::kStage);
-        __syncwarp(0x3Fu);
-        load_lane(i);
-      }
-      // every load of this CTA is issued: the next kernel in the stream may launch
-      if (lane == 0) grid_launch_dependents();
+  if (warp < kProdWarps && lane < 2) {
+    // ---------------- TMA producer k = w: the stages i = k (mod 4) of the range;
+    // lane 0 the codes (one box of 128 rows x 128 bytes), lane 1 the x' of the
+    // stage (one box of 4 BN rows).  On B200 the TMA unit works through small
+    // boxes one after another at a fixed cost each, so a stage is two boxes.
+    // Scales and zeros are not staged: the warps that use them copy 4-byte pairs
+    // ahead of use.
+    const int k = warp;
+    if (lane == 0 && k == 0) {
+      prefetch_tensormap(&tmW);
+      prefetch_tensormap(&tmX);
     }
-  } else if (warp >= kMma0 && warp < kMma0 + kMmaWarps) {
-    // ---------------- MMA issuers: issuer j issues the groups g = j (mod 4) of the
-    // range (CTA-local group index g = 2 * stage + gi), into A buffer j and
+    const bool x_lane = lane == 1;
+    auto load_lane = [&](int i) {
+      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
+      const int s = i % kNS;
+      if (!x_lane) {
+        tma_load_2d(sW + s * kWStage, &tmW, &full[s], (int32_t)(st * 128), (int32_t)(rt * kRows));
+      } else {
+        tma_load_2d(sX + s * C_::kXStage, &tmX, &full[s], 0, (int32_t)(st * 4 * BN));
+      }
+    };
+    // Weights never come from a preceding kernel: the first ring's codes are
+    // requested before waiting for the staged activations.
+    const int pre = n_it < kNS ? n_it : kNS;
+    for (int i = k; i < pre; i += kProdWarps) {
+      if (!x_lane) mbar_arrive_expect_tx(&full[i % kNS], C_::kStage);
+      __syncwarp(0x3u);
+      if (!x_lane) load_lane(i);
+    }
+    grid_dependency_wait();
+    for (int i = k; i < pre; i += kProdWarps)
+      if (x_lane) load_lane(i);
+    for (int i = pre + ((k - pre % kProdWarps + kProdWarps) % kProdWarps); i < n_it; i += kProdWarps) {
+      const int s = i % kNS;
+      // both lanes wait for the free slot; the vote keeps them on one path if a
+      // wait ever gives up
+      const bool w_ok = mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, kErrTimeoutTma);
+      if (!__all_sync(0x3u, w_ok)) break;
+      if (!x_lane) mbar_arrive_expect_tx(&full[s], C_::kStage);
+      __syncwarp(0x3u);
+      load_lane(i);
+    }
+    // every load of this CTA is issued: the next kernel in the stream may launch
+    if (!x_lane) grid_launch_dependents();
+  } else if (warp >= kMma0 && warp < kMma0 + kMmaWarps && lane == 0) {
+    // ---------------- MMA issuer j = w - 4: the groups g = j (mod 4) of the range
+    // (CTA-local group index g = 2 * stage + gi), from A buffer g mod kNA into
     // accumulator j.
     const int j = warp - kMma0;
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16(false, BN);
-      const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * j);
-      const uint32_t a_tmem = tmem + (uint32_t)(64 * j);
-      int n = 0;  // groups issued by this issuer
-      for (int g = j; g < 2 * n_it; g += kNR, ++n) {
-        const int i = g >> 1, gi = g & 1;
-        const int s = i % kNS;
-        if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutMma)) break;
-        if (!mbar_wait(&afull[j], (uint32_t)n & 1u, kErrTimeoutMma)) break;
-        if (!mbar_wait(&accempty[j], ((uint32_t)n & 1u) ^ 1u, kErrTimeoutMma)) break;
-        tc_fence_after();
-        const uint32_t xs = smem_u32(sX + s * C_::kXStage);
+    const uint32_t idesc = idesc_f16(false, BN);
+    const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * j);
+    int n = 0;  // groups issued by this issuer
+    for (int g = j; g < 2 * n_it; g += kNR, ++n) {
+      const int i = g >> 1, gi = g & 1;
+      const int s = i % kNS;
+      const int a = g % kNA;
+      const uint32_t a_tmem = tmem + (uint32_t)(64 * a);
+      if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutMma)) break;
+      if (!mbar_wait(&afull[a], (uint32_t)(g / kNA) & 1u, kErrTimeoutMma)) break;
+      if (!mbar_wait(&accempty[j], ((uint32_t)n & 1u) ^ 1u, kErrTimeoutMma)) break;
+      tc_fence_after();
+      const uint32_t xs = smem_u32(sX + s * C_::kXStage);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int b = 2 * gi + (k >> 2);
-          const uint64_t bdesc = smem_desc_k_sw128(xs + (uint32_t)(b * BN * 128)) + (uint64_t)(2 * (k & 3));
-          tc_mma_ts(d_tmem, a_tmem + 8 * k, bdesc, idesc, k > 0 ? 1u : 0u);
-        }
-        tc_commit(&aempty[j]);
-        tc_commit(&accfull[j]);
-        tc_commit(&empty[s]);
+      for (int kk = 0; kk < 8; ++kk) {
+        const int b = 2 * gi + (kk >> 2);
+        const uint64_t bdesc = smem_desc_k_sw128(xs + (uint32_t)(b * BN * 128)) + (uint64_t)(2 * (kk & 3));
+        tc_mma_ts(d_tmem, a_tmem + 8 * kk, bdesc, idesc, kk > 0 ? 1u : 0u);
       }
+      tc_commit(&aempty[a]);
+      tc_commit(&accfull[j]);
+      tc_commit(&empty[s]);
     }
   } else if (warp >= kDq0 / 32 && warp < kPr0 / 32) {
-    // ---------------- dequantization: 64 channels of every group for one weight row
+    // ---------------- dequantization: all 128 channels of every group for one weight row
     const int q = warp & 3;
     const int rr = q * 32 + lane;
+    const int dt = threadIdx.x - kDq0;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    // the zero points of both groups of stage i (adjacent fp16, one 4-byte load),
-    // requested two stages ahead of use
-    auto pair_of = [&](const uint16_t *base, int i) -> uint32_t {
-      if (i >= n_it) return 0u;
-      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
-      const int64_t n = rt * kRows + rr;
-      if (n >= N) return 0u;
-      const int64_t kg = 2 * st;
-      const uint16_t *row = base + n * Kg;
-      if (kg + 1 < Kg && ((n * Kg + kg) & 1) == 0) return __ldg(reinterpret_cast<const uint32_t *>(row + kg));
-      const uint32_t lo = __ldg(row + kg);
-      const uint32_t hi = kg + 1 < Kg ? (uint32_t)__ldg(row + kg + 1) : 0u;
-      return lo | (hi << 16);
-    };
-    uint32_t zq0 = pair_of(p.zeros, 0), zq1 = pair_of(p.zeros, 1);
+    // the zero points of both groups of a stage (adjacent fp16) go to this
+    // thread's ring slot (stage mod kPf), kPf stages ahead of use
+    PairFetcher zf(p.zeros, it0, n_it, S, N, Kg, rr, smem_u32(zring) + 4u * (uint32_t)dt, kDqThreads * 4);
+    for (int d = 0; d < kPf; ++d) zf.next();
     int g = 0;
     for (int i = 0; i < n_it; ++i) {
-      const uint32_t zpair = zq0;
-      zq0 = zq1;
-      zq1 = pair_of(p.zeros, i + 2);
+      cp_async_wait<kPf - 1>();  // this thread's copies for stage i have landed
+      const uint32_t zpair = ld_shared_u32(smem_u32(zring) + 4u * (uint32_t)((i % kPf) * kDqThreads + dt));
       const int s = i % kNS;
       // A wait that gives up raises the device error word (later waits then give up
       // quickly); the loop runs to the end all the same.
@@ -390,6 +459,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         const __half2 hi2 = __hfma2(z2, __float2half2_rn(16.0f), __float2half2_rn(1024.0f));
         const uint32_t zlo = *reinterpret_cast<const uint32_t *>(&lo2);
         const uint32_t zhi = *reinterpret_cast<const uint32_t *>(&hi2);
+        if (gi == 1) zf.next();  // stage i's pair is consumed: its slot takes stage i + kPf
         // the group's 64 bytes of codes: logical chunks 4 gi .. 4 gi + 3 (128-byte
         // swizzle), 32 bytes (64 channels, 32 TMEM columns) per store
 #pragma unroll
@@ -412,8 +482,14 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       // one store wait for both groups of the stage
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&afull[g % kNA]);
-      mbar_arrive(&afull[(g + 1) % kNA]);
+      // One arrival per warp: an mbarrier arrive is a read-modify-write of one
+      // shared-memory word, and 256 of them per group serialize into a fixed cost
+      // per stage larger than the stage's work.
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&afull[g % kNA]);
+        mbar_arrive(&afull[(g + 1) % kNA]);
+      }
       g += 2;
     }
   } else if (warp >= kPr0 / 32) {
@@ -433,21 +509,11 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     float y[kTB];
 #pragma unroll
     for (int j = 0; j < kTB; ++j) y[j] = 0.0f;
-    // The scales of both groups of stage i (adjacent fp16, one 4-byte load),
-    // requested two stages ahead of use.
-    auto scales_of = [&](int i) -> uint32_t {
-      if (i >= n_it) return 0u;
-      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
-      const int64_t n = rt * kRows + rr;
-      if (n >= N) return 0u;
-      const int64_t kg = 2 * st;
-      const uint16_t *row = p.scales + n * Kg;
-      if (kg + 1 < Kg && ((n * Kg + kg) & 1) == 0) return __ldg(reinterpret_cast<const uint32_t *>(row + kg));
-      const uint32_t lo = __ldg(row + kg);
-      const uint32_t hi = kg + 1 < Kg ? (uint32_t)__ldg(row + kg + 1) : 0u;
-      return lo | (hi << 16);
-    };
-    uint32_t scq0 = scales_of(0), scq1 = scales_of(1);
+    // The scales of both groups of a stage (adjacent fp16) go to this thread's
+    // ring slot (stage mod kPf), kPf stages ahead of use.
+    const int pt = threadIdx.x - kPr0;
+    PairFetcher sf(p.scales, it0, n_it, S, N, Kg, rr, smem_u32(sring) + 4u * (uint32_t)pt, C_::kPrThreads * 4);
+    for (int d = 0; d < kPf; ++d) sf.next();
 
     // Split-tile bookkeeping: at most two pieces of a CTA's range are partial
     // (its first and its last tile); their tickets are resolved at the end.
@@ -505,11 +571,11 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         if (cur_rt >= 0) finish_piece(cur_rt);
         cur_rt = rt;
       }
-      const uint32_t scb = scq0;
-      scq0 = scq1;
-      scq1 = scales_of(i + 2);
+      cp_async_wait<kPf - 1>();  // this thread's copies for stage i have landed
+      const uint32_t scb = ld_shared_u32(smem_u32(sring) + 4u * (uint32_t)((i % kPf) * C_::kPrThreads + pt));
       const float sc0 = __half2float(__ushort_as_half((unsigned short)(scb & 0xFFFFu)));
       const float sc1 = __half2float(__ushort_as_half((unsigned short)(scb >> 16)));
+      sf.next();  // stage i's pair is consumed: its slot takes stage i + kPf
       // both groups' accumulators, one load wait
       const int r0 = g % kNR, r1 = (g + 1) % kNR;
       const bool ok0 = mbar_wait(&accfull[r0], (uint32_t)(g / kNR) & 1u, kErrTimeoutEpilogue);
@@ -530,8 +596,11 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&accempty[r0]);
-      mbar_arrive(&accempty[r1]);
+      __syncwarp();
+      if (lane == 0) {  // one arrival per warp (see the dequantization warps)
+        mbar_arrive(&accempty[r0]);
+        mbar_arrive(&accempty[r1]);
+      }
       g += 2;
     }
     if (cur_rt >= 0) finish_piece(cur_rt);
@@ -622,6 +691,7 @@ inline int skinny_bn(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 48 ?
 
 cudaError_t launch_stage_x(const void *X, bool x_bf16, const float *awq_s, int64_t M, int64_t K, uint16_t *Xp,
                            int *xexp, cudaStream_t stream) {
+  const int bn = skinny_bn(M);
   using namespace sk_impl;
   const void *func = x_bf16 ? (awq_s ? reinterpret_cast<const void *>(stage_x_kernel<true, true>)
                                      : reinterpret_cast<const void *>(stage_x_kernel<true, false>))
@@ -629,9 +699,10 @@ cudaError_t launch_stage_x(const void *X, bool x_bf16, const float *awq_s, int64
                                      : reinterpret_cast<const void *>(stage_x_kernel<false, false>));
   const uint16_t *xp = static_cast<const uint16_t *>(X);
   const float *sp = awq_s;
-  int64_t k = K;
-  void *args[] = {&xp, &sp, &k, &Xp, &xexp};
-  return launch_pdl(func, dim3((unsigned)M), dim3(256), 0, stream, args);
+  int64_t m = M, k = K;
+  int b = bn;
+  void *args[] = {&xp, &sp, &m, &k, &b, &Xp, &xexp};
+  return launch_pdl(func, dim3((unsigned)bn), dim3(256), 0, stream, args);
 }
 
 cudaError_t launch_skinny(const CUtensorMap &tmW, const CUtensorMap &tmX, const SkinnyParams &p, int grid,

@@ -305,8 +305,8 @@ GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_ca
 
 // K3 (small token counts, group 128): one CTA per SM over a balanced partition
 // of the (128-row tile, 2-group stage) iterations; workspace = counters, the
-// staged activations x' (fp16 [M][K]), the per-token exponents, and fp32
-// partials [slots][M][N] for tiles split between CTAs.
+// staged activations x' (fp16 [K / 64][BN][64], BN = M rounded up to 16), the
+// per-token exponents, and fp32 partials [slots][M][N] for tiles split between CTAs.
 constexpr int64_t kSkinnyMaxM = 64;
 
 GemmPlan plan_skinny(int64_t M, int64_t N, int64_t K, int sm) {
@@ -320,7 +320,7 @@ GemmPlan plan_skinny(int64_t M, int64_t N, int64_t K, int sm) {
   p.grid_x = (int)C;
   p.slots = (int)(S <= 1 ? 1 : std::min<int64_t>(C, (S - 2) / L + 2));
   p.xp_off = kCounterBytes;
-  p.xexp_off = p.xp_off + align256((size_t)M * K * 2);
+  p.xexp_off = p.xp_off + align256((size_t)w4::skinny_bn(M) * K * 2);
   p.part_off = p.xexp_off + 256;
   p.ws_bytes = p.part_off + (size_t)p.slots * M * N * 4;
   return p;
@@ -565,11 +565,13 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
     int *xexp = reinterpret_cast<int *>(wsb + plan.xexp_off);
     CUtensorMap tmW, tmXp;
     CUresult r = encode_2d(enc, &tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2), (uint64_t)N,
-                           (uint64_t)(K / 2), 128u, 64u, CU_TENSOR_MAP_SWIZZLE_128B,
+                           (uint64_t)(K / 2), 128u, 128u, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
     if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for packed weights failed (CUresult %d)", (int)r);
-    r = encode_2d(enc, &tmXp, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64u,
-                  (uint32_t)w4::skinny_bn(M), CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    // x' blocked as [K / 64][BN][64]: rows of 64 channels, one stage = 4 BN rows
+    const uint32_t bn = (uint32_t)w4::skinny_bn(M);
+    r = encode_2d(enc, &tmXp, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, 64u, (uint64_t)(K / 64) * bn, 128u, 64u, 4u * bn,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
     if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for staged activations failed (CUresult %d)", (int)r);
     e = w4::launch_stage_x(X, xbf16, awq_s, M, K, xp, xexp, s);
     if (e != cudaSuccess) return cuda_fail(e, "activation staging launch");
