@@ -337,12 +337,12 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       mbar_init(&empty[s], 2);  // one commit per group, from that group's issuer
     }
     for (int a = 0; a < kNA; ++a) {
-      mbar_init(&afull[a], kDqThreads / 32);  // one arrival per dequantization warp
+      mbar_init(&afull[a], kDqThreads);
       mbar_init(&aempty[a], 1);
     }
     for (int r = 0; r < kNR; ++r) {
       mbar_init(&accfull[r], 1);
-      mbar_init(&accempty[r], C_::kPrThreads / 32);  // one arrival per promotion warp
+      mbar_init(&accempty[r], C_::kPrThreads);
     }
     fence_barrier_init();
   }
@@ -482,14 +482,8 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       // one store wait for both groups of the stage
       tc_wait_st();
       tc_fence_before();
-      // One arrival per warp: an mbarrier arrive is a read-modify-write of one
-      // shared-memory word, and 256 of them per group serialize into a fixed cost
-      // per stage larger than the stage's work.
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&afull[g % kNA]);
-        mbar_arrive(&afull[(g + 1) % kNA]);
-      }
+      mbar_arrive(&afull[g % kNA]);
+      mbar_arrive(&afull[(g + 1) % kNA]);
       g += 2;
     }
   } else if (warp >= kPr0 / 32) {
@@ -596,11 +590,8 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {  // one arrival per warp (see the dequantization warps)
-        mbar_arrive(&accempty[r0]);
-        mbar_arrive(&accempty[r1]);
-      }
+      mbar_arrive(&accempty[r0]);
+      mbar_arrive(&accempty[r1]);
       g += 2;
     }
     if (cur_rt >= 0) finish_piece(cur_rt);

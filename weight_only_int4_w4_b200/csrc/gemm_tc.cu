@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], TcWarps<kAwq>::kEpi / 32);  // one arrival per dequantization warp
+      mbar_init(&afull[s], TcWarps<kAwq>::kEpi);
     }
     mbar_init(accfull, 1);
     fence_barrier_init();
@@ -345,10 +345,7 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
       // (Deferring this wait until the next stage is dequantized measured 5-10% slower.)
       tc_wait_st();
       tc_fence_before();
-      // One arrival per warp: each mbarrier arrive is a read-modify-write of one
-      // shared-memory word, and one per thread serializes into a cost per stage.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[s]);
+      mbar_arrive(&afull[s]);
     }
 
     // ---- epilogue (the decision to run it is made uniform over the kEpi threads,
