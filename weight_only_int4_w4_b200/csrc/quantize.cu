@@ -51,6 +51,52 @@ struct Load4<__nv_bfloat16> {
 };
 
 __device__ __forceinline__ float clamp15(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
+
+// fl32(d / c) for a small odd integer constant c (7 or 15), without an fp32
+// division: the double product d * RN64(1 / c) is within 2^-52 relative of d / c,
+// while d / c, unless it is an fp32 value itself, lies at least about 2^-29
+// relative from every fp32 rounding midpoint (d has 24 significant bits), so
+// rounding the product to fp32 gives the correctly rounded quotient.  Checked
+// exhaustively for c = 7 and 15 over every fp32 d in the subnormal and lowest
+// binades, [1, 4) and the top binades (the binades between scale exactly).
+template <int kC>
+__device__ __forceinline__ float div_by_const(float d) {
+  return __double2float_rn(__dmul_rn((double)d, 1.0 / (double)kC));
+}
+
+// Reciprocal within 1 ulp (PTX rcp.approx.f32: relative error at most 2^-23).
+// Only ever applied to fp16 scales in [2^-24, 65504], whose reciprocals are normal.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// rint(fl(v / sc)) -- the rounded IEEE quotient, as the codes are defined -- without
+// a division per weight.  With inv = 1 / sc within 1 ulp and r = fl(v * inv),
+//   r = (v / sc)(1 + e1)(1 + e2),  |e1| <= 2^-23, |e2| <= 2^-24,
+// and fl(v / sc) = (v / sc)(1 + e3), |e3| <= 2^-24, so the two differ by at most
+// 2^-22 |v / sc| < 2^-16 while |v / sc| < 64.  When r is farther than 2^-15 from
+// every half-integer, r and fl(v / sc) lie strictly between the same two
+// half-integers and round to the same integer.  When |r| >= 64 both roundings are
+// beyond +-62, and every caller clamps the code to at most 15 (after adding a zero
+// point in [0, 15]) or to [-7, 7], so the code is the same.  Only an r within
+// 2^-15 of a half-integer takes the exact quotient (always correct).  NaN stays NaN.
+// near_half: |r - rint(r)| >= 0.5 - 2^-15 (r - rint(r) is exact).
+__device__ __forceinline__ bool near_half(float r, float t) { return fabsf(__fsub_rn(r, t)) >= 0.5f - 0x1p-15f; }
+__device__ __forceinline__ float rint_quotient(float v, float sc, float inv) {
+  const float r = __fmul_rn(v, inv);
+  const float t = rintf(r);
+  return near_half(r, t) ? rintf(__fdiv_rn(v, sc)) : t;
+}
+
+// Order-preserving integer key of a float (not NaN): signed-integer order of the
+// keys is the order of the values (with -0 just below +0).
+__device__ __forceinline__ int f2key(float f) {
+  const int b = __float_as_int(f);
+  return b ^ ((b >> 31) & 0x7FFFFFFF);
+}
+__device__ __forceinline__ float key2f(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF)); }
 __device__ __forceinline__ float clamp7(float v) { return fminf(fmaxf(v, -7.0f), 7.0f); }
 
 constexpr int kQuantUnroll = 4;  // 128-element chunks in flight per warp
@@ -103,10 +149,17 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
       const int64_t e = (base + u) * 128 + lane * 4;
       float mn = fminf(fminf(v[u][0], v[u][1]), fminf(v[u][2], v[u][3]));
       float mx = fmaxf(fmaxf(v[u][0], v[u][1]), fmaxf(v[u][2], v[u][3]));
+      if constexpr (lg == 32) {
+        // one warp reduction per group (integer keys order like the floats; a NaN
+        // weight has no defined code)
+        mn = key2f(__reduce_min_sync(0xffffffffu, f2key(mn)));
+        mx = key2f(__reduce_max_sync(0xffffffffu, f2key(mx)));
+      } else {
 #pragma unroll
-      for (int o = lg >> 1; o > 0; o >>= 1) {  // within each aligned run of lg lanes
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        for (int o = lg >> 1; o > 0; o >>= 1) {  // within each aligned run of lg lanes
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
       }
       uint32_t q[4];
       __half sc16;
@@ -114,26 +167,44 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
       if constexpr (kSym) {
         // scale = fp16(max|w| / 7) (1.0 if 0); q = clamp(rint(w / scale), -7, 7), stored as q + 8
         const float amax = fmaxf(fabsf(mn), fabsf(mx));
-        sc16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        sc16 = __float2half_rn(div_by_const<7>(amax));
         float sc = __half2float(sc16);
         if (sc == 0.0f) {
           sc = 1.0f;
           sc16 = __float2half_rn(1.0f);
         }
         z = 8.0f;
+        const float inv = rcp_approx(sc);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) q[j] = (uint32_t)(clamp7(rintf(__fdiv_rn(v[u][j], sc))) + 8.0f);
+        for (int j = 0; j < 4; ++j) q[j] = (uint32_t)(clamp7(rint_quotient(v[u][j], sc, inv)) + 8.0f);
       } else {
         // scale = fp16((mx - mn) / 15); a zero fp16 scale is taken as 1.0
-        sc16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+        sc16 = __float2half_rn(div_by_const<15>(__fsub_rn(mx, mn)));
         float sc = __half2float(sc16);
         if (sc == 0.0f) {
           sc = 1.0f;
           sc16 = __float2half_rn(1.0f);
         }
-        z = clamp15(rintf(__fdiv_rn(-mn, sc)));
+        const float inv = rcp_approx(sc);
+        z = clamp15(rint_quotient(-mn, sc, inv));
+        // the four weights' rounded quotients, one (rare) exact pass if any of them
+        // lies near a half-integer
+        float t[4];
+        bool near = false;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) q[j] = (uint32_t)clamp15(__fadd_rn(rintf(__fdiv_rn(v[u][j], sc)), z));
+        for (int j = 0; j < 4; ++j) {
+          const float r = __fmul_rn(v[u][j], inv);
+          t[j] = rintf(r);
+          near |= near_half(r, t[j]);
+        }
+        if (near) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) t[j] = rintf(__fdiv_rn(v[u][j], sc));
+        }
+        // clamp(t + z, 0, 15): t + z is an integer-valued float; the conversion to
+        // unsigned saturates negatives (and NaN) to 0
+#pragma unroll
+        for (int j = 0; j < 4; ++j) q[j] = min(__float2uint_rz(__fadd_rn(t[j], z)), 15u);
       }
       if (e < E) {
         const uint16_t pk = (uint16_t)(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
