@@ -192,7 +192,7 @@ __device__ __forceinline__ uint32_t dq2(uint32_t w, uint32_t mask, uint32_t zc) 
 // The two sets run decoupled: dequantization runs up to kNA groups ahead of the
 // tensor core, promotion up to kNR groups behind it, and each set pays its TMEM
 // store (or load) wait once per two groups.
-constexpr int kNR = 4;                        // per-group accumulators in TMEM
+constexpr int kIssuers = 4;                   // MMA issuer warps (see the role list)
 // Scales and zeros are copied kPf stages ahead of use into a per-thread ring in
 // shared memory (cp.async): under a full HBM stream a global load takes about a
 // microsecond, several stages.  (A register queue does not work: rotating it
@@ -262,6 +262,10 @@ struct Cfg {
   static constexpr int kPrThreads = 128 * kPW;
   // rings of zero-point pairs [kPf][dequantization threads] and scale pairs [kPf][promotion threads]
   static constexpr int kRingBytes = kPf * kDqThreads * 4 + kPf * kPrThreads * 4;
+  // Per-group accumulators: two per issuer where TMEM has room (BN <= 32), so an
+  // issuer's next group never waits for the promotion of its previous one -- that
+  // round trip (commit, promotion, arrival, wake-up) is longer than the MMAs.
+  static constexpr int kNR = BN <= 32 ? 2 * kIssuers : kIssuers;
   static constexpr int kNA = (512 - kNR * BN) / 64;  // TMEM A buffers
   static constexpr int kAccCol = 64 * kNA;          // first accumulator column
   static constexpr int kSmem =
@@ -300,6 +304,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                   const SkinnyParams p) {
   using C_ = Cfg<BN>;
+  constexpr int kNR = C_::kNR;
   constexpr int kNA = C_::kNA;
   constexpr int kAccCol = C_::kAccCol;
   constexpr int kNS = C_::kNS;
@@ -368,8 +373,22 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       prefetch_tensormap(&tmX);
     }
     const bool x_lane = lane == 1;
+    // (tile, stage) of the lane's last stage: each lane asks for its stages in
+    // increasing order, so they advance without a division per stage
+    int last_i = -1;
+    int64_t rt = 0, st = 0;
     auto load_lane = [&](int i) {
-      const int64_t it = it0 + i, rt = it / S, st = it - rt * S;
+      if (last_i < 0) {
+        rt = (it0 + i) / S;
+        st = it0 + i - rt * S;
+      } else {
+        st += i - last_i;
+        while (st >= S) {
+          st -= S;
+          ++rt;
+        }
+      }
+      last_i = i;
       const int s = i % kNS;
       if (!x_lane) {
         tma_load_2d(sW + s * kWStage, &tmW, &full[s], (int32_t)(st * 128), (int32_t)(rt * kRows));
@@ -403,19 +422,19 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   } else if (warp >= kMma0 && warp < kMma0 + kMmaWarps && lane == 0) {
     // ---------------- MMA issuer j = w - 4: the groups g = j (mod 4) of the range
     // (CTA-local group index g = 2 * stage + gi), from A buffer g mod kNA into
-    // accumulator j.
+    // accumulator g mod kNR (always one of this issuer's, as kNR is a multiple of 4).
     const int j = warp - kMma0;
     const uint32_t idesc = idesc_f16(false, BN);
-    const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * j);
-    int n = 0;  // groups issued by this issuer
-    for (int g = j; g < 2 * n_it; g += kNR, ++n) {
+    for (int g = j; g < 2 * n_it; g += kIssuers) {
       const int i = g >> 1, gi = g & 1;
       const int s = i % kNS;
       const int a = g % kNA;
+      const int r = g % kNR;
       const uint32_t a_tmem = tmem + (uint32_t)(64 * a);
+      const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * r);
       if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutMma)) break;
       if (!mbar_wait(&afull[a], (uint32_t)(g / kNA) & 1u, kErrTimeoutMma)) break;
-      if (!mbar_wait(&accempty[j], ((uint32_t)n & 1u) ^ 1u, kErrTimeoutMma)) break;
+      if (!mbar_wait(&accempty[r], ((uint32_t)(g / kNR) & 1u) ^ 1u, kErrTimeoutMma)) break;
       tc_fence_after();
       const uint32_t xs = smem_u32(sX + s * C_::kXStage);
 #pragma unroll
@@ -425,7 +444,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
         tc_mma_ts(d_tmem, a_tmem + 8 * kk, bdesc, idesc, kk > 0 ? 1u : 0u);
       }
       tc_commit(&aempty[a]);
-      tc_commit(&accfull[j]);
+      tc_commit(&accfull[r]);
       tc_commit(&empty[s]);
     }
   } else if (warp >= kDq0 / 32 && warp < kPr0 / 32) {
@@ -559,8 +578,14 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
 
     int g = 0;
     int64_t cur_rt = -1;
+    // tile and stage of iteration i, advanced without a division per stage
+    int64_t it_rt = it0 / S, it_st = it0 - it_rt * S;
     for (int i = 0; i < n_it; ++i) {
-      const int64_t rt = (it0 + i) / S;
+      const int64_t rt = it_rt;
+      if (++it_st == S) {
+        it_st = 0;
+        ++it_rt;
+      }
       if (rt != cur_rt) {
         if (cur_rt >= 0) finish_piece(cur_rt);
         cur_rt = rt;
@@ -575,17 +600,24 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       const bool ok0 = mbar_wait(&accfull[r0], (uint32_t)(g / kNR) & 1u, kErrTimeoutEpilogue);
       const bool ok1 = mbar_wait(&accfull[r1], (uint32_t)((g + 1) / kNR) & 1u, kErrTimeoutEpilogue);
       tc_fence_after();
-      // 8 tokens at a time: both groups' columns (one 8-column load each), one wait
+      // 16 tokens at a time (8 when the thread has 8): both groups' columns in one
+      // load each, one wait -- a TMEM load costs its warp about the same at any width
+      constexpr int kW = kTB % 16 == 0 ? 16 : 8;
 #pragma unroll
-      for (int c0 = 0; c0 < kTB; c0 += 8) {
+      for (int c0 = 0; c0 < kTB; c0 += kW) {
         const uint32_t col = (uint32_t)(kAccCol + tok0 + c0);
-        uint32_t v0[8], v1[8];
-        tmem_ld_32x32b_x8(lane_base + col + (uint32_t)(BN * r0), v0);
-        tmem_ld_32x32b_x8(lane_base + col + (uint32_t)(BN * r1), v1);
+        uint32_t v0[kW], v1[kW];
+        if constexpr (kW == 16) {
+          tmem_ld_32x32b_x16(lane_base + col + (uint32_t)(BN * r0), v0);
+          tmem_ld_32x32b_x16(lane_base + col + (uint32_t)(BN * r1), v1);
+        } else {
+          tmem_ld_32x32b_x8(lane_base + col + (uint32_t)(BN * r0), v0);
+          tmem_ld_32x32b_x8(lane_base + col + (uint32_t)(BN * r1), v1);
+        }
         tc_wait_ld();
         if (ok0 && ok1) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
+          for (int j = 0; j < kW; ++j)
             y[c0 + j] = fmaf(sc1, __uint_as_float(v1[j]), fmaf(sc0, __uint_as_float(v0[j]), y[c0 + j]));
         }
       }
