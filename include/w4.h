@@ -164,6 +164,24 @@ w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype,
                           w4_stream_t stream);
 
 /*
+ * The same without the wait: the copy of X_host, the matmul and the copy back
+ * into Y_host are enqueued on `stream` and the call returns; Y_host is valid
+ * once the caller has synchronized `stream` (ch. 22, section 22.3, as for
+ * w4a16_gemm).  A decode step of several layers then waits once per step
+ * instead of once per layer.  X_host and Y_host must stay valid and unchanged
+ * (X_host) or unread (Y_host) until the stream reaches the copies.  Errors:
+ * as for w4a16_gemm_host; failures of the enqueued work surface at the
+ * caller's synchronization.
+ */
+w4_status w4a16_gemm_host_async(const void *X_host, void *X_dev, w4_dtype x_dtype,
+                                int64_t M, int64_t N, int64_t K, int group,
+                                const uint8_t *packed, const uint16_t *scales,
+                                const uint16_t *zeros, const float *awq_s,
+                                void *Y_host, void *Y_dev, w4_dtype y_dtype,
+                                void *workspace, size_t workspace_bytes,
+                                w4_stream_t stream);
+
+/*
  * AWQ scale search (offline, before w4_quantize).  AWQ quantizes W / s and
  * multiplies back by s, with s a per-input-channel activation magnitude from
  * calibration data (ch. 22 "Advanced inference optimisation", section 22.3);

@@ -204,6 +204,29 @@ def test_host_entry_point(w4):
     check_close(Yh.numpy(), Yref, bound, what="host")
 
 
+def test_host_entry_point_async_waits_once(w4):
+    """Two layers through w4a16_gemm_host_async on one stream, one wait at the end:
+    both host outputs match the oracle (and the per-call-wait entry's results)."""
+    stream = torch.cuda.Stream()
+    outs = []
+    for i, (M, N, K) in enumerate(((1, 640, 2048), (3, 1024, 4096))):
+        tag = ("host-async", i)
+        W = synthetic.weight(K, N, 0.02, 0.0, tag)
+        X = synthetic.activations(M, K, "bf16", tag)
+        packed, scales, zeros = w4.w4_quantize(W.cuda())
+        torch.cuda.synchronize()
+        Xh = X.pin_memory()
+        Yh = torch.full((M, N), float("nan"), dtype=torch.float32).pin_memory()
+        Yd = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        w4.w4a16_gemm_host(Xh, torch.empty_like(X, device="cuda"), packed, scales, zeros, Yh, Yd, stream=stream,
+                           wait=False)
+        outs.append((Yh, X, W, (packed, scales, zeros, Yd)))
+    stream.synchronize()
+    for Yh, X, W, keep in outs:
+        Yref, bound, _ = oracle.reference_linear(X.float().numpy(), W.numpy())
+        check_close(Yh.numpy(), Yref, bound, what="host async")
+
+
 def test_short_workspace_rejected(w4):
     M, N, K = 1, 4096, 14336
     need = w4.w4a16_gemm_workspace_size(M, N, K)

@@ -628,10 +628,10 @@ w4_status w4a16_gemm(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int6
                      stream, nullptr, nullptr, nullptr);
 }
 
-w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K,
-                          int group, const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros,
-                          const float *awq_s, void *Y_host, void *Y_dev, w4_dtype y_dtype, void *workspace,
-                          size_t workspace_bytes, w4_stream_t stream) {
+w4_status w4a16_gemm_host_async(const void *X_host, void *X_dev, w4_dtype x_dtype, int64_t M, int64_t N,
+                                int64_t K, int group, const uint8_t *packed, const uint16_t *scales,
+                                const uint16_t *zeros, const float *awq_s, void *Y_host, void *Y_dev,
+                                w4_dtype y_dtype, void *workspace, size_t workspace_bytes, w4_stream_t stream) {
   t_last_error.clear();
   w4_status st = check_shape(M, N, K, group);
   if (st != W4_OK) return st;
@@ -649,7 +649,17 @@ w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype, int
   if (st != W4_OK) return st;
   e = cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "copy Y to host");
-  e = cudaStreamSynchronize(s);
+  return W4_OK;
+}
+
+w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype, int64_t M, int64_t N, int64_t K,
+                          int group, const uint8_t *packed, const uint16_t *scales, const uint16_t *zeros,
+                          const float *awq_s, void *Y_host, void *Y_dev, w4_dtype y_dtype, void *workspace,
+                          size_t workspace_bytes, w4_stream_t stream) {
+  w4_status st = w4a16_gemm_host_async(X_host, X_dev, x_dtype, M, N, K, group, packed, scales, zeros, awq_s, Y_host,
+                                       Y_dev, y_dtype, workspace, workspace_bytes, stream);
+  if (st != W4_OK) return st;
+  const cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
   return W4_OK;
 }

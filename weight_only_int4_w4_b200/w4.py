@@ -30,6 +30,7 @@ _lib.w4a16_gemm.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P
                             _P, _SZ, _P]
 _lib.w4a16_gemm_host.argtypes = [_P, _P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P, _P,
                                  ctypes.c_int, _P, _SZ, _P]
+_lib.w4a16_gemm_host_async.argtypes = _lib.w4a16_gemm_host.argtypes
 _lib.w4a16_gemm_decode_static.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P,
                                           ctypes.c_int, _P]
 _lib.w4a16_gemm_decode_static_capacity.argtypes = []
@@ -58,7 +59,8 @@ _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
 for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_awq_search", "w4_quantize_outliers", "w4a16_gemm_outliers",
            "w4_quantize_gptq",
-           "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_decode_static", "w4_device_error"):
+           "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_host_async", "w4a16_gemm_decode_static",
+           "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -170,16 +172,19 @@ def w4a16_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zero
 
 
 def w4a16_gemm_host(X_host: torch.Tensor, X_dev: torch.Tensor, packed, scales, zeros, Y_host: torch.Tensor,
-                    Y_dev: torch.Tensor, awq_s=None, ws=None, group: int = GROUP, stream=None) -> torch.Tensor:
-    """End-to-end call with pinned host X and Y: H2D copy, fused GEMM, D2H copy, wait."""
+                    Y_dev: torch.Tensor, awq_s=None, ws=None, group: int = GROUP, stream=None,
+                    wait: bool = True) -> torch.Tensor:
+    """End-to-end call with pinned host X and Y: H2D copy, fused GEMM, D2H copy, and
+    (wait=True) a wait for the stream.  With wait=False the work is only enqueued
+    (w4a16_gemm_host_async): Y_host is valid after the caller synchronizes the stream."""
     M, K = X_host.shape
     N = packed.shape[0]
     if ws is None:
         ws = workspace(M, N, K, X_dev.device, stream)
-    _check(_lib.w4a16_gemm_host(_ptr(X_host), _ptr(X_dev), _DT[X_host.dtype], M, N, K, group, _ptr(packed),
-                                _ptr(scales), _ptr(zeros), _ptr(awq_s), _ptr(Y_host), _ptr(Y_dev),
-                                _DT[Y_host.dtype], _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
-           "w4a16_gemm_host")
+    fn = _lib.w4a16_gemm_host if wait else _lib.w4a16_gemm_host_async
+    _check(fn(_ptr(X_host), _ptr(X_dev), _DT[X_host.dtype], M, N, K, group, _ptr(packed), _ptr(scales), _ptr(zeros),
+              _ptr(awq_s), _ptr(Y_host), _ptr(Y_dev), _DT[Y_host.dtype], _ptr(ws), 0 if ws is None else ws.numel(),
+              _stream(stream)), "w4a16_gemm_host" if wait else "w4a16_gemm_host_async")
     return Y_host
 
 
