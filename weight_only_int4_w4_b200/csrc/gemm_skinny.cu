@@ -63,16 +63,20 @@ constexpr int kWStage = kRows * 128;   // 16 KiB of codes per stage (2 groups)
 
 
 // ------------------------------------------------------------------ staging of x'
-// One CTA of 256 threads per token of the BN-token tile.  Pass 1: max |x * s|
-// over K; pass 2: x' in the permuted order (see the file head).  Channels
+// One CTA of 512 threads per token of the BN-token tile: max |x * s| over K,
+// then x' in the permuted order (see the file head).  Channels
 // k = 8j + c (c = 0..7).  Layout: x'[k / 64][token][k % 64] (64-channel blocks,
 // BN tokens each), so one stage's 4 blocks x BN tokens are consecutive rows of
 // 128 bytes and arrive in one TMA box.  Tokens M..BN-1 are zeros.
+constexpr int kStageThreads = 512;  // threads per token
+constexpr int kStageChunks = 8;     // 8-channel chunks a thread holds in the one-pass form
+
 template <bool kBf16, bool kAwq>
-__global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict__ X, const float *__restrict__ s,
-                                                      int64_t M, int64_t K, int bn, uint16_t *__restrict__ Xp,
-                                                      int *__restrict__ xexp) {
-  __shared__ float red[8];
+__global__ void __launch_bounds__(kStageThreads) stage_x_kernel(const uint16_t *__restrict__ X,
+                                                                const float *__restrict__ s, int64_t M, int64_t K,
+                                                                int bn, uint16_t *__restrict__ Xp,
+                                                                int *__restrict__ xexp) {
+  __shared__ float red[kStageThreads / 32];
   // The activations may be written by the preceding kernel, and x' may still be
   // read by the preceding matmul: wait for it, then let the matmul launch.
   grid_dependency_wait();
@@ -87,8 +91,9 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict
     return;
   }
   const uint16_t *xr = X + m * K;
-  auto load8 = [&](int64_t j, float (&v)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(xr + 8 * j));
+  auto load_raw = [&](int64_t j) { return __ldg(reinterpret_cast<const uint4 *>(xr + 8 * j)); };
+  // x (times s with AWQ) of chunk j from its raw 16 bytes
+  auto decode = [&](int64_t j, const uint4 &u, float (&v)[8]) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -108,20 +113,42 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict
       v[4] *= s1.x; v[5] *= s1.y; v[6] *= s1.z; v[7] *= s1.w;
     }
   };
+  // One pass when the token fits the registers (every shape up to K = 32768): all
+  // of a thread's loads are in flight at once and X is read once.  Otherwise two
+  // passes (max, then convert), each reading X.
+  const bool one_pass = nb <= (int64_t)kStageChunks * blockDim.x;
+  uint4 raw[kStageChunks];
   float mx = 0.0f;
-  for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) {
-    float v[8];
-    load8(j, v);
+  if (one_pass) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+    for (int c = 0; c < kStageChunks; ++c) {
+      const int64_t j = threadIdx.x + (int64_t)c * blockDim.x;
+      raw[c] = j < nb ? load_raw(j) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int c = 0; c < kStageChunks; ++c) {
+      const int64_t j = threadIdx.x + (int64_t)c * blockDim.x;
+      if (j < nb) {
+        float v[8];
+        decode(j, raw[c], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+      }
+    }
+  } else {
+    for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) {
+      float v[8];
+      decode(j, load_raw(j), v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(v[i]));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
   __syncthreads();
   mx = red[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) mx = fmaxf(mx, red[i]);
   // max |x'| in [2^13, 2^14): e = 13 - floor(log2 max); 0 for an all-zero token
   const int bits = __float_as_int(mx);
   int e = bits == 0 ? 0 : 13 - (((bits >> 23) & 0xFF) - 127);
@@ -129,9 +156,9 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict
   if (threadIdx.x == 0) xexp[m] = e;
   const float se = __uint_as_float((uint32_t)(e + 127) << 23);      // 2^e
   const float so = __uint_as_float((uint32_t)(e - 4 + 127) << 23);  // 2^(e-4): odd channels / 16
-  for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) {
+  auto convert_store = [&](int64_t j, const uint4 &u) {
     float v[8];
-    load8(j, v);
+    decode(j, u, v);
     // slots 0..7 hold channels 0, 4, 1, 5, 2, 6, 3, 7; odd channels carry 1/16
     const __half2 h0 = __floats2half2_rn(v[0] * se, v[4] * se);
     const __half2 h1 = __floats2half2_rn(v[1] * so, v[5] * so);
@@ -143,6 +170,15 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t *__restrict
     o.z = *reinterpret_cast<const uint32_t *>(&h2);
     o.w = *reinterpret_cast<const uint32_t *>(&h3);
     *reinterpret_cast<uint4 *>(out_at(j)) = o;
+  };
+  if (one_pass) {
+#pragma unroll
+    for (int c = 0; c < kStageChunks; ++c) {
+      const int64_t j = threadIdx.x + (int64_t)c * blockDim.x;
+      if (j < nb) convert_store(j, raw[c]);
+    }
+  } else {
+    for (int64_t j = threadIdx.x; j < nb; j += blockDim.x) convert_store(j, load_raw(j));
   }
 }
 
@@ -725,7 +761,7 @@ cudaError_t launch_stage_x(const void *X, bool x_bf16, const float *awq_s, int64
   int64_t m = M, k = K;
   int b = bn;
   void *args[] = {&xp, &sp, &m, &k, &b, &Xp, &xexp};
-  return launch_pdl(func, dim3((unsigned)bn), dim3(256), 0, stream, args);
+  return launch_pdl(func, dim3((unsigned)bn), dim3(kStageThreads), 0, stream, args);
 }
 
 cudaError_t launch_skinny(const CUtensorMap &tmW, const CUtensorMap &tmX, const SkinnyParams &p, int grid,
