@@ -326,18 +326,25 @@ GemmPlan plan_skinny(int64_t M, int64_t N, int64_t K, int sm) {
   return p;
 }
 
-// Measured on B200 (8B layer shapes): the decode kernel wins up to M = 8; above
-// that the tensor cores take the M-fold product: K3 up to 64 tokens (faster than
-// K2 at every 8B and 70B shape at M = 16..64), K2 above.
-bool gemv_fits(int64_t M, int64_t N, bool awq) {
-  return M <= 8 && w4::gemv_supports(M, awq);
+// Measured on B200 (8B and 70B layer shapes): the decode kernel wins at M = 1..3
+// and on the smaller layers up to M = 8; above that the tensor cores take the
+// M-fold product: K3 up to 64 tokens (faster than K2 at every 8B and 70B shape
+// at M = 16..64), K2 above.  Crossovers measured for K1 against K3: at M = 5..8,
+// K3 on every layer with N*K >= 32 M weights (8B gate_up 31 against 42..46 us,
+// 8B down 24 against 26..39 us, every 70B layer); at M = 4 only on the largest
+// (70B gate_up 92 against 109 us, 70B down 54 against 82 us).
+bool gemv_fits(int64_t M, int64_t N, int64_t K, bool awq) {
+  if (M > 8 || !w4::gemv_supports(M, awq)) return false;
+  const double nk = (double)N * (double)K;
+  const bool skinny_wins = (M >= 5 && nk >= 32.0e6) || (M == 4 && nk >= 200.0e6);
+  return !skinny_wins;
 }
 
 GemmPlan plan_gemm_raw(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_cap) {
   int f = forced_path();
   if (f == kPathTc) return plan_tc(M, N, K, awq, sm, ws_cap);
   if (f == kPathSkinny) return plan_skinny(M, N, K, sm);
-  if (f == kPathGemv || gemv_fits(M, N, awq)) {
+  if (f == kPathGemv || gemv_fits(M, N, K, awq)) {
     const GemmPlan p = plan_gemv(M, N, K, awq, sm);
     if (p.path == kPathGemv || f == kPathGemv) return p;
   }
