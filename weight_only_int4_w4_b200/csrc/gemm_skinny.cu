@@ -241,6 +241,15 @@ constexpr int kDq0 = 32 * (kProdWarps + kMmaWarps);  // first dequantization thr
 constexpr int kDqThreads = 128;               // warps 8..11
 constexpr int kPr0 = kDq0 + kDqThreads;       // first promotion thread (warp 12)
 
+// Ticket of a split tile: acquire-release at GPU scope.  After a CTA barrier, one
+// thread's release publishes the whole CTA's partial stores (no full fence); the
+// last ticket's acquire, followed by a CTA barrier, orders the loads of the
+// threads that sum every piece after all contributors' stores.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
@@ -596,9 +605,8 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
             if (t < M) __stcg(part + (int64_t)t * N + n, y[j] * s_escale[t]);
           }
         }
-        __threadfence();
-        named_bar_pr<C_::kPrThreads>();
-        if (threadIdx.x == kPr0) s_ticket[npend] = (int)atomicAdd(&p.counters[rt], 1u);
+        named_bar_pr<C_::kPrThreads>();  // every thread's partials, then one release
+        if (threadIdx.x == kPr0) s_ticket[npend] = (int)atom_add_acq_rel_gpu(&p.counters[rt], 1u);
         if (npend == 0) {
           pend_rt0 = rt;
           pend_cnt0 = (int)(last - first + 1);
@@ -670,7 +678,6 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       const int cnt = j == 0 ? pend_cnt0 : pend_cnt1;
       const int64_t rt = j == 0 ? pend_rt0 : pend_rt1;
       if (ticket != cnt - 1) continue;
-      __threadfence();
       const int64_t n = rt * kRows + rr;
       if (n < N) {
         // 8 tokens at a time, slot by slot, with every token's load of a slot in
