@@ -314,7 +314,7 @@ struct Cfg {
   static constexpr int kNA = (512 - kNR * BN) / 64;  // TMEM A buffers
   static constexpr int kAccCol = 64 * kNA;          // first accumulator column
   static constexpr int kSmem =
-      1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + kRingBytes + 64;
+      1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + kRingBytes + 16 + 64;
   static constexpr int kThreads = kPr0 + kPrThreads;
   static_assert(kAccCol + kNR * BN <= 512, "TMEM columns");
   static_assert(kSmem <= 232448, "shared memory");
@@ -369,6 +369,8 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   float *s_escale = reinterpret_cast<float *>(tmem_holder + 4);  // [64] 2^-e per token
   uint32_t *zring = reinterpret_cast<uint32_t *>(s_escale + 64);  // [kPf][kDqThreads]
   uint32_t *sring = zring + kPf * kDqThreads;                     // [kPf][kPrThreads]
+  int *s_pend = reinterpret_cast<int *>(sring + kPf * C_::kPrThreads);  // split tiles: rt0, count0, rt1, count1
+  int *s_npend = reinterpret_cast<int *>(tmem_holder + 3);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -671,43 +673,13 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       g += 2;
     }
     if (cur_rt >= 0) finish_piece(cur_rt);
-    // resolve the tickets of split tiles: the last contributor sums every piece
-    named_bar_pr<C_::kPrThreads>();
-    for (int j = 0; j < npend; ++j) {
-      const int ticket = s_ticket[j];
-      const int cnt = j == 0 ? pend_cnt0 : pend_cnt1;
-      const int64_t rt = j == 0 ? pend_rt0 : pend_rt1;
-      if (ticket != cnt - 1) continue;
-      const int64_t n = rt * kRows + rr;
-      if (n < N) {
-        // 8 tokens at a time, slot by slot, with every token's load of a slot in
-        // flight at once; the slots are summed in increasing order for every token
-#pragma unroll
-        for (int c0 = 0; c0 < kTB; c0 += 8) {
-          float acc[8];
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
-          for (int sl = 0; sl < cnt; ++sl) {
-            float v[8];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const int t = tok0 + c0 + jj;
-              v[jj] = t < M ? __ldcg(p.ws + ((int64_t)sl * M + t) * N + n) : 0.0f;
-            }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) acc[jj] += v[jj];
-          }
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int t = tok0 + c0 + jj;
-            if (t < M) {
-              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[(int64_t)t * N + n] = __float2bfloat16_rn(acc[jj]);
-              else static_cast<float *>(p.Y)[(int64_t)t * N + n] = acc[jj];
-            }
-          }
-        }
-      }
-      if (threadIdx.x == kPr0) atomicExch(&p.counters[rt], 0u);
+    // the split tiles of this range and their tickets, for the whole CTA's fix-up below
+    if (threadIdx.x == kPr0) {
+      *s_npend = npend;
+      s_pend[0] = (int)pend_rt0;
+      s_pend[1] = pend_cnt0;
+      s_pend[2] = (int)pend_rt1;
+      s_pend[3] = pend_cnt1;
     }
   }
 
@@ -716,6 +688,36 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   if (warp == kMma0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+
+  // Split tiles whose last ticket this CTA took: every thread of the CTA sums
+  // (row, token) elements of the tile over its pieces, in increasing slot order.
+  // (The ticket's acquire by one promotion thread and the barrier above order these
+  // loads after every contributor's partial stores.)
+  const int npend_all = *s_npend;
+  for (int j = 0; j < npend_all; ++j) {
+    const int cnt = s_pend[2 * j + 1];
+    const int64_t rt = s_pend[2 * j];
+    if (s_ticket[j] != cnt - 1) continue;
+    const int64_t elems = (int64_t)kRows * M;
+#pragma unroll 2
+    for (int64_t e = threadIdx.x; e < elems; e += blockDim.x) {
+      const int row = (int)(e % kRows);
+      const int64_t t = e / kRows;
+      const int64_t n = rt * kRows + row;
+      if (n >= N) continue;
+      float v[8];
+#pragma unroll
+      for (int sl = 0; sl < 8; ++sl) v[sl] = sl < cnt ? __ldcg(p.ws + ((int64_t)sl * M + t) * N + n) : 0.0f;
+      float acc = 0.0f;
+#pragma unroll
+      for (int sl = 0; sl < 8; ++sl)
+        if (sl < cnt) acc += v[sl];
+      for (int sl = 8; sl < cnt; ++sl) acc += __ldcg(p.ws + ((int64_t)sl * M + t) * N + n);
+      if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[t * N + n] = __float2bfloat16_rn(acc);
+      else static_cast<float *>(p.Y)[t * N + n] = acc;
+    }
+    if (threadIdx.x == 0) atomicExch(&p.counters[rt], 0u);
   }
 }
 
