@@ -314,7 +314,7 @@ struct Cfg {
   static constexpr int kNA = (512 - kNR * BN) / 64;  // TMEM A buffers
   static constexpr int kAccCol = 64 * kNA;          // first accumulator column
   static constexpr int kSmem =
-      1024 + kNS * kStage + (2 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + kRingBytes + 16 + 64;
+      1024 + kNS * kStage + (3 * kNS + 2 * kNA + 2 * kNR) * 8 + 16 + 64 * 4 + kRingBytes + 16 + 64;
   static constexpr int kThreads = kPr0 + kPrThreads;
   static_assert(kAccCol + kNR * BN <= 512, "TMEM columns");
   static_assert(kSmem <= 232448, "shared memory");
@@ -358,8 +358,12 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sW = smem;
   uint8_t *sX = smem + kNS * kWStage;
-  uint64_t *full = reinterpret_cast<uint64_t *>(sX + kNS * C_::kXStage);
-  uint64_t *empty = full + kNS;
+  // A stage's codes and its x' complete separate barriers: the dequantization needs
+  // only the codes, so it runs ahead while x' (which waits for the staging kernel)
+  // is still on its way; the MMA issuers wait for x'.
+  uint64_t *full = reinterpret_cast<uint64_t *>(sX + kNS * C_::kXStage);  // codes
+  uint64_t *xfull = full + kNS;                                            // x'
+  uint64_t *empty = xfull + kNS;
   uint64_t *afull = empty + kNS;
   uint64_t *aempty = afull + kNA;
   uint64_t *accfull = aempty + kNA;    // [kNR]
@@ -386,6 +390,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&xfull[s], 1);
       mbar_init(&empty[s], 2);  // one commit per group, from that group's issuer
     }
     for (int a = 0; a < kNA; ++a) {
@@ -440,28 +445,32 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       if (!x_lane) {
         tma_load_2d(sW + s * kWStage, &tmW, &full[s], (int32_t)(st * 128), (int32_t)(rt * kRows));
       } else {
-        tma_load_2d(sX + s * C_::kXStage, &tmX, &full[s], 0, (int32_t)(st * 4 * BN));
+        tma_load_2d(sX + s * C_::kXStage, &tmX, &xfull[s], 0, (int32_t)(st * 4 * BN));
       }
     };
     // Weights never come from a preceding kernel: the first ring's codes are
     // requested before waiting for the staged activations.
     const int pre = n_it < kNS ? n_it : kNS;
     for (int i = k; i < pre; i += kProdWarps) {
-      if (!x_lane) mbar_arrive_expect_tx(&full[i % kNS], C_::kStage);
-      __syncwarp(0x3u);
-      if (!x_lane) load_lane(i);
+      if (!x_lane) {
+        mbar_arrive_expect_tx(&full[i % kNS], kWStage);
+        load_lane(i);
+      }
     }
     grid_dependency_wait();
-    for (int i = k; i < pre; i += kProdWarps)
-      if (x_lane) load_lane(i);
+    for (int i = k; i < pre; i += kProdWarps) {
+      if (x_lane) {
+        mbar_arrive_expect_tx(&xfull[i % kNS], C_::kXStage);
+        load_lane(i);
+      }
+    }
     for (int i = pre + ((k - pre % kProdWarps + kProdWarps) % kProdWarps); i < n_it; i += kProdWarps) {
       const int s = i % kNS;
       // both lanes wait for the free slot; the vote keeps them on one path if a
       // wait ever gives up
       const bool w_ok = mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, kErrTimeoutTma);
       if (!__all_sync(0x3u, w_ok)) break;
-      if (!x_lane) mbar_arrive_expect_tx(&full[s], C_::kStage);
-      __syncwarp(0x3u);
+      mbar_arrive_expect_tx(x_lane ? &xfull[s] : &full[s], x_lane ? C_::kXStage : kWStage);
       load_lane(i);
     }
     // every load of this CTA is issued: the next kernel in the stream may launch
@@ -479,7 +488,7 @@ __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
       const int r = g % kNR;
       const uint32_t a_tmem = tmem + (uint32_t)(64 * a);
       const uint32_t d_tmem = tmem + (uint32_t)(kAccCol + BN * r);
-      if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutMma)) break;
+      if (!mbar_wait(&xfull[s], (uint32_t)(i / kNS) & 1u, kErrTimeoutMma)) break;
       if (!mbar_wait(&afull[a], (uint32_t)(g / kNA) & 1u, kErrTimeoutMma)) break;
       if (!mbar_wait(&accempty[r], ((uint32_t)(g / kNR) & 1u) ^ 1u, kErrTimeoutMma)) break;
       tc_fence_after();
