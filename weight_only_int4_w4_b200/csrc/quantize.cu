@@ -4,7 +4,7 @@
 // 128 input channels ("LLM inference acceleration" article, section 2.1), also
 // served with groups of 32 and 64.  Symmetric variant: INT4 as the value set
 // {-7..7} (mhpq.cn practitioner's article, section 2.1), stored as q + 8 with
-// zero point 8.  Each lane holds 4 weights; a group is held by G/4 lanes.  Optional AWQ prescale w / s[k] is applied on load (ch. 22
+// zero point 8.  Each lane holds 8 weights; a group is held by G/8 lanes.  Optional AWQ prescale w / s[k] is applied on load (ch. 22
 // "Advanced inference optimisation", section 22.3, AWQ equation).  Every
 // step uses IEEE fp32 round-to-nearest intrinsics so the results are bit-exact
 // with the definition in w4.h.  The kernel is HBM-bound: it reads W once and
@@ -99,13 +99,16 @@ __device__ __forceinline__ int f2key(float f) {
 __device__ __forceinline__ float key2f(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF)); }
 __device__ __forceinline__ float clamp7(float v) { return fminf(fmaxf(v, -7.0f), 7.0f); }
 
-constexpr int kQuantUnroll = 4;  // 128-element chunks in flight per warp
+constexpr int kQuantUnroll = 2;  // 256-element chunks in flight per warp
+constexpr int kWPL = 8;          // weights per lane
 
-// The matrix is walked as its flattened N*K elements in chunks of 128: lane l of
-// a warp holds elements 4l..4l+3 of a chunk, and a group of G (32, 64 or 128)
+// The matrix is walked as its flattened N*K elements in chunks of 256: lane l of
+// a warp holds elements 8l..8l+7 of a chunk, and a group of G (32, 64 or 128)
 // consecutive elements (groups never straddle rows, since G divides K) is held
-// by G/4 consecutive lanes, which reduce its min and max with shuffles.  Group j
-// of the flattened order is scales[j] / zeros[j] of the [N][K/G] arrays.
+// by G/8 consecutive lanes, which reduce its min and max with shuffles.  A warp
+// thus works on 2 to 8 groups at once, and the per-group steps (scale, zero
+// point, reciprocal) are shared by 8 weights per lane.  Group j of the flattened
+// order is scales[j] / zeros[j] of the [N][K/G] arrays.
 template <typename TW, bool kAwq, bool kCodes, bool kSym, int kG, bool kMask>
 __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W, const float *__restrict__ awq_s,
                                                        int64_t E, int64_t K,
@@ -115,53 +118,58 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t chunks = (E + 127) / 128;
-  constexpr int lg = kG / 4;  // lanes per group
+  constexpr int kChunk = 32 * kWPL;
+  const int64_t chunks = (E + kChunk - 1) / kChunk;
+  constexpr int lg = kG / kWPL;  // lanes per group
   // dense part of a dense + sparse split: weights with |w| >= tau count as 0 here
   const uint32_t tau = kMask ? *outlier_tau : 0xFFFFFFFFu;
 
   for (int64_t base = warp * kQuantUnroll; base < chunks; base += nwarps * kQuantUnroll) {
-    float v[kQuantUnroll][4];
+    float v[kQuantUnroll][kWPL];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t e = (base + u) * 128 + lane * 4;
-      if (e < E) {
-        Load4<TW>::run(W + e, v[u]);
+      const int64_t e = (base + u) * kChunk + lane * kWPL;
+      if (e < E) {  // E is a multiple of 32 (G divides K), so a lane's 8 are all in range
+        float h[4];
+        Load4<TW>::run(W + e, h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[u][j] = h[j];
+        Load4<TW>::run(W + e + 4, h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[u][4 + j] = h[j];
         if constexpr (kMask) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < kWPL; ++j)
             if ((__float_as_uint(v[u][j]) & 0x7FFFFFFFu) >= tau) v[u][j] = 0.0f;
         }
         if (kAwq) {
-          const int64_t k = e % K;
-          const float4 s = __ldg(reinterpret_cast<const float4 *>(awq_s + k));
-          v[u][0] = __fdiv_rn(v[u][0], s.x);
-          v[u][1] = __fdiv_rn(v[u][1], s.y);
-          v[u][2] = __fdiv_rn(v[u][2], s.z);
-          v[u][3] = __fdiv_rn(v[u][3], s.w);
+          const int64_t k = e % K;  // a lane's 8 weights lie in one row (K is a multiple of 32)
+          const float4 s0 = __ldg(reinterpret_cast<const float4 *>(awq_s + k));
+          const float4 s1 = __ldg(reinterpret_cast<const float4 *>(awq_s + k + 4));
+          const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+          for (int j = 0; j < kWPL; ++j) v[u][j] = __fdiv_rn(v[u][j], sv[j]);
         }
       } else {
-        v[u][0] = v[u][1] = v[u][2] = v[u][3] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kWPL; ++j) v[u][j] = 0.0f;
       }
     }
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t e = (base + u) * 128 + lane * 4;
-      float mn = fminf(fminf(v[u][0], v[u][1]), fminf(v[u][2], v[u][3]));
-      float mx = fmaxf(fmaxf(v[u][0], v[u][1]), fmaxf(v[u][2], v[u][3]));
-      if constexpr (lg == 32) {
-        // one warp reduction per group (integer keys order like the floats; a NaN
-        // weight has no defined code)
-        mn = key2f(__reduce_min_sync(0xffffffffu, f2key(mn)));
-        mx = key2f(__reduce_max_sync(0xffffffffu, f2key(mx)));
-      } else {
+      const int64_t e = (base + u) * kChunk + lane * kWPL;
+      float mn = v[u][0], mx = v[u][0];
 #pragma unroll
-        for (int o = lg >> 1; o > 0; o >>= 1) {  // within each aligned run of lg lanes
-          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
+      for (int j = 1; j < kWPL; ++j) {
+        mn = fminf(mn, v[u][j]);
+        mx = fmaxf(mx, v[u][j]);
       }
-      uint32_t q[4];
+#pragma unroll
+      for (int o = lg >> 1; o > 0; o >>= 1) {  // within each aligned run of lg lanes
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      uint32_t q[kWPL];
       __half sc16;
       float z;
       if constexpr (kSym) {
@@ -176,7 +184,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
         z = 8.0f;
         const float inv = rcp_approx(sc);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) q[j] = (uint32_t)(clamp7(rint_quotient(v[u][j], sc, inv)) + 8.0f);
+        for (int j = 0; j < kWPL; ++j) q[j] = (uint32_t)(clamp7(rint_quotient(v[u][j], sc, inv)) + 8.0f);
       } else {
         // scale = fp16((mx - mn) / 15); a zero fp16 scale is taken as 1.0
         sc16 = __float2half_rn(div_by_const<15>(__fsub_rn(mx, mn)));
@@ -187,29 +195,35 @@ __global__ void __launch_bounds__(256) quantize_kernel(const TW *__restrict__ W,
         }
         const float inv = rcp_approx(sc);
         z = clamp15(rint_quotient(-mn, sc, inv));
-        // the four weights' rounded quotients, one (rare) exact pass if any of them
-        // lies near a half-integer
-        float t[4];
+        // the lane's rounded quotients, one (rare) exact pass if any of them lies
+        // near a half-integer
+        float t[kWPL];
         bool near = false;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kWPL; ++j) {
           const float r = __fmul_rn(v[u][j], inv);
           t[j] = rintf(r);
           near |= near_half(r, t[j]);
         }
         if (near) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) t[j] = rintf(__fdiv_rn(v[u][j], sc));
+          for (int j = 0; j < kWPL; ++j) t[j] = rintf(__fdiv_rn(v[u][j], sc));
         }
         // clamp(t + z, 0, 15): t + z is an integer-valued float; the conversion to
         // unsigned saturates negatives (and NaN) to 0
 #pragma unroll
-        for (int j = 0; j < 4; ++j) q[j] = min(__float2uint_rz(__fadd_rn(t[j], z)), 15u);
+        for (int j = 0; j < kWPL; ++j) q[j] = min(__float2uint_rz(__fadd_rn(t[j], z)), 15u);
       }
       if (e < E) {
-        const uint16_t pk = (uint16_t)(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
-        reinterpret_cast<uint16_t *>(packed)[e >> 2] = pk;
-        if (kCodes) reinterpret_cast<uint32_t *>(codes)[e >> 2] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+        uint32_t pk = 0;
+#pragma unroll
+        for (int j = 0; j < kWPL; ++j) pk |= q[j] << (4 * j);
+        reinterpret_cast<uint32_t *>(packed)[e >> 3] = pk;
+        if (kCodes) {
+          const uint32_t c0 = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+          const uint32_t c1 = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
+          reinterpret_cast<uint2 *>(codes)[e >> 3] = make_uint2(c0, c1);
+        }
         if ((lane & (lg - 1)) == 0) {
           const int64_t gi = e / kG;
           scales[gi] = __half_as_ushort(sc16);
@@ -259,7 +273,7 @@ cudaError_t launch_quantize_g(const void *W, const float *awq_s, int64_t N, int6
                               uint8_t *packed, uint16_t *scales, uint16_t *zeros, uint8_t *codes, int sm_count,
                               cudaStream_t stream) {
   const int64_t E = N * K;
-  const int64_t chunks = (E + 127) / 128;
+  const int64_t chunks = (E + 32 * kWPL - 1) / (32 * kWPL);
   const int grid = grid_for(chunks, 8 * kQuantUnroll, sm_count, 8);
   const TW *w = static_cast<const TW *>(W);
   if (awq_s) {
