@@ -157,6 +157,34 @@ def test_split_k_reduction_ragged(w4, monkeypatch, capfd, M, N, K, awq, splits):
     assert f"tensor-core: bn=64 splits={splits} " in err, err
 
 
+@pytest.mark.parametrize("M,N,K,awq,out,bn,tiles,pieces", [
+    (300, 9688, 4096, False, "f32", 256, 152, 4),    # 4 tail tiles in 4 pieces, ragged last n-tile and tokens
+    (300, 9688, 3200, True, "bf16", 256, 152, 3),    # AWQ kernel, uneven last piece, bf16 output
+    (100, 38149, 5120, False, "f32", 128, 299, 5),  # two CTAs per SM (296 slots): one batch of 4 pieces + 1
+])
+def test_tail_split_last_wave(w4, monkeypatch, capfd, M, N, K, awq, out, bn, tiles, pieces):
+    """Tensor-core tail split: whole tiles fill complete waves and the last,
+    mostly empty wave's tiles are cut along K; the reduction kernel sums the
+    pieces.  Every output of the tail tiles is checked, with a sample elsewhere.
+    W4_FORCE_TAIL takes the split at these small depths, where the planner's
+    cost rule would keep whole tiles."""
+    monkeypatch.setenv("W4_DEBUG_PLAN", "1")
+    monkeypatch.setenv("W4_FORCE_TAIL", "1")
+    ntx = (N + 127) // 128
+    slots = 148 * (1 if (awq or bn == 256) else 2)
+    head = tiles - tiles % slots
+    tail_rows = set()
+    for t in range(head, tiles):
+        n0 = (t % ntx) * 128
+        tail_rows.update(range(n0, min(n0 + 128, N)))
+    rows = np.array(sorted(tail_rows | set(sample_rows(N, 48, seed=N ^ K).tolist())))
+    _run_case(w4, M, N, K, awq=awq, path="tc", rows=rows,
+              out_dtype=torch.bfloat16 if out == "bf16" else torch.float32, tag=("tail", M, N, K, awq))
+    err = capfd.readouterr().err
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert f"bn={bn} splits=1 " in err and f"head_tiles={head} tail_pieces={pieces} " in err, err
+
+
 def test_long_k_split_both_paths(w4):
     """K = 28672 (70B down_proj depth) at small M: split-K on both paths."""
     for path in ("gemv", "skinny", "tc"):

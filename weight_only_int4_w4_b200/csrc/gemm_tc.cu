@@ -37,8 +37,17 @@ struct TcParams {
   float *ws;           // [splits][M][N] partials (split-K only)
   uint32_t *counters;  // [tiles] arrival counters (split-K only)
   int splits;
-  int kb_per_split;  // k-blocks of 64 per split
+  int kb_per_split;  // k-blocks of 64 per split (per tail piece in tail mode)
   int group;         // quantization group: 32, 64 or 128 input channels
+  // Tail mode (tail_pieces > 0; splits is then 1): tiles t = y * n-tiles + x
+  // below head_tiles are computed whole; each later tile is cut into
+  // tail_pieces k-ranges.  Piece 0 runs at the tile's own grid position, pieces
+  // 1.. in extra grid rows after the tiles (so they are dispatched last), and
+  // piece z of tail tile i writes its fp32 partial tile to
+  // ws[i * tail_pieces + z][BN][128]; tail_reduce_kernel sums the pieces.
+  int64_t head_tiles;
+  int tail_pieces;
+  int64_t ntx;  // output tiles along N
 };
 
 namespace tc_impl {
@@ -182,7 +191,7 @@ __device__ __forceinline__ bool epilogue_vote(bool v) {
   return r != 0;
 }
 
-template <int BN, bool kBf16, bool kAwq>
+template <int BN, bool kBf16, bool kAwq, bool kTail>
 __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                    const TcParams p) {
@@ -203,12 +212,35 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t M = p.M, N = p.N, K = p.K;
-  const int64_t n0 = (int64_t)blockIdx.x * 128;
-  const int64_t m0 = (int64_t)blockIdx.y * BN;
-  const int split = blockIdx.z;
   const int total_kb = (int)(K / kBK);
-  const int kb0 = split * p.kb_per_split;
-  const int kb1 = min(kb0 + p.kb_per_split, total_kb);
+  int64_t tile_n = blockIdx.x, tile_m = blockIdx.y;
+  int split = blockIdx.z, kbps = p.kb_per_split;
+  int64_t tail_unit = -1;  // tail mode: this CTA's partial slot, -1 for a whole tile
+  // (A separate instantiation: compiled into every launch, the tail mapping
+  // made the plain kernel 15-18 % slower on B200.)
+  if constexpr (kTail) {
+    const int64_t tiles_m = (M + BN - 1) / BN;
+    const int64_t t = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+    if (blockIdx.y < tiles_m) {
+      if (t < p.head_tiles) kbps = total_kb;                   // a whole tile
+      else tail_unit = (t - p.head_tiles) * p.tail_pieces;  // piece 0 of a tail tile
+    } else {  // rows past the tiles: pieces 1.. of the tail tiles, then idle CTAs
+      const int pm1 = p.tail_pieces - 1;
+      const int e = (int)(t - tiles_m * gridDim.x);
+      const int64_t rest = tiles_m * gridDim.x - p.head_tiles;
+      if (e >= rest * pm1) return;
+      const int tt = e / pm1;
+      split = 1 + e % pm1;
+      tail_unit = (int64_t)tt * p.tail_pieces + split;
+      const int64_t tile = p.head_tiles + tt;
+      tile_n = tile % gridDim.x;
+      tile_m = tile / gridDim.x;
+    }
+  }
+  const int64_t n0 = tile_n * 128;
+  const int64_t m0 = tile_m * BN;
+  const int kb0 = split * kbps;
+  const int kb1 = min(kb0 + kbps, total_kb);
   const int nkb = max(kb1 - kb0, 0);
 
   if (threadIdx.x == 0) {
@@ -354,7 +386,21 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
     go = epilogue_vote<kEpi>(go);
     if (go) {
       tc_fence_after();
-      const bool direct = p.splits == 1;
+      const bool direct = p.splits == 1 && tail_unit < 0;
+      // This row's fp32 destination (Y, the split's partial rows, or the tail
+      // piece's partial tile) and the distance between consecutive tokens there.
+      const bool out16 = direct && p.y_bf16;
+      float *dst;
+      int64_t ld = N;
+      if (tail_unit >= 0) {
+        dst = p.ws + tail_unit * (int64_t)BN * 128 + r;
+        ld = 128;
+      } else if (direct) {
+        dst = static_cast<float *>(p.Y) + m0 * N + n;
+      } else {
+        dst = p.ws + ((int64_t)split * M + m0) * N + n;
+      }
+      __nv_bfloat16 *dst16 = static_cast<__nv_bfloat16 *>(p.Y) + m0 * N + n;
 #pragma unroll 1
       for (int c = h * (BN / 32 / kHalves); c < (h + 1) * (BN / 32 / kHalves); ++c) {  // this warp's columns
         uint32_t v[32];
@@ -363,23 +409,19 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
         if (!row_ok) continue;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int64_t m = m0 + c * 32 + j;
-          if (m < M) {
+          const int t = c * 32 + j;
+          if (m0 + t < M) {
             const float val = __uint_as_float(v[j]);
-            if (direct) {
-              if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.Y)[m * N + n] = __float2bfloat16_rn(val);
-              else static_cast<float *>(p.Y)[m * N + n] = val;
-            } else {
-              p.ws[((int64_t)split * M + m) * N + n] = val;
-            }
+            if (out16) dst16[t * N] = __float2bfloat16_rn(val);
+            else dst[t * ld] = val;
           }
         }
       }
-      if (!direct) {
+      if (!direct && tail_unit < 0) {
         // last CTA of this output tile to arrive sums the split-K partials
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"n"(kEpi) : "memory");
-        const int64_t tile = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+        const int64_t tile = tile_m * gridDim.x + tile_n;
         if (r == 0 && h == 0) {
           const uint32_t prev = atomicAdd(&p.counters[tile], 1u);
           *s_last = prev == (uint32_t)(p.splits - 1);
@@ -445,12 +487,67 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
 template <int BN, bool kBf16, bool kAwq>
 cudaError_t launch_t(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, cudaStream_t stream) {
   using Cfg = TcCfg<BN>;
-  auto kern = gemm_tc_kernel<BN, kBf16, kAwq>;
-  static std::atomic<int> smem_set[kAttrDevices];  // largest size already set, per device
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), Cfg::kSmem, smem_set);
+  auto kern = p.tail_pieces > 0 ? gemm_tc_kernel<BN, kBf16, kAwq, true> : gemm_tc_kernel<BN, kBf16, kAwq, false>;
+  static std::atomic<int> smem_set[kAttrDevices][2];  // largest size already set, per device and variant
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), Cfg::kSmem, smem_set[p.tail_pieces > 0]);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + BN - 1) / BN), (unsigned)p.splits);
+  if (p.tail_pieces > 0) {  // extra rows of CTAs for pieces 1.. of the tail tiles
+    const int64_t extra = ((int64_t)grid.x * grid.y - p.head_tiles) * (p.tail_pieces - 1);
+    grid.y += (unsigned)((extra + grid.x - 1) / grid.x);
+  }
   kern<<<grid, TcWarps<kAwq>::kThreads, Cfg::kSmem, stream>>>(tmX, tmP, p);
+  return cudaGetLastError();
+}
+
+// Sums the tail pieces' partial tiles in piece order and writes Y.  One thread
+// per 4 output channels of one token of one tail tile; partials [u][BN][128].
+template <int BN>
+__global__ void __launch_bounds__(256) tail_reduce_kernel(const TcParams p) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t q = idx % 32, j = (idx / 32) % BN, tt = idx / (32 * BN);
+  const int64_t tiles = p.ntx * ((p.M + BN - 1) / BN);
+  if (tt >= tiles - p.head_tiles) return;
+  const int64_t t = p.head_tiles + tt;
+  const int64_t m = (t / p.ntx) * BN + j;
+  const int64_t n = (t % p.ntx) * 128 + 4 * q;
+  if (m >= p.M || n >= p.N) return;
+  const float4 *src = reinterpret_cast<const float4 *>(p.ws) + (tt * p.tail_pieces * BN + j) * 32 + q;
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  int s = 0;
+  for (; s + 4 <= p.tail_pieces; s += 4) {  // 4 loads in flight, summed in piece order
+    float4 v[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) v[c] = __ldcg(src + (int64_t)(s + c) * BN * 32);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      acc[0] += v[c].x; acc[1] += v[c].y; acc[2] += v[c].z; acc[3] += v[c].w;
+    }
+  }
+  for (; s < p.tail_pieces; ++s) {
+    const float4 v = __ldcg(src + (int64_t)s * BN * 32);
+    acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
+  }
+  const int nv = p.N - n < 4 ? (int)(p.N - n) : 4;
+  if (p.y_bf16) {
+    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.Y) + m * p.N + n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < nv) y[i] = __float2bfloat16_rn(acc[i]);
+  } else {
+    float *y = static_cast<float *>(p.Y) + m * p.N + n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < nv) y[i] = acc[i];
+  }
+}
+
+template <int BN>
+cudaError_t launch_tail_reduce_bn(const TcParams &p, cudaStream_t stream) {
+  const int64_t tiles = p.ntx * ((p.M + BN - 1) / BN);
+  const int64_t threads = (tiles - p.head_tiles) * BN * 32;
+  if (threads <= 0) return cudaSuccess;
+  tail_reduce_kernel<BN><<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -470,6 +567,15 @@ cudaError_t launch_gemm_tc(const CUtensorMap &tmX, const CUtensorMap &tmP, const
     case 64: return tc_impl::launch_bn<64>(tmX, tmP, p, x_bf16, stream);
     case 128: return tc_impl::launch_bn<128>(tmX, tmP, p, x_bf16, stream);
     default: return tc_impl::launch_bn<256>(tmX, tmP, p, x_bf16, stream);
+  }
+}
+
+// Tail mode only: the reduction of the tail pieces, enqueued after the GEMM.
+cudaError_t launch_tail_reduce(const TcParams &p, int bn, cudaStream_t stream) {
+  switch (bn) {
+    case 64: return tc_impl::launch_tail_reduce_bn<64>(p, stream);
+    case 128: return tc_impl::launch_tail_reduce_bn<128>(p, stream);
+    default: return tc_impl::launch_tail_reduce_bn<256>(p, stream);
   }
 }
 

@@ -171,6 +171,8 @@ struct GemmPlan {
   bool sc_tma = false;
   // K2
   int bn = 256, splits = 1, kb_per_split = 1;
+  int64_t head_tiles = 0;  // tail mode (tail_pieces > 0): tiles computed whole
+  int tail_pieces = 0;
   // K3 workspace regions (bytes from the start of the workspace)
   size_t xp_off = 0, xexp_off = 0, part_off = 0;
   size_t ws_bytes = 0;
@@ -300,6 +302,34 @@ GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_ca
   p.splits = (int)splits;
   p.kb_per_split = (int)kbps;
   if (splits > 1) p.ws_bytes = kCounterBytes + (size_t)splits * M * N * 4;
+  // Tail split: where the tiles fill whole waves of resident CTAs and leave a
+  // last wave at most half full, that wave's tiles are cut along K into pieces
+  // (each >= 16 k-blocks) that run on the SMs the full waves free; a reduction
+  // kernel sums the pieces.  At the 70B qkv shape, M = 512 (160 tiles of
+  // 128 x 256 on 148 SMs), the second wave otherwise costs as much as the first.
+  // Measured on B200 at the 70B shapes (M = 512, 2048, 8192), it pays where the
+  // part of a wave it saves, total_kb * (1 - 1 / pieces) k-blocks of BN / 256
+  // work, exceeds about 45 + 13 * (full waves) k-block times: the reduction and
+  // the pieces' start-up, and a cost per wave of the tail kernel's whole tiles
+  // (qkv at M = 512 and down at M = 2048 gained 20 % and 10 %; gate_up at
+  // M = 2048, 24 full waves, lost 5 %).  W4_FORCE_TAIL=1 skips that test (tests).
+  if (splits == 1 && tiles > slots) {
+    const int64_t rest = tiles % slots;
+    if (rest > 0 && 2 * rest <= slots) {
+      int64_t pieces = std::min<int64_t>(slots / rest, total_kb / 16);
+      while (pieces > 1 && kCounterBytes + (size_t)(rest * pieces) * p.bn * 128 * 4 > ws_cap) --pieces;
+      const double saved = (double)total_kb * (1.0 - 1.0 / (double)std::max<int64_t>(pieces, 1)) * p.bn / 256.0;
+      const bool pays = saved > 45.0 + 13.0 * (double)(tiles / slots) || getenv("W4_FORCE_TAIL");
+      if (pieces >= 2 && pays) {
+        const int64_t kpp = cdiv(total_kb, pieces);
+        pieces = cdiv(total_kb, kpp);
+        p.head_tiles = tiles - rest;
+        p.tail_pieces = (int)pieces;
+        p.kb_per_split = (int)kpp;
+        p.ws_bytes = kCounterBytes + (size_t)(rest * pieces) * p.bn * 128 * 4;
+      }
+    }
+  }
   return p;
 }
 
@@ -371,8 +401,11 @@ void debug_plan(const GemmPlan &p, int64_t M, int64_t N, int64_t K) {
               (long long)M, (long long)N, (long long)K, p.t8, p.kr, p.kslices, p.grid_x, p.slots, p.xs_bytes,
               (int)p.sc_tma, p.ws_bytes);
     else
-      fprintf(stderr, "[w4] M=%lld N=%lld K=%lld tensor-core: bn=%d splits=%d kb_per_split=%d ws=%zu\n",
-              (long long)M, (long long)N, (long long)K, p.bn, p.splits, p.kb_per_split, p.ws_bytes);
+      fprintf(stderr,
+              "[w4] M=%lld N=%lld K=%lld tensor-core: bn=%d splits=%d kb_per_split=%d head_tiles=%lld "
+              "tail_pieces=%d ws=%zu\n",
+              (long long)M, (long long)N, (long long)K, p.bn, p.splits, p.kb_per_split, (long long)p.head_tiles,
+              p.tail_pieces, p.ws_bytes);
   }
 }
 
@@ -615,8 +648,13 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
   p.Y = Y; p.y_bf16 = y_dtype == W4_BF16;
   p.ws = partials; p.counters = counters; p.splits = plan.splits; p.kb_per_split = plan.kb_per_split;
   p.group = group;
+  p.head_tiles = plan.head_tiles; p.tail_pieces = plan.tail_pieces; p.ntx = (N + 127) / 128;
   e = w4::launch_gemm_tc(tmX, tmP, p, xbf16, plan.bn, s);
   if (e != cudaSuccess) return cuda_fail(e, "tensor-core gemm launch");
+  if (plan.tail_pieces > 0) {
+    e = w4::launch_tail_reduce(p, plan.bn, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tail reduction launch");
+  }
   if (row_ptr) {
     e = w4::launch_sparse_add(X, xbf16, M, N, K, row_ptr, col, val, Y, y_dtype == W4_BF16, s);
     if (e != cudaSuccess) return cuda_fail(e, "sparse add");
