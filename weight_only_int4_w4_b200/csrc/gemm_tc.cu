@@ -48,6 +48,9 @@ struct TcParams {
   int64_t head_tiles;
   int tail_pieces;
   int64_t ntx;  // output tiles along N
+  // 1: whole tiles write Y through the tmY tensor map (N * element size is a
+  // multiple of 16 bytes and M, N >= 32); tail pieces always use tmT.
+  int y_tma;
 };
 
 namespace tc_impl {
@@ -83,6 +86,7 @@ struct TcCfg {
   static constexpr int kNS = 4;
   static constexpr int kXStage = BN * 128;
   static_assert(BN + 32 * kNS <= 512, "accumulator + A stages exceed TMEM");
+  static_assert(kNS * kXStage >= BN * 128 * 4, "the epilogue stages a BN x 128 fp32 tile in the X ring");
   static constexpr uint32_t kTmemCols = (BN + 32 * kNS <= 256) ? 256u : 512u;
   static constexpr int kSStage = kBK * 4;  // AWQ s of the stage's 64 channels (fp32)
   static constexpr int kSmem = 1024 /*align slack*/ + kNS * (kXStage + kPStage + kSStage) + (3 * kNS + 2) * 8;
@@ -194,6 +198,7 @@ __device__ __forceinline__ bool epilogue_vote(bool v) {
 template <int BN, bool kBf16, bool kAwq, bool kTail>
 __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
   constexpr int kNS = Cfg::kNS;
@@ -387,33 +392,61 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
     if (go) {
       tc_fence_after();
       const bool direct = p.splits == 1 && tail_unit < 0;
-      // This row's fp32 destination (Y, the split's partial rows, or the tail
-      // piece's partial tile) and the distance between consecutive tokens there.
-      const bool out16 = direct && p.y_bf16;
-      float *dst;
-      int64_t ld = N;
-      if (tail_unit >= 0) {
-        dst = p.ws + tail_unit * (int64_t)BN * 128 + r;
-        ld = 128;
-      } else if (direct) {
-        dst = static_cast<float *>(p.Y) + m0 * N + n;
-      } else {
-        dst = p.ws + ((int64_t)split * M + m0) * N + n;
-      }
-      __nv_bfloat16 *dst16 = static_cast<__nv_bfloat16 *>(p.Y) + m0 * N + n;
+      if (tail_unit >= 0 || (direct && p.y_tma)) {
+        // Each warp stages its 32 rows x 32 tokens of a chunk in the X ring (idle
+        // once the accumulator is complete) as [token][row] and writes the chunk
+        // with one TMA store, which clips rows >= M and columns >= N.  Measured on
+        // B200: per-thread stores of the same tile took 5-13 us per CTA.
+        const bool out16 = tail_unit < 0 && p.y_bf16;
+        const int esz = out16 ? 2 : 4;
+        uint8_t *stage = sX + (size_t)q * (BN / 32) * (32 * 32 * esz);
 #pragma unroll 1
-      for (int c = h * (BN / 32 / kHalves); c < (h + 1) * (BN / 32 / kHalves); ++c) {  // this warp's columns
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), v);
-        tc_wait_ld();
-        if (!row_ok) continue;
+        for (int c = h * (BN / 32 / kHalves); c < (h + 1) * (BN / 32 / kHalves); ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), v);
+          tc_wait_ld();
+          if (m0 + c * 32 >= M) continue;
+          uint8_t *chunk = stage + (size_t)c * (32 * 32 * esz);
+          if (out16) {
+            __nv_bfloat16 *c16 = reinterpret_cast<__nv_bfloat16 *>(chunk);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = c * 32 + j;
-          if (m0 + t < M) {
-            const float val = __uint_as_float(v[j]);
-            if (out16) dst16[t * N] = __float2bfloat16_rn(val);
-            else dst[t * ld] = val;
+            for (int j = 0; j < 32; ++j) c16[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j]));
+          } else {
+            float *c32 = reinterpret_cast<float *>(chunk);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) c32[j * 32 + lane] = __uint_as_float(v[j]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (tail_unit >= 0) tma_store_2d(&tmT, chunk, q * 32, (int32_t)(tail_unit * BN + c * 32));
+            else if (n0 + q * 32 < N) tma_store_2d(&tmY, chunk, (int32_t)(n0 + q * 32), (int32_t)(m0 + c * 32));
+            bulk_commit_group();
+          }
+        }
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      } else {
+        // Per-thread stores (Y rows not 16-byte multiples, or split-K partials):
+        // this row's fp32 destination, Y or the split's partial rows, with a
+        // token stride of N, or the bf16 Y row.
+        const bool out16 = direct && p.y_bf16;
+        float *dst = direct ? static_cast<float *>(p.Y) + m0 * N + n : p.ws + ((int64_t)split * M + m0) * N + n;
+        __nv_bfloat16 *dst16 = static_cast<__nv_bfloat16 *>(p.Y) + m0 * N + n;
+#pragma unroll 1
+        for (int c = h * (BN / 32 / kHalves); c < (h + 1) * (BN / 32 / kHalves); ++c) {  // this warp's columns
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), v);
+          tc_wait_ld();
+          if (!row_ok) continue;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = c * 32 + j;
+            if (m0 + t < M) {
+              const float val = __uint_as_float(v[j]);
+              if (out16) dst16[t * N] = __float2bfloat16_rn(val);
+              else dst[t * N] = val;
+            }
           }
         }
       }
@@ -485,7 +518,8 @@ __global__ void __launch_bounds__(TcWarps<kAwq>::kThreads, kAwq ? 1 : 2)
 }
 
 template <int BN, bool kBf16, bool kAwq>
-cudaError_t launch_t(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, cudaStream_t stream) {
+cudaError_t launch_t(const CUtensorMap &tmX, const CUtensorMap &tmP, const CUtensorMap &tmY, const CUtensorMap &tmT,
+                     const TcParams &p, cudaStream_t stream) {
   using Cfg = TcCfg<BN>;
   auto kern = p.tail_pieces > 0 ? gemm_tc_kernel<BN, kBf16, kAwq, true> : gemm_tc_kernel<BN, kBf16, kAwq, false>;
   static std::atomic<int> smem_set[kAttrDevices][2];  // largest size already set, per device and variant
@@ -496,7 +530,7 @@ cudaError_t launch_t(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcPar
     const int64_t extra = ((int64_t)grid.x * grid.y - p.head_tiles) * (p.tail_pieces - 1);
     grid.y += (unsigned)((extra + grid.x - 1) / grid.x);
   }
-  kern<<<grid, TcWarps<kAwq>::kThreads, Cfg::kSmem, stream>>>(tmX, tmP, p);
+  kern<<<grid, TcWarps<kAwq>::kThreads, Cfg::kSmem, stream>>>(tmX, tmP, tmY, tmT, p);
   return cudaGetLastError();
 }
 
@@ -552,21 +586,25 @@ cudaError_t launch_tail_reduce_bn(const TcParams &p, cudaStream_t stream) {
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, bool bf16,
-                      cudaStream_t stream) {
+cudaError_t launch_bn(const CUtensorMap &tmX, const CUtensorMap &tmP, const CUtensorMap &tmY,
+                      const CUtensorMap &tmT, const TcParams &p, bool bf16, cudaStream_t stream) {
   const bool awq = p.awq_s != nullptr;
-  if (bf16) return awq ? launch_t<BN, true, true>(tmX, tmP, p, stream) : launch_t<BN, true, false>(tmX, tmP, p, stream);
-  return awq ? launch_t<BN, false, true>(tmX, tmP, p, stream) : launch_t<BN, false, false>(tmX, tmP, p, stream);
+  if (bf16)
+    return awq ? launch_t<BN, true, true>(tmX, tmP, tmY, tmT, p, stream)
+               : launch_t<BN, true, false>(tmX, tmP, tmY, tmT, p, stream);
+  return awq ? launch_t<BN, false, true>(tmX, tmP, tmY, tmT, p, stream)
+             : launch_t<BN, false, false>(tmX, tmP, tmY, tmT, p, stream);
 }
 
 }  // namespace tc_impl
 
-cudaError_t launch_gemm_tc(const CUtensorMap &tmX, const CUtensorMap &tmP, const TcParams &p, bool x_bf16, int bn,
+cudaError_t launch_gemm_tc(const CUtensorMap &tmX, const CUtensorMap &tmP, const CUtensorMap &tmY,
+                           const CUtensorMap &tmT, const TcParams &p, bool x_bf16, int bn,
                            cudaStream_t stream) {
   switch (bn) {
-    case 64: return tc_impl::launch_bn<64>(tmX, tmP, p, x_bf16, stream);
-    case 128: return tc_impl::launch_bn<128>(tmX, tmP, p, x_bf16, stream);
-    default: return tc_impl::launch_bn<256>(tmX, tmP, p, x_bf16, stream);
+    case 64: return tc_impl::launch_bn<64>(tmX, tmP, tmY, tmT, p, x_bf16, stream);
+    case 128: return tc_impl::launch_bn<128>(tmX, tmP, tmY, tmT, p, x_bf16, stream);
+    default: return tc_impl::launch_bn<256>(tmX, tmP, tmY, tmT, p, x_bf16, stream);
   }
 }
 

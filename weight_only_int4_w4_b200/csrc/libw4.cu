@@ -649,7 +649,25 @@ w4_status gemm_common(const void *X, w4_dtype x_dtype, int64_t M, int64_t N, int
   p.ws = partials; p.counters = counters; p.splits = plan.splits; p.kb_per_split = plan.kb_per_split;
   p.group = group;
   p.head_tiles = plan.head_tiles; p.tail_pieces = plan.tail_pieces; p.ntx = (N + 127) / 128;
-  e = w4::launch_gemm_tc(tmX, tmP, p, xbf16, plan.bn, s);
+  // Tile stores by TMA (32 x 32 boxes): Y where its rows are 16-byte multiples,
+  // and the tail pieces' partial tiles [tail tiles x pieces x BN][128] fp32.
+  // Unused maps are copies of tmX and are never read.
+  CUtensorMap tmY = tmX, tmT = tmX;
+  const int ysz = y_dtype == W4_BF16 ? 2 : 4;
+  if ((N * ysz) % 16 == 0 && M >= 32 && N >= 32) {
+    CUresult r = encode_2d(enc, &tmY, ysz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y,
+                           (uint64_t)N, (uint64_t)M, (uint64_t)N * ysz, 32u, 32u, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for Y failed (CUresult %d)", (int)r);
+    p.y_tma = 1;
+  }
+  if (plan.tail_pieces > 0) {
+    const uint64_t rows = (uint64_t)(cdiv(N, 128) * cdiv(M, plan.bn) - plan.head_tiles) * plan.tail_pieces * plan.bn;
+    CUresult r = encode_2d(enc, &tmT, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, partials, 128u, rows, 512u, 32u, 32u,
+                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (r != CUDA_SUCCESS) return fail(W4_ERR_CUDA, "tensor map for tail partials failed (CUresult %d)", (int)r);
+  }
+  e = w4::launch_gemm_tc(tmX, tmP, tmY, tmT, p, xbf16, plan.bn, s);
   if (e != cudaSuccess) return cuda_fail(e, "tensor-core gemm launch");
   if (plan.tail_pieces > 0) {
     e = w4::launch_tail_reduce(p, plan.bn, s);
