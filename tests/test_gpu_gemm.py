@@ -165,11 +165,8 @@ def test_split_k_reduction_ragged(w4, monkeypatch, capfd, M, N, K, awq, splits):
 def test_tail_split_last_wave(w4, monkeypatch, capfd, M, N, K, awq, out, bn, tiles, pieces):
     """Tensor-core tail split: whole tiles fill complete waves and the last,
     mostly empty wave's tiles are cut along K; the reduction kernel sums the
-    pieces.  Every output of the tail tiles is checked, with a sample elsewhere.
-    W4_FORCE_TAIL takes the split at these small depths, where the planner's
-    cost rule would keep whole tiles."""
+    pieces.  Every output of the tail tiles is checked, with a sample elsewhere."""
     monkeypatch.setenv("W4_DEBUG_PLAN", "1")
-    monkeypatch.setenv("W4_FORCE_TAIL", "1")
     ntx = (N + 127) // 128
     slots = 148 * (1 if (awq or bn == 256) else 2)
     head = tiles - tiles % slots

@@ -307,20 +307,16 @@ GemmPlan plan_tc(int64_t M, int64_t N, int64_t K, bool awq, int sm, size_t ws_ca
   // (each >= 16 k-blocks) that run on the SMs the full waves free; a reduction
   // kernel sums the pieces.  At the 70B qkv shape, M = 512 (160 tiles of
   // 128 x 256 on 148 SMs), the second wave otherwise costs as much as the first.
-  // Measured on B200 at the 70B shapes (M = 512, 2048, 8192), it pays where the
-  // part of a wave it saves, total_kb * (1 - 1 / pieces) k-blocks of BN / 256
-  // work, exceeds about 45 + 13 * (full waves) k-block times: the reduction and
-  // the pieces' start-up, and a cost per wave of the tail kernel's whole tiles
-  // (qkv at M = 512 and down at M = 2048 gained 20 % and 10 %; gate_up at
-  // M = 2048, 24 full waves, lost 5 %).  W4_FORCE_TAIL=1 skips that test (tests).
+  // Measured on B200 at the 70B shapes, with tiles stored by TMA, every call
+  // that qualifies ran as fast or faster split (gate_up at M = 512 447 -> 415 us,
+  // qkv and o_proj at M = 2048 312 -> 290 and 250 -> 231 us, qkv at M = 8192
+  // 1144 -> 1124 us; qkv at M = 512 137 -> 110 us before the TMA stores).
   if (splits == 1 && tiles > slots) {
     const int64_t rest = tiles % slots;
     if (rest > 0 && 2 * rest <= slots) {
       int64_t pieces = std::min<int64_t>(slots / rest, total_kb / 16);
       while (pieces > 1 && kCounterBytes + (size_t)(rest * pieces) * p.bn * 128 * 4 > ws_cap) --pieces;
-      const double saved = (double)total_kb * (1.0 - 1.0 / (double)std::max<int64_t>(pieces, 1)) * p.bn / 256.0;
-      const bool pays = saved > 45.0 + 13.0 * (double)(tiles / slots) || getenv("W4_FORCE_TAIL");
-      if (pieces >= 2 && pays) {
+      if (pieces >= 2) {
         const int64_t kpp = cdiv(total_kb, pieces);
         pieces = cdiv(total_kb, kpp);
         p.head_tiles = tiles - rest;
