@@ -90,3 +90,30 @@ def test_group32_needs_k_multiple_of_64(w4):
 
 def test_no_device_error(w4):
     assert w4.w4_device_error() == 0
+
+
+@pytest.mark.parametrize("group", [32, 64])
+def test_tail_split_with_small_groups(w4, monkeypatch, capfd, group):
+    """The tensor-core tail split (the last, mostly empty wave's tiles cut into
+    k-pieces summed by a reduction kernel) with groups of 32 and 64: every
+    output of the tail tiles, plus sampled rows elsewhere, against the oracle."""
+    monkeypatch.setenv("W4_DEBUG_PLAN", "1")
+    M, N, K = 300, 9688, 2048
+    tag = ("variants-tail", group)
+    W = synthetic.weight(K, N, 0.02, 0.0, tag)
+    X = synthetic.activations(M, K, "bf16", tag)
+    packed, scales, zeros = w4.w4_quantize(W.cuda(), group=group)
+    Y = w4.w4a16_gemm(X.cuda(), packed, scales, zeros, group=group)
+    torch.cuda.synchronize()
+    ntx = (N + 127) // 128
+    tiles = ntx * 2  # BN = 256 for M = 300
+    head = tiles - tiles % 148
+    tail_rows = {n for t in range(head, tiles) for n in range((t % ntx) * 128, min((t % ntx) * 128 + 128, N))}
+    rows = np.array(sorted(tail_rows | set(np.random.default_rng(group).choice(N, 48, replace=False).tolist())))
+    c, sc, zp = oracle.quantize(W.numpy()[rows], group=group)
+    What = oracle.dequant(c, sc, zp, group=group)
+    Yref, bound = oracle.gemm(X.float().numpy(), What)
+    check_close(Y.cpu().numpy()[:, rows], Yref, bound, what=f"tail G={group}")
+    err = capfd.readouterr().err
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert f"head_tiles={head} tail_pieces=2 " in err, err
