@@ -125,8 +125,10 @@ w4_status w4_pack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *packed,
  *   Y         device [M][N], y_dtype F32 or BF16 (overwritten)
  *   workspace device scratch of at least w4a16_gemm_workspace_size(M,N,K)
  *             bytes (may be NULL when that size is 0).  It must be zero-filled
- *             once before its first use; every call leaves it zero-filled
- *             again.  Calls that share a workspace must not overlap in time.
+ *             once before its first use.  Every call leaves its first 128 KiB
+ *             (tile arrival counters) zero again; the bytes after them hold
+ *             partial sums that each call writes before it reads them.  Calls
+ *             that share a workspace must not overlap in time.
  * Accuracy: |Y - Y_exact| <= 2e-3 * sum_k |X[m][k] * W^[n][k]| per element on
  * the library's test distributions (fp32 accumulation; the prefill path rounds
  * W^ to 16 bits once, the decode path keeps (q - z) exact and, with AWQ,
@@ -200,7 +202,7 @@ w4_status w4a16_gemm_host_async(const void *X_host, void *X_dev, w4_dtype x_dtyp
  *   best      HOST out: index of the best exponent
  *   workspace device scratch of w4_awq_search_workspace_size(Mc, N, K, group)
  *             bytes, zero-filled before its first use (it holds a w4a16_gemm
- *             workspace, left zero-filled by every call).
+ *             workspace, whose counters every call leaves zero).
  * Runs the quantizer and w4a16_gemm once per exponent and a dense fp32
  * reference GEMM once; synchronizes `stream` before returning.
  */

@@ -139,8 +139,8 @@ _ws_cache: dict = {}
 
 
 def workspace(M: int, N: int, K: int, device, stream=None) -> torch.Tensor | None:
-    """A zero-filled workspace (cached per device and stream) large enough for (M, N, K).
-    The library leaves it zero-filled after every call, so it can be reused."""
+    """A workspace (cached per device and stream) large enough for (M, N, K), zero-filled
+    when allocated.  Every call leaves its counters zero again, so it can be reused."""
     need = w4a16_gemm_workspace_size(M, N, K)
     if need == 0:
         return None
