@@ -182,6 +182,22 @@ def test_tail_split_last_wave(w4, monkeypatch, capfd, M, N, K, awq, out, bn, til
         assert f"bn={bn} splits=1 " in err and f"head_tiles={head} tail_pieces={pieces} " in err, err
 
 
+@pytest.mark.parametrize("M,N,K,out", [
+    (200, 1000, 512, "bf16"),  # ragged tokens (last 32-token box partly past M), last 128-row tile partly past N
+    (200, 904, 512, "f32"),    # the last tile's second 32-row box starts past N and is skipped
+    (33, 904, 512, "bf16"),    # one token past a 32-token box
+])
+def test_tma_store_epilogue_ragged(w4, monkeypatch, capfd, M, N, K, out):
+    """Tensor-core tiles written by 32 x 32 TMA stores (Y rows are 16-byte
+    multiples, M and N >= 32, one split): the stores clip at M and N, and
+    every output is checked."""
+    monkeypatch.setenv("W4_DEBUG_PLAN", "1")
+    _run_case(w4, M, N, K, path="tc", out_dtype=torch.bfloat16 if out == "bf16" else torch.float32,
+              tag=("tma-store", M, N, K, out))
+    err = capfd.readouterr().err
+    assert "splits=1 " in err and "tail_pieces=0 " in err, err
+
+
 def test_long_k_split_both_paths(w4):
     """K = 28672 (70B down_proj depth) at small M: split-K on both paths."""
     for path in ("gemv", "skinny", "tc"):
