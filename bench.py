@@ -13,6 +13,8 @@ Also reported on the same JSON line:
     the same rotating weight copies;
   * e2e: the same metric through the C ABI's host-buffer entry point
     (pinned X in, fp32 Y out, copies inside the timed region);
+  * e2e_batched: the same through the batched host-buffer entry point (the
+    step's four independent matmuls in one call: one copy in, one copy out);
   * quantize: the quantize+pack kernel on the same four layers (fp32 W in);
   * prefill: TFLOP/s of the tensor-core path at Llama-3-70B shapes, M = 8192;
   * cpu_baseline: the oracle (plain C, one core) on a bounded sample.
@@ -466,6 +468,54 @@ def e2e_leg(w4, layers, steps, warmup, world):
     return a.elapsed_time(b), h2d, d2h
 
 
+def e2e_batch_leg(w4, layers, steps, warmup, world):
+    """The step's four independent matmuls in one call of the batched host-buffer entry
+    (w4a16_gemm_host_batch_async): the four pinned X in one copy, the four matmuls, the
+    four fp32 Y back in one copy; the host waits for the stream once per step."""
+    xo, yo, offs = 0, 0, {}
+    for name in LAYERS:
+        L = layers[name]
+        offs[name] = (xo, yo)
+        xo += -(-2 * L["K"] // 16) * 16
+        yo += -(-4 * L["N"] // 16) * 16
+    Xh = torch.zeros(xo, dtype=torch.uint8).pin_memory()
+    for name in LAYERS:
+        x = layers[name]["X"].cpu().contiguous().view(torch.uint8).reshape(-1)
+        Xh[offs[name][0]:offs[name][0] + x.numel()] = x
+    Yh = torch.empty(yo, dtype=torch.uint8).pin_memory()
+    dev = layers[LAYERS[0]]["X"].device
+    Xd = torch.empty(xo, dtype=torch.uint8, device=dev)
+    Yd = torch.empty(yo, dtype=torch.uint8, device=dev)
+    ws = max((layers[n]["ws"] for n in LAYERS), key=lambda t: t.numel())
+    batches = []
+    for c in range(N_COPIES):
+        items = []
+        for name in LAYERS:
+            L = layers[name]
+            packed, scales, zeros = L["copies"][c]
+            items.append(dict(M=1, N=L["N"], K=L["K"], packed=packed, scales=scales, zeros=zeros,
+                              x_offset=offs[name][0], y_offset=offs[name][1]))
+        batches.append(w4.gemm_batch(items))
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        w4.w4a16_gemm_host_batch(batches[i % N_COPIES], Xh, Xd, Yh, Yd, ws=ws, stream=stream, wait=False)
+        stream.synchronize()  # the step's outputs are in host memory
+
+    for i in range(warmup):
+        step(i)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return a.elapsed_time(b), xo, yo
+
+
 def quantize_leg(w4, steps=5):
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev)
@@ -755,6 +805,8 @@ def main():
 
     e2e_ms, h2d, d2h = e2e_leg(w4, layers, max(20, args.steps // 4), args.warmup, world)
     e2e_value, e2e_ms = job_throughput(step_bytes * max(20, args.steps // 4), e2e_ms, world)
+    eb_ms, eb_h2d, eb_d2h = e2e_batch_leg(w4, layers, max(20, args.steps // 4), args.warmup, world)
+    eb_value, eb_ms = job_throughput(step_bytes * max(20, args.steps // 4), eb_ms, world)
     del layers
     torch.cuda.empty_cache()
 
@@ -807,6 +859,10 @@ def main():
                     "api": "w4a16_gemm_host_async per layer (pinned host X/Y, copies enqueued with the matmul), one stream wait per step",
                     "note": "the gap to value is host-side enqueueing of 4 x (copy in, matmul, copy out) and one "
                             "host synchronization per step; the copies themselves are only h2d+d2h bytes per step"},
+            "e2e_batched": {"value": round(eb_value, 2), "unit": "GB/s", "h2d_bytes_per_step": eb_h2d,
+                            "d2h_bytes_per_step": eb_d2h,
+                            "api": "w4a16_gemm_host_batch_async: the step's four independent matmuls in one call "
+                                   "(one copy in, four matmuls, one copy out), one stream wait per step"},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
             "repeats": repeats,

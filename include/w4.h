@@ -184,6 +184,52 @@ w4_status w4a16_gemm_host_async(const void *X_host, void *X_dev, w4_dtype x_dtyp
                                 w4_stream_t stream);
 
 /*
+ * One matmul of a host-buffer batch (w4a16_gemm_host_batch_async): the
+ * arguments of w4a16_gemm, with X and Y given as byte offsets into the batch's
+ * staging buffers instead of as pointers.
+ */
+typedef struct {
+  int64_t M, N, K;
+  int group;
+  w4_dtype x_dtype;        /* F16 or BF16 */
+  w4_dtype y_dtype;        /* F32 or BF16 */
+  const uint8_t *packed;   /* device, as produced by w4_quantize */
+  const uint16_t *scales;  /* device */
+  const uint16_t *zeros;   /* device */
+  const float *awq_s;      /* device [K] or NULL */
+  size_t x_offset;         /* bytes into X_host / X_dev, a multiple of 16 */
+  size_t y_offset;         /* bytes into Y_host / Y_dev, a multiple of 16 */
+} w4_gemm_item;
+
+/*
+ * Several independent fused dequantize-matmuls with host activations and
+ * outputs, in one call (ch. 22, section 22.3, as for w4a16_gemm): one copy of
+ * X_host[0, x_bytes) into X_dev, then items[0..count) in order on `stream` (item
+ * i reads [M][K] at X_dev + x_offset and writes [M][N] at Y_dev + y_offset), then
+ * one copy of Y_dev[0, y_bytes) into Y_host.  Nothing waits: Y_host is valid once
+ * the caller has synchronized `stream`.  A step of independent layers (projections
+ * with separate weights, experts) then pays two copies and one wait in all.
+ *   X_host, Y_host   HOST, pinned for asynchronous copies; unchanged (X_host) and
+ *                    unread (Y_host) until the stream reaches the copies
+ *   X_dev, Y_dev     device staging buffers of x_bytes and y_bytes
+ *   workspace        as for w4a16_gemm, at least the largest
+ *                    w4a16_gemm_workspace_size of the items; the items run one
+ *                    after another, so they share it
+ *   count            1 .. 4096
+ * Errors: every item is checked (shape, dtypes, offsets 16-byte aligned and
+ * inside x_bytes / y_bytes, pointers, workspace size) before anything is
+ * enqueued; W4_ERR_INVALID_ARG or W4_ERR_UNSUPPORTED then names the item in
+ * w4_last_error().  Failures of the enqueued work surface at the caller's
+ * synchronization.
+ */
+w4_status w4a16_gemm_host_batch_async(const w4_gemm_item *items, int count,
+                                      const void *X_host, void *X_dev,
+                                      size_t x_bytes, void *Y_host, void *Y_dev,
+                                      size_t y_bytes, void *workspace,
+                                      size_t workspace_bytes,
+                                      w4_stream_t stream);
+
+/*
  * AWQ scale search (offline, before w4_quantize).  AWQ quantizes W / s and
  * multiplies back by s, with s a per-input-channel activation magnitude from
  * calibration data (ch. 22 "Advanced inference optimisation", section 22.3);

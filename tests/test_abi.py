@@ -108,6 +108,49 @@ def test_gemm_rejects(lib):
     assert b"aligned" in lib.w4_last_error()
 
 
+class _Item(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("group", ctypes.c_int),
+                ("x_dtype", ctypes.c_int), ("y_dtype", ctypes.c_int), ("packed", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p), ("awq_s", ctypes.c_void_p),
+                ("x_offset", ctypes.c_size_t), ("y_offset", ctypes.c_size_t)]
+
+
+def test_batch_host_entry_rejects_before_enqueueing(lib):
+    """w4a16_gemm_host_batch_async checks every item on the host (no device call
+    happens before these rejections) and names the bad item."""
+    P = ctypes.c_void_p
+    lib.w4a16_gemm_host_batch_async.argtypes = [ctypes.POINTER(_Item), ctypes.c_int, P, P, ctypes.c_size_t, P, P,
+                                                ctypes.c_size_t, P, ctypes.c_size_t, P]
+    lib.w4a16_gemm_host_batch_async.restype = ctypes.c_int
+    lib.w4_last_error.restype = ctypes.c_char_p
+
+    def item(**kw):
+        it = _Item(kw.get("M", 1), kw.get("N", 256), kw.get("K", 1024), kw.get("G", 128), kw.get("xd", 2),
+                   kw.get("yd", 0), kw.get("P", A), A, A, None, kw.get("xo", 0), kw.get("yo", 0))
+        return it
+
+    def call(items, xb=1 << 20, yb=1 << 20, X=A, Y=A):
+        arr = (_Item * max(len(items), 1))(*items)
+        return lib.w4a16_gemm_host_batch_async(arr if items else None, len(items), A, X, xb, A, Y, yb, None, 0, None)
+
+    assert call([]) == 1
+    assert call([item()], X=None) == 1
+    assert call([item()], Y=A + 8) == 1                   # staging buffers must be 16-byte aligned
+    assert call([item(), item(M=0)]) == 1
+    assert b"item 1" in lib.w4_last_error()
+    assert call([item(xd=0)]) == 2                         # fp32 activations are not served
+    assert call([item(yd=1)]) == 2                         # fp16 output is not served
+    assert call([item(G=48)]) == 2
+    assert call([item(P=A + 2)]) == 1
+    assert call([item(xo=8)]) == 1                         # offsets are 16-byte multiples
+    assert call([item(), item(xo=2064)], xb=4096) == 1     # item 1's 2048 bytes of X end past 4096
+    assert b"item 1" in lib.w4_last_error() and b"outside" in lib.w4_last_error()
+    assert call([item(xo=4096)], xb=4096) == 1
+    assert b"outside" in lib.w4_last_error()
+    assert call([item(N=256, yo=1024)], yb=1024 + 1023) == 1  # one row of 256 fp32 outputs needs 1024 bytes
+    assert b"outside" in lib.w4_last_error()
+
+
 def test_workspace_size_plan(lib):
     _setup(lib)
     # decode of a 14336-deep layer splits K across CTAs -> needs partials + counters

@@ -268,6 +268,48 @@ def test_host_entry_point_async_waits_once(w4):
         check_close(Yh.numpy(), Yref, bound, what="host async")
 
 
+def test_host_batch_entry_matches_the_oracle_and_single_calls(w4):
+    """Four independent matmuls through w4a16_gemm_host_batch_async (one copy in,
+    the matmuls, one copy out, one wait): decode, small-M and prefill shapes, f16
+    and bf16 activations, fp32 and bf16 outputs, one with AWQ.  Each output matches
+    the oracle and, bit for bit, the same matmul through w4a16_gemm."""
+    cases = [(1, 640, 2048, "bf16", torch.float32, False), (5, 384, 1024, "f16", torch.bfloat16, True),
+             (24, 512, 1024, "bf16", torch.float32, False), (300, 256, 512, "bf16", torch.bfloat16, False)]
+    items, keep, xo, yo = [], [], 0, 0
+    for i, (M, N, K, xd, yd, awq) in enumerate(cases):
+        tag = ("host-batch", i)
+        W = synthetic.weight(K, N, 0.02, 0.0, tag)
+        s = synthetic.awq_scale(K, tag) if awq else None
+        X = synthetic.activations(M, K, xd, tag)
+        packed, scales, zeros, (codes, sc, zp) = _upload_oracle_weights(W.numpy(), None if s is None else s.numpy())
+        s_dev = None if s is None else s.cuda()
+        items.append(dict(M=M, N=N, K=K, packed=packed, scales=scales, zeros=zeros, awq_s=s_dev, x_offset=xo,
+                          y_offset=yo, x_dtype=X.dtype, y_dtype=yd))
+        keep.append((X, s, s_dev, codes, sc, zp, xo, yo, yd))
+        xo += -(-M * K * 2 // 16) * 16
+        yo += -(-M * N * (4 if yd == torch.float32 else 2) // 16) * 16
+    Xh = torch.zeros(xo, dtype=torch.uint8).pin_memory()
+    for (X, *_rest), it in zip(keep, items):
+        Xh[it["x_offset"]:it["x_offset"] + X.numel() * 2] = X.contiguous().view(torch.uint8).reshape(-1)
+    Yh = torch.full((yo,), 0xFF, dtype=torch.uint8).pin_memory()
+    Xd = torch.empty(xo, dtype=torch.uint8, device="cuda")
+    Yd = torch.empty(yo, dtype=torch.uint8, device="cuda")
+    need = max(w4.w4a16_gemm_workspace_size(it["M"], it["N"], it["K"]) for it in items)
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    w4.w4a16_gemm_host_batch(w4.gemm_batch(items), Xh, Xd, Yh, Yd, ws=ws, stream=stream, wait=True)
+    for (X, s, s_dev, codes, sc, zp, xo_i, yo_i, yd), it in zip(keep, items):
+        M, N = it["M"], it["N"]
+        nb = M * N * (4 if yd == torch.float32 else 2)
+        Yb = Yh[yo_i:yo_i + nb].view(yd).reshape(M, N)
+        What = oracle.dequant(codes, sc, zp, None if s is None else s.numpy())
+        Yref, bound = oracle.gemm(X.float().numpy(), What)
+        check_close(Yb.float().numpy(), Yref, bound, out_bf16=yd == torch.bfloat16, what=f"batch M={M}")
+        Y1 = w4.w4a16_gemm(X.cuda(), it["packed"], it["scales"], it["zeros"], s_dev, out_dtype=yd)
+        torch.cuda.synchronize()
+        assert torch.equal(Y1.cpu().view(torch.uint8), Yb.view(torch.uint8)), f"batch M={M}: not the single-call bits"
+
+
 def test_short_workspace_rejected(w4):
     M, N, K = 1, 4096, 14336
     need = w4.w4a16_gemm_workspace_size(M, N, K)

@@ -723,6 +723,68 @@ w4_status w4a16_gemm_host(const void *X_host, void *X_dev, w4_dtype x_dtype, int
   return W4_OK;
 }
 
+w4_status w4a16_gemm_host_batch_async(const w4_gemm_item *items, int count, const void *X_host, void *X_dev,
+                                      size_t x_bytes, void *Y_host, void *Y_dev, size_t y_bytes, void *workspace,
+                                      size_t workspace_bytes, w4_stream_t stream) {
+  t_last_error.clear();
+  if (!items || count < 1 || count > 4096) return fail(W4_ERR_INVALID_ARG, "items: need 1..4096, got %d", count);
+  if (!X_host || !Y_host || !X_dev || !Y_dev) return fail(W4_ERR_INVALID_ARG, "null host or staging buffer");
+  if (!aligned16(X_dev) || !aligned16(Y_dev)) return fail(W4_ERR_INVALID_ARG, "staging buffers must be 16-byte aligned");
+  // Everything an item's matmul would reject is checked here, before the copy of
+  // X is enqueued, so a bad item leaves nothing half done on the stream.
+  for (int i = 0; i < count; ++i) {
+    const w4_gemm_item &it = items[i];
+    w4_status st = check_shape(it.M, it.N, it.K, it.group);
+    if (st != W4_OK) return fail(st, "item %d: %s", i, t_last_error.c_str());
+    if (it.x_dtype != W4_F16 && it.x_dtype != W4_BF16)
+      return fail(W4_ERR_UNSUPPORTED, "item %d: activation dtype must be F16 or BF16", i);
+    if (it.y_dtype != W4_F32 && it.y_dtype != W4_BF16)
+      return fail(W4_ERR_UNSUPPORTED, "item %d: output dtype must be F32 or BF16", i);
+    if (!it.packed || !it.scales || !it.zeros) return fail(W4_ERR_INVALID_ARG, "item %d: null weights", i);
+    if (!aligned16(it.packed) || !aligned16(it.scales) || !aligned16(it.zeros) || (it.awq_s && !aligned16(it.awq_s)))
+      return fail(W4_ERR_INVALID_ARG, "item %d: device pointers must be 16-byte aligned", i);
+    if (it.x_offset % 16 != 0 || it.y_offset % 16 != 0)
+      return fail(W4_ERR_INVALID_ARG, "item %d: offsets must be multiples of 16 bytes", i);
+    const size_t xb = (size_t)it.M * it.K * 2, yb = (size_t)it.M * it.N * (it.y_dtype == W4_F32 ? 4 : 2);
+    if (it.x_offset > x_bytes || xb > x_bytes - it.x_offset)
+      return fail(W4_ERR_INVALID_ARG, "item %d: X [%zu, %zu) is outside the %zu staged bytes", i, it.x_offset,
+                  it.x_offset + xb, x_bytes);
+    if (it.y_offset > y_bytes || yb > y_bytes - it.y_offset)
+      return fail(W4_ERR_INVALID_ARG, "item %d: Y [%zu, %zu) is outside the %zu staged bytes", i, it.y_offset,
+                  it.y_offset + yb, y_bytes);
+  }
+  int sm = 0;
+  cudaError_t e = current_sm_count(&sm);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  for (int i = 0; i < count; ++i) {
+    const w4_gemm_item &it = items[i];
+    const GemmPlan plan = it.group == w4::kGroup ? plan_gemm(it.M, it.N, it.K, it.awq_s != nullptr, sm)
+                                                 : plan_tc(it.M, it.N, it.K, it.awq_s != nullptr, sm);
+    if (it.group != w4::kGroup && (it.K % 64 != 0 || forced_path() == kPathGemv || forced_path() == kPathSkinny))
+      return fail(W4_ERR_UNSUPPORTED, "item %d: group=%d needs K a multiple of 64 and the tensor-core kernel", i,
+                  it.group);
+    if (plan.path == 0 || (plan.path == kPathGemv && !w4::gemv_supports(it.M, it.awq_s != nullptr)))
+      return fail(W4_ERR_UNSUPPORTED, "item %d: the forced kernel (W4_FORCE_PATH) cannot serve this shape", i);
+    if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes))
+      return fail(W4_ERR_INVALID_ARG, "item %d: workspace too small: need %zu bytes, got %zu", i, plan.ws_bytes,
+                  workspace ? workspace_bytes : (size_t)0);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  e = cudaMemcpyAsync(X_dev, X_host, x_bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy X to device");
+  for (int i = 0; i < count; ++i) {
+    const w4_gemm_item &it = items[i];
+    const w4_status st =
+        w4a16_gemm(static_cast<uint8_t *>(X_dev) + it.x_offset, it.x_dtype, it.M, it.N, it.K, it.group, it.packed,
+                   it.scales, it.zeros, it.awq_s, static_cast<uint8_t *>(Y_dev) + it.y_offset, it.y_dtype, workspace,
+                   workspace_bytes, stream);
+    if (st != W4_OK) return fail(st, "item %d: %s", i, t_last_error.c_str());
+  }
+  e = cudaMemcpyAsync(Y_host, Y_dev, y_bytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy Y to host");
+  return W4_OK;
+}
+
 w4_status w4_device_error(int *flag) {
   t_last_error.clear();
   if (!flag) return fail(W4_ERR_INVALID_ARG, "null flag");

@@ -53,14 +53,25 @@ _lib.w4_gptq_workspace_size.argtypes = [_I64, _I64]
 _lib.w4_gptq_workspace_size.restype = _SZ
 _lib.w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
 _lib.w4a16_gemm_workspace_size.restype = _SZ
+
+
+class GemmItem(ctypes.Structure):
+    """w4_gemm_item of include/w4.h: one matmul of a host-buffer batch."""
+    _fields_ = [("M", _I64), ("N", _I64), ("K", _I64), ("group", ctypes.c_int), ("x_dtype", ctypes.c_int),
+                ("y_dtype", ctypes.c_int), ("packed", _P), ("scales", _P), ("zeros", _P), ("awq_s", _P),
+                ("x_offset", _SZ), ("y_offset", _SZ)]
+
+
+_lib.w4a16_gemm_host_batch_async.argtypes = [ctypes.POINTER(GemmItem), ctypes.c_int, _P, _P, _SZ, _P, _P, _SZ, _P,
+                                             _SZ, _P]
 _lib.w4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
 _lib.w4_status_string.argtypes = [ctypes.c_int]
 _lib.w4_status_string.restype = ctypes.c_char_p
 _lib.w4_last_error.restype = ctypes.c_char_p
 for _f in ("w4_quantize", "w4_quantize_symmetric", "w4_awq_search", "w4_quantize_outliers", "w4a16_gemm_outliers",
            "w4_quantize_gptq",
-           "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_host_async", "w4a16_gemm_decode_static",
-           "w4_device_error"):
+           "w4_pack", "w4a16_gemm", "w4a16_gemm_host", "w4a16_gemm_host_async", "w4a16_gemm_host_batch_async",
+           "w4a16_gemm_decode_static", "w4_device_error"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -185,6 +196,40 @@ def w4a16_gemm_host(X_host: torch.Tensor, X_dev: torch.Tensor, packed, scales, z
     _check(fn(_ptr(X_host), _ptr(X_dev), _DT[X_host.dtype], M, N, K, group, _ptr(packed), _ptr(scales), _ptr(zeros),
               _ptr(awq_s), _ptr(Y_host), _ptr(Y_dev), _DT[Y_host.dtype], _ptr(ws), 0 if ws is None else ws.numel(),
               _stream(stream)), "w4a16_gemm_host" if wait else "w4a16_gemm_host_async")
+    return Y_host
+
+
+def gemm_batch(items) -> ctypes.Array:
+    """The w4_gemm_item array for w4a16_gemm_host_batch: one entry per matmul, each a dict
+    with M, N, K, packed, scales, zeros, x_offset and y_offset (bytes into the staging
+    buffers), and optionally awq_s, group (128), x_dtype (torch.bfloat16) and y_dtype
+    (torch.float32).  Build it once and reuse it while the weights stay in place."""
+    arr = (GemmItem * len(items))()
+    for a, it in zip(arr, items):
+        a.M, a.N, a.K = it["M"], it["N"], it["K"]
+        a.group = it.get("group", GROUP)
+        a.x_dtype = _DT[it.get("x_dtype", torch.bfloat16)]
+        a.y_dtype = _DT[it.get("y_dtype", torch.float32)]
+        a.packed, a.scales, a.zeros = it["packed"].data_ptr(), it["scales"].data_ptr(), it["zeros"].data_ptr()
+        a.awq_s = it["awq_s"].data_ptr() if it.get("awq_s") is not None else None
+        a.x_offset, a.y_offset = it["x_offset"], it["y_offset"]
+    return arr
+
+
+def w4a16_gemm_host_batch(batch: ctypes.Array, X_host: torch.Tensor, X_dev: torch.Tensor, Y_host: torch.Tensor,
+                          Y_dev: torch.Tensor, ws=None, stream=None, wait: bool = True):
+    """Independent matmuls with pinned host activations and outputs in one call
+    (w4a16_gemm_host_batch_async): one copy of X_host into X_dev, the matmuls of `batch`
+    (from gemm_batch) in order, one copy of Y_dev into Y_host.  The staging buffers are
+    byte views (any dtype); with wait=False Y_host is valid after the caller
+    synchronizes the stream."""
+    xb, yb = X_host.numel() * X_host.element_size(), Y_host.numel() * Y_host.element_size()
+    assert X_dev.numel() * X_dev.element_size() >= xb and Y_dev.numel() * Y_dev.element_size() >= yb
+    _check(_lib.w4a16_gemm_host_batch_async(batch, len(batch), _ptr(X_host), _ptr(X_dev), xb, _ptr(Y_host),
+                                            _ptr(Y_dev), yb, _ptr(ws), 0 if ws is None else ws.numel(),
+                                            _stream(stream)), "w4a16_gemm_host_batch_async")
+    if wait:
+        (stream if stream is not None else torch.cuda.current_stream()).synchronize()
     return Y_host
 
 
