@@ -19,9 +19,12 @@
 //               6-22% and slow plain weights by 9-15%, so plain keeps 4).
 //   warp 1      one thread issues tcgen05.mma (A from TMEM, B = X from shared
 //               memory, fp32 accumulator in TMEM) and tcgen05.commit.
-//   warps 4..7  epilogue: tcgen05.ld of the accumulator, fp32 or bf16 stores
-//   (..11)      (each warp store covers 32 consecutive output channels).
+//   warps 4..7  epilogue: tcgen05.ld of the accumulator; 32 x 32 chunks staged
+//   (..11)      in the idle X ring and written by TMA stores (per-thread stores
+//               where Y's rows are not 16-byte multiples, and for split-K).
 // TMEM columns: [0, BN) accumulator, then NS stages of 32 columns of A.
+// Output tiles that leave a last wave at most half full are cut along K into
+// pieces (tail mode, see TcParams), summed by tail_reduce_kernel.
 // All waits are bounded (see common.cuh).  No TMA multicast anywhere.
 #include "common.cuh"
 
